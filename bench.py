@@ -1,0 +1,423 @@
+"""Benchmark of the NF4 / double-quant / QLoRA-linear hot path on B200.
+
+One step = one pass of the whole path over the LLaMA-7B-shaped layer set
+(q,k,v,o 4096x4096; gate,up 11008x4096; down 4096x11008; 2048 tokens, r=64,
+alpha=16): for every matrix, quantize + double-quantize the bf16 weight,
+dequantize it to bf16, QLoRA forward (Y, T) and backward (dX, dA, dB).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  `value` = fwd+bwd algorithmic TFLOP/s of the
+whole step (quantize and dequantize time included in the denominator),
+summed over ranks; components report GB/s of quantize / dequantize / decode
+GEMV and TFLOP/s of forward / backward separately.  The step's working set
+(~1.3 GB) is far larger than the 126 MB L2, so no flush is needed between
+steps; the decode component flushes L2 between calls.  N > 1 runs
+independent replicas (weak scaling, no collective on the data path).
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_nf4_quantized_12_b200 import workloads  # noqa: E402
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+# ------------------------------------------------------------------ algorithmic work
+def quant_bytes(N, K):
+    numel = N * K
+    nb = (numel + 63) // 64
+    return 2 * numel + (numel + 1) // 2 + nb + 4 * ((nb + 255) // 256)
+
+
+def fwd_flops(M, N, K, r):
+    return 2 * M * N * K + 2 * M * r * (K + N)
+
+
+def bwd_flops(M, N, K, r):
+    return 2 * M * N * K + 4 * M * N * r + 4 * M * K * r
+
+
+def decode_bytes(M, N, K, r):
+    numel = N * K
+    nb = (numel + 63) // 64
+    return (numel + 1) // 2 + nb + 4 * ((nb + 255) // 256) + 2 * M * K + 2 * M * N + 2 * r * (K + N)
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.QUERY,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ our arm
+class Step:
+    """All buffers of one step over the 7B layer set, resident on the GPU."""
+
+    def __init__(self, device, wl, host_copy=False):
+        from bit_nf4_quantized_12_b200 import binding
+        self.b = binding
+        self.wl = wl
+        self.dev = device
+        self.mats = []
+        M, r = wl.tokens, wl.r
+        for idx, (name, N, K) in enumerate(wl.mats):
+            seed = workloads.matrix_seed(wl.name, 0, idx)
+            d = dict(name=name, N=N, K=K)
+            d["W"] = workloads.weight(N, K, wl.w_std, seed=seed, device=device)
+            d.update(workloads.layer_inputs(M, N, K, r, seed=seed, device=device))
+            d["qw"] = binding.empty_quantized(N, K, device)
+            d["Wd"] = torch.empty(N, K, dtype=torch.bfloat16, device=device)
+            d["Y"] = torch.empty(M, N, dtype=torch.bfloat16, device=device)
+            d["T"] = torch.empty(M, r, dtype=torch.bfloat16, device=device)
+            d["dX"] = torch.empty(M, K, dtype=torch.bfloat16, device=device)
+            d["dA"] = torch.empty(K, r, dtype=torch.float32, device=device)
+            d["dB"] = torch.empty(r, N, dtype=torch.float32, device=device)
+            d["ws"] = binding.workspace(M, N, K, r, device)
+            if host_copy:
+                d["host"] = {k: d[k].cpu().pin_memory() for k in ("W", "X", "dY", "A", "B")}
+                d["host_out"] = {k: torch.empty(d[k].shape, dtype=d[k].dtype).pin_memory() for k in ("dA", "dB")}
+            self.mats.append(d)
+        self.launches_per_step = 7 * (1 + 1 + 2 + 4)
+
+    def run(self, events=None):
+        b, wl = self.b, self.wl
+        for d in self.mats:
+            if events is not None:
+                events["q"][0].append(_ev())
+            b.quantize(d["W"], out=d["qw"])
+            if events is not None:
+                events["q"][1].append(_ev())
+                events["dq"][0].append(_ev())
+            b.dequant(d["qw"], out=d["Wd"])
+            if events is not None:
+                events["dq"][1].append(_ev())
+                events["fwd"][0].append(_ev())
+            b.linear_fwd(d["X"], d["qw"], d["A"], d["B"], wl.s, ws=d["ws"], Y=d["Y"], T=d["T"])
+            if events is not None:
+                events["fwd"][1].append(_ev())
+                events["bwd"][0].append(_ev())
+            b.linear_bwd(d["dY"], d["X"], d["qw"], d["A"], d["B"], wl.s, T=d["T"], ws=d["ws"], dX=d["dX"],
+                         dA=d["dA"], dB=d["dB"])
+            if events is not None:
+                events["bwd"][1].append(_ev())
+
+    def run_e2e(self):
+        """Same step through the public API with host buffers: H2D inputs,
+        compute, D2H of the LoRA gradients."""
+        for d in self.mats:
+            for k, h in d["host"].items():
+                d[k].copy_(h, non_blocking=True)
+        self.run()
+        for d in self.mats:
+            for k, h in d["host_out"].items():
+                h.copy_(d[k], non_blocking=True)
+
+    def e2e_bytes(self):
+        h2d = sum(t.numel() * t.element_size() for d in self.mats for t in d["host"].values())
+        d2h = sum(t.numel() * t.element_size() for d in self.mats for t in d["host_out"].values())
+        return h2d, d2h
+
+
+def _ev():
+    e = torch.cuda.Event(enable_timing=True)
+    e.record()
+    return e
+
+
+def _pair_ms(starts, ends):
+    return [s.elapsed_time(e) for s, e in zip(starts, ends)]
+
+
+def decode_component(device, peaks):
+    """Decode GEMV (fused dequant, r=16) on 28672x8192 and 8192x28672 at
+    M in {1,4,16}: each call timed alone, L2 flushed before it."""
+    from bit_nf4_quantized_12_b200 import binding
+    wl = workloads.WORKLOADS["decode"]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    res = {}
+    for (name, N, K) in wl.mats:
+        W = workloads.weight(N, K, wl.w_std, seed=0, device=device)
+        qw = binding.quantize(W)
+        del W
+        for M in wl.decode_m:
+            io = workloads.layer_inputs(M, N, K, wl.r, seed=1, device=device)
+            ws = binding.workspace(M, N, K, wl.r, device)
+            Y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
+            T = torch.empty(M, wl.r, dtype=torch.bfloat16, device=device)
+            times = []
+            for it in range(13):
+                flush.zero_()
+                s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                s.record()
+                binding.linear_fwd(io["X"], qw, io["A"], io["B"], wl.s, ws=ws, Y=Y, T=T)
+                e.record()
+                torch.cuda.synchronize()
+                if it >= 3:
+                    times.append(s.elapsed_time(e))
+            ms = statistics.median(times)
+            gbs = decode_bytes(M, N, K, wl.r) / (ms * 1e-3) / 1e9
+            res[f"{N}x{K}_m{M}"] = {"us": round(ms * 1e3, 2), "GB/s": round(gbs, 1),
+                                     "frac": round(gbs / peaks["hbm_gbs"], 3)}
+        del qw
+    return res
+
+
+# ------------------------------------------------------------------ oracle arm
+def oracle_sample_step(wl, frac_rows, seed=0):
+    """The oracle over a row sample of every matrix of the step: quantize and
+    dequantize the sampled W rows (group-aligned), forward for those output
+    features, backward restricted to them.  Returns (flops done, seconds)."""
+    import oracle
+    M, r, s = wl.tokens, wl.r, wl.s
+    flops = 0.0
+    secs = 0.0
+    for idx, (name, N, K) in enumerate(wl.mats):
+        mseed = workloads.matrix_seed(wl.name, 0, idx)
+        n_rows = max(16, int(N * frac_rows) // 16 * 16)
+        n0 = (seed * 7919 + idx * 104729) % (N - n_rows + 1)
+        W = workloads.weight(N, K, wl.w_std, seed=mseed)
+        io = workloads.layer_inputs(M, N, K, r, seed=mseed)
+        Wb = workloads.bits(W[n0:n0 + n_rows])
+        X, A = workloads.bits(io["X"]), workloads.bits(io["A"])
+        Bs = workloads.bits(io["B"][:, n0:n0 + n_rows].contiguous())
+        dYs = workloads.bits(io["dY"][:, n0:n0 + n_rows].contiguous())
+        t0 = time.perf_counter()
+        packed, c1q, c2, _ = oracle.quantize(Wb)
+        Wd = oracle.dequant(packed, c1q, c2, Wb.size).reshape(n_rows, K)
+        Y, T = oracle.qlora_fwd(X, Wd, A, Bs, s)
+        oracle.qlora_bwd(dYs, X, Wd, A, Bs, s, T)
+        secs += time.perf_counter() - t0
+        flops += fwd_flops(M, n_rows, K, r) + bwd_flops(M, n_rows, K, r)
+    return flops, secs
+
+
+def run_reference(args, wl, rank, world):
+    if rank != 0:
+        return
+    frac = 1.0 / 256
+    for _ in range(args.warmup):
+        oracle_sample_step(wl, frac)
+    flops, secs = 0.0, 0.0
+    for k in range(args.steps):
+        f, s_ = oracle_sample_step(wl, frac, seed=k + 1)
+        flops += f
+        secs += s_
+    value = flops / secs / 1e12
+    sample = (f"oracle (plain C quantize/dequant + float64 numpy GEMM) on 1/256 of the output features of each of "
+              f"the 7 matrices per step (group-aligned row slice), all {wl.tokens} tokens")
+    cores = torch.get_num_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_dict(wl, 1),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+METRIC = "NF4 dequant/quant GB/s and qlora_linear TFLOP/s, % of B200 roofline"
+
+
+def config_dict(wl, n):
+    return {"workload": "llama7b_layer_set: q,k,v,o 4096x4096; gate,up 11008x4096; down 4096x11008; "
+                        "quantize+dq, dequant, qlora fwd+bwd at 2048 tokens, r=64, alpha=16",
+            "global_batch": wl.tokens * n, "seq_len": 512, "rank": wl.r, "alpha": wl.alpha,
+            "parallelism": f"replicas{n}" if n > 1 else "single",
+            "l2": "step working set ~1.3 GB > 126 MB L2; no flush between steps"}
+
+
+# ------------------------------------------------------------------ main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-components", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    wl = workloads.WORKLOADS["llama7b"]
+
+    if args.impl == "reference":
+        run_reference(args, wl, rank, world)
+        return
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+        pg = dist
+    peaks, peak_kind = load_peaks()
+
+    step = Step(device, wl, host_copy=True)
+    step_launches = step.launches_per_step
+    for _ in range(max(3, args.warmup)):
+        step.run()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K device-resident steps
+    ev = {k: ([], []) for k in ("q", "dq", "fwd", "bwd")}
+    clocks = ClockSampler(local)
+    clocks.start()
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    t0 = _ev()
+    for _ in range(args.steps):
+        step.run(events=ev)
+    t1 = _ev()
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1)
+    if pg:
+        t = torch.tensor([ms], device=device)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms = float(t.item())
+
+    M, r = wl.tokens, wl.r
+    step_flops = sum(fwd_flops(M, N, K, r) + bwd_flops(M, N, K, r) for _, N, K in wl.mats)
+    value = world * step_flops * args.steps / (ms * 1e-3) / 1e12
+
+    comp = {}
+    qb = sum(quant_bytes(N, K) for _, N, K in wl.mats) * args.steps
+    q_ms = sum(_pair_ms(*ev["q"]))
+    dq_ms = sum(_pair_ms(*ev["dq"]))
+    f_ms = sum(_pair_ms(*ev["fwd"]))
+    b_ms = sum(_pair_ms(*ev["bwd"]))
+    fl_f = sum(fwd_flops(M, N, K, r) for _, N, K in wl.mats) * args.steps
+    fl_b = sum(bwd_flops(M, N, K, r) for _, N, K in wl.mats) * args.steps
+    comp["quantize"] = {"GB/s": qb / (q_ms * 1e-3) / 1e9, "ms_per_step": q_ms / args.steps}
+    comp["dequant"] = {"GB/s": qb / (dq_ms * 1e-3) / 1e9, "ms_per_step": dq_ms / args.steps}
+    comp["fwd"] = {"TFLOP/s": fl_f / (f_ms * 1e-3) / 1e12, "ms_per_step": f_ms / args.steps}
+    comp["bwd"] = {"TFLOP/s": fl_b / (b_ms * 1e-3) / 1e12, "ms_per_step": b_ms / args.steps}
+    for k in ("quantize", "dequant"):
+        comp[k]["frac"] = comp[k]["GB/s"] / peaks["hbm_gbs"]
+    for k in ("fwd", "bwd"):
+        comp[k]["frac"] = comp[k]["TFLOP/s"] / peaks["bf16_tflops_sustained"]
+
+    # dominant work: the qlora_linear calls (forward + backward)
+    gemm_tflops = (fl_f + fl_b) / ((f_ms + b_ms) * 1e-3) / 1e12
+    roofline = {"kernel": "qlora_linear_fwd+bwd calls (nf4_gemm_kernel + skinny_gemm_kernel)",
+                "bound": "tensor", "achieved": gemm_tflops, "peak": peaks["bf16_tflops_sustained"],
+                "unit": "TFLOP/s", "frac": gemm_tflops / peaks["bf16_tflops_sustained"],
+                "peak_kind": f"{peak_kind} bf16_tflops_sustained", "traffic": None}
+
+    # ---- end to end through the public API with host buffers
+    h2d, d2h = step.e2e_bytes()
+    for _ in range(2):
+        step.run_e2e()
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    e0 = _ev()
+    for _ in range(args.steps):
+        step.run_e2e()
+    e1 = _ev()
+    torch.cuda.synchronize()
+    ems = e0.elapsed_time(e1)
+    if pg:
+        t = torch.tensor([ems], device=device)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ems = float(t.item())
+    e2e_value = world * step_flops * args.steps / (ems * 1e-3) / 1e12
+
+    if not args.no_components and rank == 0:
+        del step
+        torch.cuda.empty_cache()
+        comp["decode"] = decode_component(device, peaks)
+
+    cpu = None
+    if rank == 0 and world == 1:
+        flops, secs = oracle_sample_step(wl, 1.0 / 256)
+        cpu = {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": torch.get_num_threads(),
+               "kind": "oracle",
+               "sample": "oracle on 1/256 of the output features of each of the 7 matrices "
+                         "(quantize+dequant of those rows, fwd+bwd restricted to them), all 2048 tokens"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+                "warmup": max(3, args.warmup), "ms_per_step": ms / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": config_dict(wl, world), "roofline": roofline, "components": comp,
+                "cpu_baseline": cpu, "clocks": clk,
+                "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                        "d2h_bytes_per_step": d2h},
+                "gpu_launches": step_launches * args.steps,
+                "peaks": {"kind": peak_kind, "hbm_gbs": peaks["hbm_gbs"],
+                          "bf16_tflops_sustained": peaks["bf16_tflops_sustained"]}}
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,184 @@
+"""Thin Python binding of libqlora_nf4.so (include/qlora_nf4.h).
+
+Argument marshalling only: torch tensors supply device memory and the current
+CUDA stream; every step of the computation runs in the library's kernels.
+There is no fallback: a missing library or a CPU tensor raises.
+"""
+import ctypes
+import os
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqlora_nf4.so")
+
+NF4_OK = 0
+STATUS_NONFINITE = 1
+STATUS_TIMEOUT = 2
+
+_lib = None
+
+
+class NF4Error(RuntimeError):
+    pass
+
+
+class NF4Weight(ctypes.Structure):
+    _fields_ = [("packed", ctypes.c_void_p), ("c1q", ctypes.c_void_p), ("c2", ctypes.c_void_p),
+                ("rows", ctypes.c_int64), ("cols", ctypes.c_int64)]
+
+
+# (name, restype, argtypes) for every symbol of include/qlora_nf4.h
+_P, _I64, _I32, _F, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "nf4_build_codebook": (ctypes.c_int, [_P, _P]),
+    "nf4_sizes": (ctypes.c_int, [_I64, _P, _P, _P]),
+    "nf4_quantize_dq": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _P, _P]),
+    "nf4_dequant_bf16": (ctypes.c_int, [NF4Weight, _P, _P]),
+    "qlora_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I32]),
+    "qlora_linear_fwd": (ctypes.c_int, [_P, _I64, NF4Weight, _P, _P, _I32, _F, _P, _P, _P, _SZ, _P]),
+    "qlora_linear_bwd": (ctypes.c_int, [_P, _P, _I64, NF4Weight, _P, _P, _I32, _F, _P, _P, _P, _P, _P,
+                                        _SZ, _P]),
+    "nf4_status_str": (ctypes.c_char_p, [ctypes.c_int]),
+}
+
+
+def lib():
+    """Load the library (raises NF4Error when it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise NF4Error(f"{LIB_PATH} not found: run `python -m bit_nf4_quantized_12_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(code):
+    if code != NF4_OK:
+        raise NF4Error(lib().nf4_status_str(code).decode())
+
+
+def _dev(t, dtype, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise NF4Error(f"{name} must be a CUDA tensor (no CPU path exists)")
+    if t.dtype != dtype:
+        raise NF4Error(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise NF4Error(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+# ---------------------------------------------------------------- format
+def build_codebook():
+    codes = np.zeros(16, np.float32)
+    thr = np.zeros(15, np.float32)
+    _check(lib().nf4_build_codebook(codes.ctypes.data_as(_P), thr.ctypes.data_as(_P)))
+    return codes, thr
+
+
+def sizes(numel):
+    pb, nb, ng = ctypes.c_size_t(), ctypes.c_int64(), ctypes.c_int64()
+    _check(lib().nf4_sizes(int(numel), ctypes.byref(pb), ctypes.byref(nb), ctypes.byref(ng)))
+    return pb.value, nb.value, ng.value
+
+
+@dataclass
+class QuantizedWeight:
+    packed: torch.Tensor   # uint8 [ceil(numel/2)]
+    c1q: torch.Tensor      # uint8 [nblocks]
+    c2: torch.Tensor       # float32 [ngroups]
+    rows: int
+    cols: int
+
+    def abi(self):
+        return NF4Weight(self.packed.data_ptr(), self.c1q.data_ptr(), self.c2.data_ptr(), self.rows, self.cols)
+
+
+def empty_quantized(rows, cols, device):
+    pb, nb, ng = sizes(rows * cols)
+    # packed is padded to 16 bytes so its size is a multiple of the vector width
+    packed = torch.zeros(((pb + 15) // 16) * 16, dtype=torch.uint8, device=device)[:pb]
+    return QuantizedWeight(packed, torch.zeros(nb, dtype=torch.uint8, device=device),
+                           torch.zeros(ng, dtype=torch.float32, device=device), rows, cols)
+
+
+def quantize(W, out: QuantizedWeight = None, status: torch.Tensor = None):
+    """NF4 + double quantization of a bf16 CUDA tensor [rows, cols]."""
+    rows, cols = W.shape
+    if out is None:
+        out = empty_quantized(rows, cols, W.device)
+    _check(lib().nf4_quantize_dq(_dev(W, torch.bfloat16, "W"), rows, cols, ctypes.c_void_p(out.packed.data_ptr()),
+                                 ctypes.c_void_p(out.c1q.data_ptr()), ctypes.c_void_p(out.c2.data_ptr()),
+                                 None if status is None else _dev(status, torch.int32, "status"), _stream()))
+    return out
+
+
+def dequant(qw: QuantizedWeight, out: torch.Tensor = None):
+    if out is None:
+        out = torch.empty(qw.rows, qw.cols, dtype=torch.bfloat16, device=qw.packed.device)
+    _check(lib().nf4_dequant_bf16(qw.abi(), _dev(out, torch.bfloat16, "out"), _stream()))
+    return out
+
+
+# ---------------------------------------------------------------- linear layer
+def workspace_bytes(M, N, K, r):
+    return int(lib().qlora_workspace_bytes(int(M), int(N), int(K), int(r)))
+
+
+def workspace(M, N, K, r, device):
+    return torch.zeros(workspace_bytes(M, N, K, r), dtype=torch.uint8, device=device)
+
+
+def linear_fwd(X, qw: QuantizedWeight, A, B, s, ws=None, Y=None, T=None, want_T=True):
+    """Y = X Wd^T + s (X A) B; returns (Y, T)."""
+    M, K = X.shape
+    r = A.shape[1]
+    if ws is None:
+        ws = workspace(M, qw.rows, K, r, X.device)
+    if Y is None:
+        Y = torch.empty(M, qw.rows, dtype=torch.bfloat16, device=X.device)
+    if T is None and want_T:
+        T = torch.empty(M, r, dtype=torch.bfloat16, device=X.device)
+    _check(lib().qlora_linear_fwd(_dev(X, torch.bfloat16, "X"), M, qw.abi(), _dev(A, torch.bfloat16, "A"),
+                                  _dev(B, torch.bfloat16, "B"), r, float(s), _dev(Y, torch.bfloat16, "Y"),
+                                  None if T is None else _dev(T, torch.bfloat16, "T"),
+                                  _dev(ws, torch.uint8, "ws"), ws.numel(), _stream()))
+    return Y, T
+
+
+def linear_bwd(dY, X, qw: QuantizedWeight, A, B, s, T=None, ws=None, dX=None, dA=None, dB=None):
+    """Returns (dX bf16 [M,K], dA fp32 [K,r], dB fp32 [r,N])."""
+    M, K = X.shape
+    r = A.shape[1]
+    N = qw.rows
+    if ws is None:
+        ws = workspace(M, N, K, r, X.device)
+    if dX is None:
+        dX = torch.empty(M, K, dtype=torch.bfloat16, device=X.device)
+    if dA is None:
+        dA = torch.empty(K, r, dtype=torch.float32, device=X.device)
+    if dB is None:
+        dB = torch.empty(r, N, dtype=torch.float32, device=X.device)
+    _check(lib().qlora_linear_bwd(_dev(dY, torch.bfloat16, "dY"), _dev(X, torch.bfloat16, "X"), M, qw.abi(),
+                                  _dev(A, torch.bfloat16, "A"), _dev(B, torch.bfloat16, "B"), r, float(s),
+                                  None if T is None else _dev(T, torch.bfloat16, "T"),
+                                  _dev(dX, torch.bfloat16, "dX"), _dev(dA, torch.float32, "dA"),
+                                  _dev(dB, torch.float32, "dB"), _dev(ws, torch.uint8, "ws"), ws.numel(),
+                                  _stream()))
+    return dX, dA, dB
+
+
+def workspace_status(ws):
+    """The status word a linear call leaves in its workspace (read after sync)."""
+    return int(ws[:4].view(torch.int32).item())

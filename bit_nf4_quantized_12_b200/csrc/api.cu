@@ -1,0 +1,223 @@
+// api.cu -- the extern "C" entry points of libqlora_nf4 (include/qlora_nf4.h):
+// argument validation, workspace layout, and the launch sequence of each call.
+#include <cstdint>
+#include <cstring>
+#include <cuda_runtime.h>
+
+#include "../../include/qlora_nf4.h"
+#include "format.h"
+#include "kernels.h"
+
+namespace {
+
+using namespace nf4;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int device_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) return 148;
+  return sms;
+}
+
+int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
+
+// Workspace: [status word + split counters | low-rank hi/lo | T scratch | split partials]
+struct WsLayout {
+  size_t counters = 16;      // 1023 counters after the 16-byte status slot
+  size_t hilo = 0, t_scratch = 0, partial = 0, total = 0;
+  size_t partial_bytes = 0;
+};
+constexpr size_t kHeaderBytes = 4096;
+
+WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int r, int sms) {
+  WsLayout L;
+  const int64_t rp = round_up(r, 64);
+  size_t off = kHeaderBytes;
+  L.hilo = off;
+  off += size_t(round_up(M * 2 * rp * 2, 256));
+  L.t_scratch = off;
+  off += size_t(round_up(M * r * 2, 256));
+  L.partial = off;
+  size_t pb = 0;
+  auto upd = [&](size_t b) { if (b > pb) pb = b; };
+  upd(plan_nf4_gemm(0, M, N, K, r, sms).partial_bytes);
+  upd(plan_nf4_gemm(1, M, N, K, r, sms).partial_bytes);
+  for (int kind = 0; kind < 4; ++kind) upd(plan_skinny(kind, M, N, K, r, sms).partial_bytes);
+  L.partial_bytes = pb;
+  off += size_t(round_up(int64_t(pb), 256));
+  L.total = off;
+  return L;
+}
+
+nf4_status check_linear_shapes(int64_t M, const nf4_weight& w, int32_t r) {
+  if (M < 1 || w.rows < 1 || w.cols < 1 || r < 1 || r > 256) return NF4_ERR_INVALID_ARG;
+  if (!w.packed || !w.c1q || !w.c2) return NF4_ERR_INVALID_ARG;
+  if (w.cols % 64 != 0 || w.rows % 8 != 0 || r % 8 != 0) return NF4_ERR_UNSUPPORTED;
+  if (w.rows > (int64_t(1) << 31) || w.cols > (int64_t(1) << 31) || M > (int64_t(1) << 31))
+    return NF4_ERR_UNSUPPORTED;
+  if (!aligned16(w.packed)) return NF4_ERR_MISALIGNED;
+  return NF4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+nf4_status nf4_build_codebook(float codes[16], float thresholds[15]) {
+  const Codebook& cb = host_codebook();
+  if (codes) memcpy(codes, cb.code, sizeof(cb.code));
+  if (thresholds) memcpy(thresholds, cb.thr, sizeof(cb.thr));
+  return NF4_OK;
+}
+
+nf4_status nf4_sizes(int64_t numel, size_t* packed_bytes, int64_t* nblocks, int64_t* ngroups) {
+  if (numel < 1) return NF4_ERR_INVALID_ARG;
+  if (packed_bytes) *packed_bytes = size_t(packed_bytes_of(numel));
+  if (nblocks) *nblocks = nblocks_of(numel);
+  if (ngroups) *ngroups = ngroups_of(numel);
+  return NF4_OK;
+}
+
+nf4_status nf4_quantize_dq(const uint16_t* W, int64_t rows, int64_t cols, uint8_t* packed, uint8_t* c1q, float* c2,
+                           int32_t* d_status, void* stream) {
+  if (!W || !packed || !c1q || !c2 || rows < 1 || cols < 1) return NF4_ERR_INVALID_ARG;
+  if (rows > (int64_t(1) << 40) / cols) return NF4_ERR_UNSUPPORTED;
+  if (!aligned16(W) || !aligned16(packed)) return NF4_ERR_MISALIGNED;
+  if (!quantize_table_ok()) return NF4_ERR_UNSUPPORTED;
+  cudaError_t e = launch_quantize(W, rows * cols, packed, c1q, c2, reinterpret_cast<uint32_t*>(d_status),
+                                  device_sms(), static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NF4_OK : NF4_ERR_CUDA;
+}
+
+nf4_status nf4_dequant_bf16(nf4_weight w, uint16_t* out, void* stream) {
+  if (!w.packed || !w.c1q || !w.c2 || !out || w.rows < 1 || w.cols < 1) return NF4_ERR_INVALID_ARG;
+  if (w.rows > (int64_t(1) << 40) / w.cols) return NF4_ERR_UNSUPPORTED;
+  if (!aligned16(w.packed) || !aligned16(out)) return NF4_ERR_MISALIGNED;
+  cudaError_t e = launch_dequant(w.packed, w.c1q, w.c2, w.rows * w.cols, out, device_sms(),
+                                 static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NF4_OK : NF4_ERR_CUDA;
+}
+
+size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t r) {
+  if (M < 1 || N < 1 || K < 1 || r < 1 || r > 256) return 0;
+  return ws_layout(M, N, K, r, device_sms()).total;
+}
+
+nf4_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight w, const uint16_t* A, const uint16_t* B,
+                            int32_t r, float s, uint16_t* Y, uint16_t* T_out, void* ws, size_t ws_bytes,
+                            void* stream) {
+  nf4_status st = check_linear_shapes(M, w, r);
+  if (st != NF4_OK) return st;
+  if (!X || !A || !B || !Y) return NF4_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(Y) || (T_out && !aligned16(T_out)))
+    return NF4_ERR_MISALIGNED;
+  const int sms = device_sms();
+  const int64_t N = w.rows, K = w.cols;
+  const WsLayout L = ws_layout(M, N, K, r, sms);
+  if (!ws || ws_bytes < L.total) return NF4_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return NF4_ERR_MISALIGNED;
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  uint32_t* status = reinterpret_cast<uint32_t*>(wsb);
+  uint32_t* counters = reinterpret_cast<uint32_t*>(wsb + L.counters);
+  uint16_t* hilo = reinterpret_cast<uint16_t*>(wsb + L.hilo);
+  uint16_t* t_dst = T_out ? T_out : reinterpret_cast<uint16_t*>(wsb + L.t_scratch);
+  float* partial = reinterpret_cast<float*>(wsb + L.partial);
+  const int rp = int(round_up(r, 64));
+
+  if (cudaMemsetAsync(ws, 0, kHeaderBytes, strm) != cudaSuccess) return NF4_ERR_CUDA;
+
+  SkinnyArgs sa{};
+  sa.M = M; sa.N = N; sa.K = K; sa.r = r; sa.rp = rp; sa.s = s;
+  sa.X = X; sa.A = A; sa.B = B;
+  sa.T_out = t_dst; sa.hilo_out = hilo;
+  sa.partial = partial; sa.counters = counters; sa.status = status;
+  if (launch_skinny(plan_skinny(kSkinnyT, M, N, K, r, sms), sa, strm) != cudaSuccess) return NF4_ERR_CUDA;
+
+  Nf4GemmArgs ga{};
+  ga.M = M; ga.N = N; ga.K = K; ga.r = r; ga.rp = rp;
+  ga.packed = w.packed; ga.c1q = w.c1q; ga.c2 = w.c2;
+  ga.act = X; ga.lora_w = B; ga.lora_act = hilo; ga.out = Y;
+  ga.partial = partial; ga.counters = counters; ga.status = status;
+  if (launch_nf4_gemm(plan_nf4_gemm(0, M, N, K, r, sms), ga, strm) != cudaSuccess) return NF4_ERR_CUDA;
+  return NF4_OK;
+}
+
+nf4_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, nf4_weight w, const uint16_t* A,
+                            const uint16_t* B, int32_t r, float s, const uint16_t* T, uint16_t* dX, float* dA,
+                            float* dB, void* ws, size_t ws_bytes, void* stream) {
+  nf4_status st = check_linear_shapes(M, w, r);
+  if (st != NF4_OK) return st;
+  if (!dY || !X || !A || !B || !dX || !dA || !dB) return NF4_ERR_INVALID_ARG;
+  if (!aligned16(dY) || !aligned16(X) || !aligned16(A) || !aligned16(B) || !aligned16(dX) || !aligned16(dA) ||
+      !aligned16(dB) || (T && !aligned16(T)))
+    return NF4_ERR_MISALIGNED;
+  const int sms = device_sms();
+  const int64_t N = w.rows, K = w.cols;
+  const WsLayout L = ws_layout(M, N, K, r, sms);
+  if (!ws || ws_bytes < L.total) return NF4_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return NF4_ERR_MISALIGNED;
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  uint32_t* status = reinterpret_cast<uint32_t*>(wsb);
+  uint32_t* counters = reinterpret_cast<uint32_t*>(wsb + L.counters);
+  uint16_t* hilo = reinterpret_cast<uint16_t*>(wsb + L.hilo);
+  float* partial = reinterpret_cast<float*>(wsb + L.partial);
+  const int rp = int(round_up(r, 64));
+
+  if (cudaMemsetAsync(ws, 0, kHeaderBytes, strm) != cudaSuccess) return NF4_ERR_CUDA;
+
+  SkinnyArgs sa{};
+  sa.M = M; sa.N = N; sa.K = K; sa.r = r; sa.rp = rp; sa.s = s;
+  sa.X = X; sa.dY = dY; sa.A = A; sa.B = B;
+  sa.partial = partial; sa.counters = counters; sa.status = status;
+
+  const uint16_t* Tin = T;
+  if (!Tin) {  // recompute T = bf16(X A) into scratch (the hi/lo output is overwritten by G below)
+    uint16_t* tw = reinterpret_cast<uint16_t*>(wsb + L.t_scratch);
+    sa.T_out = tw;
+    sa.hilo_out = hilo;
+    if (launch_skinny(plan_skinny(kSkinnyT, M, N, K, r, sms), sa, strm) != cudaSuccess) return NF4_ERR_CUDA;
+    Tin = tw;
+  }
+  // G = s dY B^T as a bf16 hi/lo pair
+  sa.T_out = nullptr;
+  sa.hilo_out = hilo;
+  if (launch_skinny(plan_skinny(kSkinnyG, M, N, K, r, sms), sa, strm) != cudaSuccess) return NF4_ERR_CUDA;
+
+  // dX = dY Wd + G A^T
+  Nf4GemmArgs ga{};
+  ga.M = M; ga.N = N; ga.K = K; ga.r = r; ga.rp = rp;
+  ga.packed = w.packed; ga.c1q = w.c1q; ga.c2 = w.c2;
+  ga.act = dY; ga.lora_w = A; ga.lora_act = hilo; ga.out = dX;
+  ga.partial = partial; ga.counters = counters; ga.status = status;
+  if (launch_nf4_gemm(plan_nf4_gemm(1, M, N, K, r, sms), ga, strm) != cudaSuccess) return NF4_ERR_CUDA;
+
+  // dA = X^T G  (G hi + G lo)
+  sa.hilo_in = hilo;
+  sa.f32_out = dA;
+  if (launch_skinny(plan_skinny(kSkinnyDA, M, N, K, r, sms), sa, strm) != cudaSuccess) return NF4_ERR_CUDA;
+  // dB = s T^T dY
+  sa.T = Tin;
+  sa.f32_out = dB;
+  if (launch_skinny(plan_skinny(kSkinnyDB, M, N, K, r, sms), sa, strm) != cudaSuccess) return NF4_ERR_CUDA;
+  return NF4_OK;
+}
+
+const char* nf4_status_str(nf4_status status) {
+  switch (status) {
+    case NF4_OK: return "NF4_OK";
+    case NF4_ERR_INVALID_ARG: return "NF4_ERR_INVALID_ARG";
+    case NF4_ERR_MISALIGNED: return "NF4_ERR_MISALIGNED";
+    case NF4_ERR_UNSUPPORTED: return "NF4_ERR_UNSUPPORTED";
+    case NF4_ERR_WORKSPACE: return "NF4_ERR_WORKSPACE";
+    case NF4_ERR_NONFINITE: return "NF4_ERR_NONFINITE";
+    case NF4_ERR_CUDA: return "NF4_ERR_CUDA";
+  }
+  return "NF4_ERR_UNKNOWN";
+}
+
+}  // extern "C"

@@ -1,0 +1,784 @@
+// gemm.cu -- tensor-core kernels of the QLoRA linear layer on sm_100a.
+//
+// The layer ("LoRA、Q-LoRA 与 PortLLM" §3.4; "从LoRA到QLoRA" §3.1) is
+//     Y = X Wd^T + s (X A) B,    s = alpha / r,
+// with Wd the frozen NF4 weight dequantized to BF16 on the fly.  Backward
+// passes gradients to X, A and B only:
+//     G = s dY B^T,  dX = dY Wd + G A^T,  dA = X^T G,  dB = s T^T dY,  T = X A.
+//
+// nf4_gemm_kernel: the two products with the frozen weight (Y and dX).  Both
+// are computed transposed, with the W dimension as the 128-row MMA "M" and
+// tokens as the MMA "N", so that the dequantized weight tile is the A operand:
+//   forward : A = Wd[n0:n0+128, k:k+64]  written by the dequant warps straight
+//             into tensor memory (tcgen05.st), one 64-weight block per thread;
+//   backward: A = Wd[n:n+64, k0:k0+128]^T written into shared memory in the
+//             MN-major 128-byte-swizzled layout the MMA reads (the NF4 blocks
+//             run along k, which is the MN dimension there).
+// The activation operand (X or dY) is staged by TMA.  The low-rank term is
+// appended as extra 64-wide reduction steps into the same fp32 accumulator,
+// using a bf16 hi/lo split of s*T (forward) or G (backward) so the low-rank
+// product carries ~16 significant bits.  A fixed split of the reduction with
+// a deterministic last-CTA reduction serves small grids (decode, k/v).
+//
+// skinny_gemm_kernel: the rank-r products T, G, dA, dB (N = r padded to 64),
+// both operands by TMA, split reduction with the same last-CTA scheme.
+//
+// Warp roles (nf4_gemm, 384 threads): warp 0 TMA producer, warp 1 MMA issuer,
+// warp 2 tensor-memory allocator, warps 4-11 two dequant warpgroups that take
+// alternate reduction steps and then run the epilogue.  Every wait is bounded
+// (common.cuh) and reports kStatusTimeout instead of hanging.
+#include <cstdint>
+#include <cstring>
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include "common.cuh"
+#include "kernels.h"
+
+namespace nf4 {
+namespace {
+
+constexpr int kStages = 4;
+constexpr int kGemmThreads = 384;
+constexpr int kSkinnyThreads = 192;
+constexpr int kSkinnyStages = 4;
+
+struct CodeTable {
+  float v[16];
+};
+
+struct Nf4GemmParams {
+  CUtensorMap tm_act;   // X [M,K] / dY [M,N], bf16, box {64, bt}, 128B swizzle
+  CUtensorMap tm_pk;    // packed [N, K/2] bytes; box {32,128} fwd, {64,64} bwd
+  CUtensorMap tm_lact;  // hi/lo [M, 2rp] bf16, box {64, bt}, 128B swizzle
+  CUtensorMap tm_lw;    // backward: A [K, r] bf16, box {64, 128}, 128B swizzle
+  Nf4GemmArgs a;
+  CodeTable code;
+  int bt;
+  int splits;
+  int64_t main_steps;   // total 64-wide steps of the main reduction
+  int lora_steps;
+};
+
+// ---------------------------------------------------------------- dequant
+// 16-entry bf16 table of one block (code[q] * scale1, each an fp32 multiply
+// rounded to bf16) split into low-byte and high-byte planes so that four
+// lookups are a handful of byte permutes.
+struct BlockTable {
+  uint32_t lo[4], hi[4];
+};
+
+__device__ __forceinline__ BlockTable make_table(const CodeTable& code, float s1) {
+  uint32_t pr[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) pr[i] = pack_bf16x2(code.v[2 * i] * s1, code.v[2 * i + 1] * s1);
+  BlockTable t;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    t.lo[k] = prmt(pr[2 * k], pr[2 * k + 1], 0x6420);
+    t.hi[k] = prmt(pr[2 * k], pr[2 * k + 1], 0x7531);
+  }
+  return t;
+}
+
+// Four nibbles (bits 0-15 of s, element j in nibble j) -> two bf16x2 words.
+__device__ __forceinline__ void lookup4(const BlockTable& t, uint32_t s, uint32_t& o01, uint32_t& o23) {
+  const uint32_t sel_a = s;                   // entries 0-7 (bit 3 clear)
+  const uint32_t sel_b = s ^ 0x8888u;         // entries 8-15
+  const uint32_t sel2 = ((s >> 1) & 0x4444u) | 0x3210u;   // pick a or b per byte by bit 3
+  const uint32_t lo = prmt(prmt(t.lo[0], t.lo[1], sel_a), prmt(t.lo[2], t.lo[3], sel_b), sel2);
+  const uint32_t hi = prmt(prmt(t.hi[0], t.hi[1], sel_a), prmt(t.hi[2], t.hi[3], sel_b), sel2);
+  o01 = prmt(lo, hi, 0x5140);
+  o23 = prmt(lo, hi, 0x7362);
+}
+
+// 32 packed bytes (64 weights) -> 32 bf16x2 words in element order.
+__device__ __forceinline__ void dequant64(const BlockTable& t, const uint4& p0, const uint4& p1,
+                                          uint32_t (&o)[32]) {
+  const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    lookup4(t, w[i] & 0xFFFFu, o[4 * i + 0], o[4 * i + 1]);
+    lookup4(t, w[i] >> 16, o[4 * i + 2], o[4 * i + 3]);
+  }
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+__device__ __forceinline__ float block_scale(const Nf4GemmArgs& a, int64_t b) {
+  return e4m3_to_f32(__ldg(a.c1q + b)) * __ldg(a.c2 + (b >> 8));
+}
+
+// ---------------------------------------------------------------- kernel
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+// Wait ignoring the abort flag (used only to drain in-flight copies/MMAs).
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > 100000000ull) break;   // 100 ms
+  }
+}
+
+// Forward tensor-memory layout: accumulator in columns [0, acc), the four
+// 32-column A stages after it.
+__host__ __device__ constexpr int fwd_a_col0(int bt) { return bt <= 128 ? 128 : 256; }
+__host__ __device__ constexpr uint32_t fwd_tmem_cols(int bt) { return bt <= 128 ? 256u : 512u; }
+
+template <bool BWD>
+__global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_constant__ Nf4GemmParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const Nf4GemmArgs& a = P.a;
+  const int bt = P.bt;
+  const uint32_t act_bytes = uint32_t(bt) * 128u;
+  uint8_t* act_s = smem;                                   // kStages x act_bytes
+  uint8_t* pk_s = act_s + kStages * act_bytes;             // kStages x 4096
+  uint8_t* a_s = pk_s + kStages * 4096;                    // backward: kStages x 16384
+  uint64_t* bars = reinterpret_cast<uint64_t*>(a_s + (BWD ? kStages * 16384 : 0));
+  uint64_t* full = bars;
+  uint64_t* afull = bars + kStages;
+  uint64_t* empty = bars + 2 * kStages;
+  uint64_t* accf = bars + 3 * kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_flag = abort_flag + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t tile_w = blockIdx.x, tile_t = blockIdx.y;
+  const int split = blockIdx.z;
+  const int64_t w0 = tile_w * 128;          // forward: first W row; backward: first W column
+  const int64_t m0 = tile_t * bt;
+  const int64_t per = (P.main_steps + P.splits - 1) / P.splits;
+  const int64_t g_begin = split * per;
+  const int64_t g_end = (g_begin + per < P.main_steps) ? g_begin + per : P.main_steps;
+  const int64_t my_main = g_end > g_begin ? g_end - g_begin : 0;
+  const int my_lora = (split == 0) ? P.lora_steps : 0;
+  const int64_t nsteps = my_main + my_lora;
+  const int64_t KB = a.K / kBlock;          // NF4 blocks per W row
+  const uint32_t tmem_cols = BWD ? uint32_t(bt < 32 ? 32 : bt) : fwd_tmem_cols(bt);
+  const uint32_t a_col0 = uint32_t(fwd_a_col0(bt));
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&afull[s], 4);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accf, 1);
+    *abort_flag = 0;
+    *last_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_slot, tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (elect_one()) {
+      tma_prefetch_desc(&P.tm_act);
+      tma_prefetch_desc(&P.tm_pk);
+      tma_prefetch_desc(&P.tm_lact);
+      if (BWD) tma_prefetch_desc(&P.tm_lw);
+      int64_t issued = 0;
+      for (int64_t ks = 0; ks < nsteps; ++ks) {
+        const int s = int(ks % kStages);
+        const uint32_t ph = uint32_t(ks / kStages) & 1u;
+        if (ks >= kStages && !mbar_wait(&empty[s], ph ^ 1u, a.status, abort_flag)) break;
+        uint8_t* act_dst = act_s + s * act_bytes;
+        if (ks < my_main) {
+          const int64_t g = g_begin + ks;
+          mbar_arrive_expect_tx(&full[s], act_bytes + 4096u);
+          tma_load_2d(act_dst, &P.tm_act, &full[s], int32_t(g * 64), int32_t(m0));
+          if (!BWD) tma_load_2d(pk_s + s * 4096, &P.tm_pk, &full[s], int32_t(g * 32), int32_t(w0));
+          else      tma_load_2d(pk_s + s * 4096, &P.tm_pk, &full[s], int32_t(w0 / 2), int32_t(g * 64));
+        } else {
+          const int l = int(ks - my_main);
+          const int nchunk = a.rp / 64;
+          const int part = l / nchunk, c = l % nchunk;
+          const int32_t col = int32_t(part * a.rp + c * 64);
+          if (!BWD) {
+            mbar_arrive_expect_tx(&full[s], act_bytes);
+            tma_load_2d(act_dst, &P.tm_lact, &full[s], col, int32_t(m0));
+          } else {
+            mbar_arrive_expect_tx(&full[s], act_bytes + 16384u);
+            tma_load_2d(act_dst, &P.tm_lact, &full[s], col, int32_t(m0));
+            tma_load_2d(a_s + s * 16384, &P.tm_lw, &full[s], int32_t(c * 64), int32_t(w0));
+          }
+        }
+        issued = ks + 1;
+      }
+      if (*abort_flag) {   // let copies already in flight land before the CTA exits
+        for (int64_t ks = (issued > kStages ? issued - kStages : 0); ks < issued; ++ks)
+          mbar_drain(&full[ks % kStages], uint32_t(ks / kStages) & 1u);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t idesc_main = make_idesc_bf16(128, bt, BWD ? 1 : 0, 0);
+    const uint32_t idesc_lora = make_idesc_bf16(128, bt, 0, 0);
+    for (int64_t ks = 0; ks < nsteps; ++ks) {
+      const int s = int(ks % kStages);
+      const uint32_t ph = uint32_t(ks / kStages) & 1u;
+      if (!mbar_wait(&full[s], ph, a.status, abort_flag)) break;
+      const bool need_a = !BWD || ks < my_main;
+      if (need_a && !mbar_wait(&afull[s], ph, a.status, abort_flag)) break;
+      tc_fence_after();
+      if (elect_one()) {
+        const uint32_t act_addr = smem_u32(act_s + s * act_bytes);
+        const uint32_t a_addr = smem_u32(a_s + s * 16384);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t bdesc = make_sdesc_sw128(act_addr + kk * 32, 16, 1024);
+          const uint32_t acc = (ks > 0 || kk > 0) ? 1u : 0u;
+          if (!BWD) {
+            mma_ts(tmem_base, tmem_base + a_col0 + s * 32 + kk * 8, bdesc, idesc_main, acc);
+          } else if (ks < my_main) {
+            mma_ss(tmem_base, make_sdesc_sw128(a_addr + kk * 2048, 8192, 1024), bdesc, idesc_main, acc);
+          } else {
+            mma_ss(tmem_base, make_sdesc_sw128(a_addr + kk * 32, 16, 1024), bdesc, idesc_lora, acc);
+          }
+        }
+        mma_commit(&empty[s]);
+      }
+      __syncwarp();
+    }
+    if (elect_one()) {
+      mma_commit(accf);
+      if (*abort_flag) mbar_drain(accf, 0);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ dequant warpgroups
+    const int wg = (warp - 4) >> 2;
+    const int t = threadIdx.x - 128 - 128 * wg;               // TMEM lane 0..127
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    bool ok = true;
+    for (int64_t ks = wg; ks < nsteps && ok; ks += 2) {
+      const int s = int(ks % kStages);
+      const uint32_t ph = uint32_t(ks / kStages) & 1u;
+      if (ks < my_main) {
+        const int64_t g = g_begin + ks;
+        uint32_t o[32];
+        if (!BWD) {
+          const int64_t n = w0 + t;
+          const float s1 = (n < a.N) ? block_scale(a, n * KB + g) : 0.0f;
+          if (!(ok = mbar_wait(&full[s], ph, a.status, abort_flag))) break;
+          const uint32_t pa = smem_u32(pk_s + s * 4096 + t * 32);
+          const uint4 p0 = lds128(pa), p1 = lds128(pa + 16);
+          dequant64(make_table(P.code, s1), p0, p1, o);
+          tmem_st_32x32b_x32(tmem_base + lane_base + a_col0 + s * 32, o);
+          tmem_wait_st();
+        } else {
+          const int nl = t & 63, kb = t >> 6;
+          const int64_t n = g * 64 + nl;
+          const int64_t kblk = w0 / 64 + kb;
+          const float s1 = (n < a.N && kblk < KB) ? block_scale(a, n * KB + kblk) : 0.0f;
+          if (!(ok = mbar_wait(&full[s], ph, a.status, abort_flag))) break;
+          const uint32_t pa = smem_u32(pk_s + s * 4096 + nl * 64 + kb * 32);
+          const uint4 p0 = lds128(pa), p1 = lds128(pa + 16);
+          dequant64(make_table(P.code, s1), p0, p1, o);
+          const uint32_t row = smem_u32(a_s + s * 16384) + kb * 8192 + (nl >> 3) * 1024 + (nl & 7) * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            sts128(row + ((c ^ (nl & 7)) << 4), o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+          fence_proxy_async_smem();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&afull[s]);
+      } else if (!BWD) {
+        // low-rank step: column n of B (rank chunk c) is row n of the A operand
+        const int l = int(ks - my_main);
+        const int c = l % (a.rp / 64);
+        const int64_t n = w0 + t;
+        uint32_t o[32];
+#pragma unroll 8
+        for (int i = 0; i < 32; ++i) {
+          const int j0 = c * 64 + 2 * i;
+          const uint32_t lo = (n < a.N && j0 < a.r) ? uint32_t(__ldg(a.lora_w + int64_t(j0) * a.N + n)) : 0u;
+          const uint32_t hi = (n < a.N && j0 + 1 < a.r) ? uint32_t(__ldg(a.lora_w + int64_t(j0 + 1) * a.N + n)) : 0u;
+          o[i] = lo | (hi << 16);
+        }
+        if (!(ok = mbar_wait(&full[s], ph, a.status, abort_flag))) break;
+        tmem_st_32x32b_x32(tmem_base + lane_base + a_col0 + s * 32, o);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&afull[s]);
+      }
+    }
+
+    // ------------------------------------------------------------ epilogue
+    const int64_t wdim = BWD ? a.K : a.N;       // extent of the W dimension of the output
+    const int64_t ld = wdim;                    // Y [M,N] / dX [M,K] row length
+    const int64_t i = w0 + t;
+    const int nchunks = bt / 32;
+    const int64_t tile_lin = tile_t * gridDim.x + tile_w;
+    const bool got_acc = ok && mbar_wait(accf, 0, a.status, abort_flag);
+    if (got_acc) {
+      tc_fence_after();
+      for (int c = wg; c < nchunks; c += 2) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem_base + lane_base + c * 32, v);
+        tmem_wait_ld();
+        if (P.splits == 1) {
+          if (i < wdim) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int64_t m = m0 + c * 32 + j;
+              if (m < a.M) {
+                const uint32_t b = pack_bf16x2(__uint_as_float(v[j]), 0.0f);
+                a.out[m * ld + i] = uint16_t(b & 0xFFFFu);
+              }
+            }
+          }
+        } else {
+          float* dst = a.partial + ((tile_lin * P.splits + split) * bt + c * 32) * 128 + t;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) dst[j * 128] = __uint_as_float(v[j]);
+        }
+      }
+    }
+    if (P.splits > 1) {
+      __threadfence();
+      named_bar_sync(1, 256);
+      if (threadIdx.x == 128) {
+        const uint32_t old = atomicAdd(a.counters + tile_lin, 1u);
+        *last_flag = (old == uint32_t(P.splits - 1)) ? 1 : 0;
+      }
+      named_bar_sync(1, 256);
+      if (*last_flag) {
+        __threadfence();
+        for (int c = wg; c < nchunks; c += 2) {
+          for (int j = 0; j < 32; ++j) {
+            float acc = 0.0f;
+            for (int sp = 0; sp < P.splits; ++sp)
+              acc += __ldcg(a.partial + ((tile_lin * P.splits + sp) * bt + c * 32 + j) * 128 + t);
+            const int64_t m = m0 + c * 32 + j;
+            if (i < wdim && m < a.M) a.out[m * ld + i] = uint16_t(pack_bf16x2(acc, 0.0f) & 0xFFFFu);
+          }
+        }
+        if (threadIdx.x == 128) a.counters[tile_lin] = 0u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, tmem_cols);
+  }
+}
+
+// ============================================================================
+// skinny GEMM for the rank-r products
+// ============================================================================
+struct SkinnyParams {
+  CUtensorMap tm_a;
+  CUtensorMap tm_b;
+  SkinnyArgs a;
+  int kind;
+  int a_mn, b_mn;      // operand majors (1 = MN-major)
+  int splits;
+  int64_t steps;       // total 64-wide reduction steps
+  int64_t pass_steps;  // steps per pass (dA: one pass over G hi, one over G lo)
+  int64_t rows;
+};
+
+__device__ __forceinline__ uint32_t bf16_bits(float x) { return pack_bf16x2(x, 0.0f) & 0xFFFFu; }
+
+__device__ __forceinline__ void skinny_finish(const SkinnyParams& P, int64_t i, int j, float acc) {
+  const SkinnyArgs& a = P.a;
+  switch (P.kind) {
+    case kSkinnyT: {
+      if (i >= a.M) return;
+      const uint32_t tb = bf16_bits(acc);                 // T in the bf16 compute type
+      if (j < a.r && a.T_out) a.T_out[i * a.r + j] = uint16_t(tb);
+      const float v = (j < a.r) ? a.s * __uint_as_float(tb << 16) : 0.0f;
+      const uint32_t hi = bf16_bits(v);
+      const uint32_t lo = bf16_bits(v - __uint_as_float(hi << 16));
+      a.hilo_out[i * 2 * a.rp + j] = uint16_t(hi);
+      a.hilo_out[i * 2 * a.rp + a.rp + j] = uint16_t(lo);
+      break;
+    }
+    case kSkinnyG: {
+      if (i >= a.M) return;
+      const float v = (j < a.r) ? a.s * acc : 0.0f;
+      const uint32_t hi = bf16_bits(v);
+      const uint32_t lo = bf16_bits(v - __uint_as_float(hi << 16));
+      a.hilo_out[i * 2 * a.rp + j] = uint16_t(hi);
+      a.hilo_out[i * 2 * a.rp + a.rp + j] = uint16_t(lo);
+      break;
+    }
+    case kSkinnyDA:
+      if (i < a.K && j < a.r) a.f32_out[i * a.r + j] = acc;
+      break;
+    default:  // kSkinnyDB: computed as dB^T
+      if (i < a.N && j < a.r) a.f32_out[int64_t(j) * a.N + i] = a.s * acc;
+      break;
+  }
+}
+
+__global__ void __launch_bounds__(kSkinnyThreads, 1) skinny_gemm_kernel(const __grid_constant__ SkinnyParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const SkinnyArgs& a = P.a;
+  const int rp = a.rp;
+  const uint32_t b_bytes = uint32_t(rp) * 128u;
+  constexpr uint32_t a_bytes = 16384u;
+  const uint32_t stage_bytes = a_bytes + 32768u;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSkinnyStages * stage_bytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kSkinnyStages;
+  uint64_t* accf = bars + 2 * kSkinnyStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_flag = abort_flag + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int64_t tile = blockIdx.x;
+  const int split = blockIdx.y;
+  const int64_t i0 = tile * 128;
+  const int64_t per = (P.steps + P.splits - 1) / P.splits;
+  const int64_t g_begin = split * per;
+  const int64_t g_end = (g_begin + per < P.steps) ? g_begin + per : P.steps;
+  const int64_t nsteps = g_end > g_begin ? g_end - g_begin : 0;
+  const uint32_t tmem_cols = rp <= 32 ? 32u : (rp <= 64 ? 64u : (rp <= 128 ? 128u : 256u));
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kSkinnyStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accf, 1);
+    *abort_flag = 0;
+    *last_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (elect_one()) {
+      tma_prefetch_desc(&P.tm_a);
+      tma_prefetch_desc(&P.tm_b);
+      int64_t issued = 0;
+      for (int64_t ks = 0; ks < nsteps; ++ks) {
+        const int s = int(ks % kSkinnyStages);
+        const uint32_t ph = uint32_t(ks / kSkinnyStages) & 1u;
+        if (ks >= kSkinnyStages && !mbar_wait(&empty[s], ph ^ 1u, a.status, abort_flag)) break;
+        const int64_t g = g_begin + ks;
+        const int64_t pass = g / P.pass_steps, gi = g % P.pass_steps;
+        uint8_t* as = smem + s * stage_bytes;
+        uint8_t* bs = as + a_bytes;
+        mbar_arrive_expect_tx(&full[s], a_bytes + b_bytes);
+        const int32_t kc = int32_t(gi * 64);
+        if (P.a_mn) {   // two 64x64 boxes along the MN dimension
+          tma_load_2d(as, &P.tm_a, &full[s], int32_t(i0), kc);
+          tma_load_2d(as + 8192, &P.tm_a, &full[s], int32_t(i0 + 64), kc);
+        } else {
+          tma_load_2d(as, &P.tm_a, &full[s], kc, int32_t(i0));
+        }
+        if (P.b_mn) {
+          for (int q = 0; q < rp / 64; ++q)
+            tma_load_2d(bs + q * 8192, &P.tm_b, &full[s], int32_t(pass * rp + q * 64), kc);
+        } else {
+          tma_load_2d(bs, &P.tm_b, &full[s], kc, 0);
+        }
+        issued = ks + 1;
+      }
+      if (*abort_flag) {
+        for (int64_t ks = (issued > kSkinnyStages ? issued - kSkinnyStages : 0); ks < issued; ++ks)
+          mbar_drain(&full[ks % kSkinnyStages], uint32_t(ks / kSkinnyStages) & 1u);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    const uint32_t idesc = make_idesc_bf16(128, rp, P.a_mn, P.b_mn);
+    for (int64_t ks = 0; ks < nsteps; ++ks) {
+      const int s = int(ks % kSkinnyStages);
+      const uint32_t ph = uint32_t(ks / kSkinnyStages) & 1u;
+      if (!mbar_wait(&full[s], ph, a.status, abort_flag)) break;
+      tc_fence_after();
+      if (elect_one()) {
+        const uint32_t aa = smem_u32(smem + s * stage_bytes);
+        const uint32_t ba = aa + a_bytes;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t ad = P.a_mn ? make_sdesc_sw128(aa + kk * 2048, 8192, 1024)
+                                     : make_sdesc_sw128(aa + kk * 32, 16, 1024);
+          const uint64_t bd = P.b_mn ? make_sdesc_sw128(ba + kk * 2048, 8192, 1024)
+                                     : make_sdesc_sw128(ba + kk * 32, 16, 1024);
+          mma_ss(tmem_base, ad, bd, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&empty[s]);
+      }
+      __syncwarp();
+    }
+    if (elect_one()) {
+      mma_commit(accf);
+      if (*abort_flag) mbar_drain(accf, 0);
+    }
+    __syncwarp();
+  } else {
+    // epilogue: warps 2..5, TMEM lane quarter = warp % 4
+    const int q = warp & 3;
+    const int t = q * 32 + (threadIdx.x & 31);
+    const uint32_t lane_base = uint32_t(q * 32) << 16;
+    const int64_t i = i0 + t;
+    const bool got = nsteps > 0 && mbar_wait(accf, 0, a.status, abort_flag);
+    if (got) {
+      tc_fence_after();
+      for (int c = 0; c < rp / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem_base + lane_base + c * 32, v);
+        tmem_wait_ld();
+        if (P.splits == 1) {
+          for (int j = 0; j < 32; ++j) skinny_finish(P, i, c * 32 + j, __uint_as_float(v[j]));
+        } else {
+          float* dst = a.partial + ((tile * P.splits + split) * int64_t(rp) + c * 32) * 128 + t;
+          for (int j = 0; j < 32; ++j) dst[j * 128] = __uint_as_float(v[j]);
+        }
+      }
+    } else if (P.splits > 1 && nsteps == 0) {
+      // an empty split contributes zeros
+      for (int j = 0; j < rp; ++j) a.partial[((tile * P.splits + split) * int64_t(rp) + j) * 128 + t] = 0.0f;
+    }
+    if (P.splits > 1) {
+      __threadfence();
+      named_bar_sync(1, 128);
+      if (threadIdx.x == 64) {
+        const uint32_t old = atomicAdd(a.counters + tile, 1u);
+        *last_flag = (old == uint32_t(P.splits - 1)) ? 1 : 0;
+      }
+      named_bar_sync(1, 128);
+      if (*last_flag) {
+        __threadfence();
+        for (int j = 0; j < rp; ++j) {
+          float acc = 0.0f;
+          for (int sp = 0; sp < P.splits; ++sp)
+            acc += __ldcg(a.partial + ((tile * P.splits + sp) * int64_t(rp) + j) * 128 + t);
+          skinny_finish(P, i, j, acc);
+        }
+        if (threadIdx.x == 64) a.counters[tile] = 0u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, tmem_cols);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+}  // namespace
+
+bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
+                    uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Split counters live in the 4 KB workspace header after a 16-byte status slot.
+constexpr int64_t kMaxCounters = 1000;
+
+static int choose_splits(int64_t base_ctas, int64_t steps, int num_sms, int min_steps) {
+  if (base_ctas >= num_sms) return 1;
+  int best = 1;
+  double best_eff = 0.0;
+  for (int s = 1; s <= 32; ++s) {
+    if (steps / s < min_steps && s > 1) break;
+    const int64_t ctas = base_ctas * s;
+    const int64_t waves = cdiv(ctas, num_sms);
+    const double eff = double(ctas) / double(waves * num_sms);
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = s;
+    }
+  }
+  return best;
+}
+
+Nf4GemmPlan plan_nf4_gemm(int backward, int64_t M, int64_t N, int64_t K, int r, int num_sms) {
+  Nf4GemmPlan p{};
+  p.backward = backward;
+  p.bt = M <= 32 ? 32 : (M <= 64 ? 64 : (M <= 128 ? 128 : 256));
+  const int64_t wdim = backward ? K : N;
+  p.tiles_w = cdiv(wdim, 128);
+  p.tiles_t = cdiv(M, p.bt);
+  p.main_steps = backward ? cdiv(N, 64) : K / 64;
+  const int rp = int(cdiv(r, 64) * 64);
+  p.lora_steps = 2 * (rp / 64);
+  p.splits = choose_splits(p.tiles_w * p.tiles_t, p.main_steps, num_sms, 4);
+  if (p.tiles_w * p.tiles_t > kMaxCounters) p.splits = 1;
+  p.splits = int(cdiv(p.main_steps, cdiv(p.main_steps, p.splits)));   // no empty split
+  p.partial_bytes = p.splits > 1 ? size_t(p.tiles_w * p.tiles_t * p.splits) * p.bt * 128 * 4 : 0;
+  return p;
+}
+
+SkinnyPlan plan_skinny(int kind, int64_t M, int64_t N, int64_t K, int r, int num_sms) {
+  SkinnyPlan p{};
+  p.kind = kind;
+  switch (kind) {
+    case kSkinnyT: p.rows = M; p.red = K; p.steps = cdiv(K, 64); break;
+    case kSkinnyG: p.rows = M; p.red = N; p.steps = cdiv(N, 64); break;
+    case kSkinnyDA: p.rows = K; p.red = M; p.steps = 2 * cdiv(M, 64); break;
+    default: p.rows = N; p.red = M; p.steps = cdiv(M, 64); break;
+  }
+  p.tiles = cdiv(p.rows, 128);
+  p.splits = choose_splits(p.tiles, p.steps, num_sms, 2);
+  if (p.tiles > kMaxCounters) p.splits = 1;
+  p.splits = int(cdiv(p.steps, cdiv(p.steps, p.splits)));   // no empty split
+  const int rp = int(cdiv(r, 64) * 64);
+  p.partial_bytes = p.splits > 1 ? size_t(p.tiles * p.splits) * rp * 128 * 4 : 0;
+  return p;
+}
+
+static size_t nf4_gemm_smem(int backward, int bt) {
+  return 1024 + size_t(kStages) * (size_t(bt) * 128 + 4096 + (backward ? 16384 : 0)) + 256;
+}
+static size_t skinny_smem() { return 1024 + size_t(kSkinnyStages) * (16384 + 32768) + 256; }
+
+cudaError_t launch_nf4_gemm(const Nf4GemmPlan& plan, const Nf4GemmArgs& a, cudaStream_t stream) {
+  Nf4GemmParams P;
+  memset(&P, 0, sizeof(P));
+  P.a = a;
+  P.bt = plan.bt;
+  P.splits = plan.splits;
+  P.main_steps = plan.main_steps;
+  P.lora_steps = plan.lora_steps;
+  const Codebook& cb = host_codebook();
+  for (int i = 0; i < 16; ++i) P.code.v[i] = cb.code[i];
+  const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
+  const auto NOSW = CU_TENSOR_MAP_SWIZZLE_NONE;
+  bool ok = true;
+  const uint64_t M = a.M, N = a.N, K = a.K;
+  const uint64_t hw = 2 * uint64_t(a.rp);
+  if (!plan.backward) {
+    ok &= encode_tmap_2d(&P.tm_act, BF, a.act, K, M, K * 2, 64, plan.bt, SW);
+    ok &= encode_tmap_2d(&P.tm_pk, U8, a.packed, K / 2, N, K / 2, 32, 128, NOSW);
+  } else {
+    ok &= encode_tmap_2d(&P.tm_act, BF, a.act, N, M, N * 2, 64, plan.bt, SW);
+    ok &= encode_tmap_2d(&P.tm_pk, U8, a.packed, K / 2, N, K / 2, 64, 64, NOSW);
+    ok &= encode_tmap_2d(&P.tm_lw, BF, a.lora_w, uint64_t(a.r), K, uint64_t(a.r) * 2, 64, 128, SW);
+  }
+  ok &= encode_tmap_2d(&P.tm_lact, BF, a.lora_act, hw, M, hw * 2, 64, plan.bt, SW);
+  if (!ok) return cudaErrorInvalidValue;
+  const size_t smem = nf4_gemm_smem(plan.backward, plan.bt);
+  dim3 grid(unsigned(plan.tiles_w), unsigned(plan.tiles_t), unsigned(plan.splits));
+  cudaError_t e;
+  if (plan.backward) {
+    e = cudaFuncSetAttribute(nf4_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    nf4_gemm_kernel<true><<<grid, kGemmThreads, smem, stream>>>(P);
+  } else {
+    e = cudaFuncSetAttribute(nf4_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    nf4_gemm_kernel<false><<<grid, kGemmThreads, smem, stream>>>(P);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_skinny(const SkinnyPlan& plan, const SkinnyArgs& a, cudaStream_t stream) {
+  SkinnyParams P;
+  memset(&P, 0, sizeof(P));
+  P.a = a;
+  P.kind = plan.kind;
+  P.splits = plan.splits;
+  P.steps = plan.steps;
+  P.rows = plan.rows;
+  P.pass_steps = plan.steps;
+  const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
+  const uint64_t M = a.M, N = a.N, K = a.K, r = uint64_t(a.r), rp = uint64_t(a.rp);
+  bool ok = true;
+  switch (plan.kind) {
+    case kSkinnyT:   // A-op X [M,K] K-major; B-op A [K,r] MN-major
+      P.a_mn = 0; P.b_mn = 1;
+      ok &= encode_tmap_2d(&P.tm_a, BF, a.X, K, M, K * 2, 64, 128, SW);
+      ok &= encode_tmap_2d(&P.tm_b, BF, a.A, r, K, r * 2, 64, 64, SW);
+      break;
+    case kSkinnyG:   // A-op dY [M,N] K-major; B-op B [r,N] K-major
+      P.a_mn = 0; P.b_mn = 0;
+      ok &= encode_tmap_2d(&P.tm_a, BF, a.dY, N, M, N * 2, 64, 128, SW);
+      ok &= encode_tmap_2d(&P.tm_b, BF, a.B, N, r, N * 2, 64, uint32_t(rp), SW);
+      break;
+    case kSkinnyDA:  // A-op X^T (MN-major view of X); B-op G hi/lo MN-major
+      P.a_mn = 1; P.b_mn = 1;
+      P.pass_steps = plan.steps / 2;
+      ok &= encode_tmap_2d(&P.tm_a, BF, a.X, K, M, K * 2, 64, 64, SW);
+      ok &= encode_tmap_2d(&P.tm_b, BF, a.hilo_in, 2 * rp, M, 2 * rp * 2, 64, 64, SW);
+      break;
+    default:         // dB^T: A-op dY^T (MN-major view of dY); B-op T MN-major
+      P.a_mn = 1; P.b_mn = 1;
+      ok &= encode_tmap_2d(&P.tm_a, BF, a.dY, N, M, N * 2, 64, 64, SW);
+      ok &= encode_tmap_2d(&P.tm_b, BF, a.T, r, M, r * 2, 64, 64, SW);
+      break;
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  const size_t smem = skinny_smem();
+  cudaError_t e = cudaFuncSetAttribute(skinny_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid(unsigned(plan.tiles), unsigned(plan.splits));
+  skinny_gemm_kernel<<<grid, kSkinnyThreads, smem, stream>>>(P);
+  return cudaGetLastError();
+}
+
+}  // namespace nf4

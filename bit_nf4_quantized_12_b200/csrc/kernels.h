@@ -1,0 +1,94 @@
+// kernels.h -- internal launchers of libqlora_nf4 (not part of the C ABI).
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace nf4 {
+
+cudaError_t launch_quantize(const uint16_t* W, int64_t numel, uint8_t* packed, uint8_t* c1q, float* c2,
+                            uint32_t* status, int num_sms, cudaStream_t stream);
+cudaError_t launch_dequant(const uint8_t* packed, const uint8_t* c1q, const float* c2, int64_t numel,
+                           uint16_t* out, int num_sms, cudaStream_t stream);
+bool quantize_table_ok();
+
+// ---------------------------------------------------------------- fused NF4 GEMM
+// Computes, for a tile grid over (W-dim x tokens):
+//   forward : Y[m, n]  = sum_k X[m,k] Wd[n,k]  + sum_j (sT)[m,j] B[j,n]
+//   backward: dX[m, k] = sum_n dY[m,n] Wd[n,k] + sum_j G[m,j]  A[k,j]
+// with Wd dequantized on chip from (packed, c1q, c2); the low-rank operand
+// (sT or G) arrives as a bf16 hi/lo pair [M, 2*rp] (columns [0,rp) hi,
+// [rp,2rp) lo).
+struct Nf4GemmPlan {
+  int backward;      // 0 forward, 1 backward
+  int bt;            // token tile (MMA N): 16..256, multiple of 16
+  int splits;        // split of the main reduction
+  int64_t tiles_w;   // tiles along the W dimension (128 each)
+  int64_t tiles_t;   // tiles along tokens
+  int64_t main_steps;  // 64-wide reduction steps of the main product
+  int lora_steps;    // 64-wide steps of the low-rank product (hi and lo)
+  size_t partial_bytes;  // fp32 split partials (0 when splits == 1)
+};
+Nf4GemmPlan plan_nf4_gemm(int backward, int64_t M, int64_t N, int64_t K, int r, int num_sms);
+
+struct Nf4GemmArgs {
+  // problem
+  int64_t M, N, K;      // tokens, W rows, W cols
+  int r, rp;            // LoRA rank and its padding to 64
+  const uint8_t* packed;
+  const uint8_t* c1q;
+  const float* c2;
+  const uint16_t* act;       // X (forward) or dY (backward), [M, K] or [M, N]
+  const uint16_t* lora_w;    // B [r, N] (forward; read by the dequant warps) or A [K, r] (backward)
+  const uint16_t* lora_act;  // sT hi/lo (forward) or G hi/lo (backward), [M, 2*rp] bf16
+  uint16_t* out;             // Y [M, N] or dX [M, K], bf16
+  float* partial;            // split partials
+  uint32_t* counters;        // one per output tile (split reduction)
+  uint32_t* status;          // kStatusTimeout on a failed wait
+};
+cudaError_t launch_nf4_gemm(const Nf4GemmPlan& plan, const Nf4GemmArgs& a, cudaStream_t stream);
+
+// ---------------------------------------------------------------- skinny GEMM
+// D[i, j] = sum_k Aop[i,k] Bop[j,k] for the low-rank products, j < rp <= 256.
+enum SkinnyKind : int {
+  kSkinnyT = 0,   // T = X A      -> T bf16 [M,r], sT hi/lo [M,2rp]
+  kSkinnyG = 1,   // G = s dY B^T -> G hi/lo [M,2rp]
+  kSkinnyDA = 2,  // dA = X^T G   -> fp32 [K,r]   (reduction over tokens, G hi then lo)
+  kSkinnyDB = 3,  // dB = s T^T dY-> fp32 [r,N]   (computed transposed, reduction over tokens)
+};
+struct SkinnyPlan {
+  int kind;
+  int64_t rows;        // extent of i
+  int64_t red;         // reduction length
+  int64_t tiles;       // 128-row tiles of i
+  int64_t steps;       // 64-wide reduction steps (total, all passes)
+  int splits;
+  size_t partial_bytes;
+};
+SkinnyPlan plan_skinny(int kind, int64_t M, int64_t N, int64_t K, int r, int num_sms);
+
+struct SkinnyArgs {
+  int64_t M, N, K;
+  int r, rp;
+  float s;
+  const uint16_t* X;
+  const uint16_t* dY;
+  const uint16_t* A;
+  const uint16_t* B;
+  const uint16_t* T;        // bf16 [M, r] (input of kSkinnyDB)
+  const uint16_t* hilo_in;  // G hi/lo (input of kSkinnyDA)
+  uint16_t* T_out;          // kSkinnyT
+  uint16_t* hilo_out;       // kSkinnyT (sT) / kSkinnyG (G)
+  float* f32_out;           // kSkinnyDA / kSkinnyDB
+  float* partial;
+  uint32_t* counters;
+  uint32_t* status;
+};
+cudaError_t launch_skinny(const SkinnyPlan& plan, const SkinnyArgs& a, cudaStream_t stream);
+
+// Tensor-map helper (driver entry point resolved through the runtime).
+bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
+                    uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                    CUtensorMapSwizzle swizzle);
+
+}  // namespace nf4

@@ -1,0 +1,128 @@
+/*
+ * qlora_nf4.h -- C ABI of libqlora_nf4.so: 4-bit NormalFloat (NF4) storage
+ * of a frozen weight with double quantization of its block constants, and
+ * the QLoRA linear layer that computes in BF16 from that storage, on NVIDIA
+ * B200 (sm_100a).
+ *
+ * Sources (web pages about QLoRA; titles and sections):
+ *   [P1] "从LoRA到QLoRA：量化技术如何改变预训练模型的微调方式" -- §2.3 NF4
+ *        (quantiles of N(0,1), normalized to [-1,1]); §3.1 storage type NF4,
+ *        compute type BF16, gradients only for the LoRA parameters.
+ *   [P2] "QLoRA 原理精讲" -- §2.1 NF4 (block of 64, absmax, nearest code);
+ *        §2.2 double quantization (FP8 scale1 per 64 weights, one FP32
+ *        scale2 per 256 scale1, dequantize in reverse order); §三 误区1 (LoRA
+ *        factors stay BF16); §三 误区3 (serve with the adapter kept separate,
+ *        dequantizing on the fly).
+ *   [P4] "LoRA、Q-LoRA 与 PortLLM" (developer.volcengine.com) -- §3.1-§3.4,
+ *        the QLoRA linear layer for one layer of the quantized base model.
+ *
+ * Conventions (all calls):
+ *   - bf16 tensors are passed as uint16_t bit patterns, row-major.
+ *   - Every pointer argument named d_* or documented "device" is a device
+ *     pointer owned by the caller; the library allocates no memory and keeps
+ *     no state between calls besides the constant NF4 table.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     asynchronous on it; the return value reports argument validation and
+ *     launch errors only.  Device pointers must be 16-byte aligned
+ *     (NF4_ERR_MISALIGNED otherwise).
+ *   - Sizes are element counts.  No kernel traps, asserts or waits without a
+ *     bound: a wait that gives up sets bit 1 of the status word (below).
+ *   - Status words: a device int32 the caller zero-fills and reads after the
+ *     stream synchronizes: bit 0 = a NaN/Inf weight was seen by the
+ *     quantizer (outputs then unspecified), bit 1 = a bounded device wait
+ *     timed out (outputs unspecified).
+ */
+#ifndef QLORA_NF4_H
+#define QLORA_NF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  NF4_OK = 0,
+  NF4_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, bad rank */
+  NF4_ERR_MISALIGNED = 2,  /* a device pointer is not 16-byte aligned */
+  NF4_ERR_UNSUPPORTED = 3, /* a shape the library does not handle */
+  NF4_ERR_WORKSPACE = 4,   /* workspace missing or smaller than qlora_workspace_bytes() */
+  NF4_ERR_NONFINITE = 5,   /* reserved for callers mapping status bit 0 */
+  NF4_ERR_CUDA = 6         /* a CUDA runtime call or kernel launch failed */
+} nf4_status;
+
+/* A quantized weight W [rows, cols] (device buffers, see nf4_quantize_dq). */
+typedef struct {
+  const uint8_t* packed; /* ceil(rows*cols/2) bytes */
+  const uint8_t* c1q;    /* nblocks bytes */
+  const float* c2;       /* ngroups floats */
+  int64_t rows;          /* N: output features */
+  int64_t cols;          /* K: input features */
+} nf4_weight;
+
+/* The 16 NF4 values, ascending (codes) and the 15 decision thresholds
+ * (thresholds[i] = midpoint of codes i and i+1 rounded down to fp32), as
+ * used by the kernels.  [P1] §2.3, [P2] §2.1.  Host only; never fails. */
+nf4_status nf4_build_codebook(float codes[16], float thresholds[15]);
+
+/* Storage sizes for numel weights: packed bytes = ceil(numel/2), nblocks =
+ * ceil(numel/64), ngroups = ceil(nblocks/256).  Any output may be NULL.
+ * [P2] §2.2.  NF4_ERR_INVALID_ARG for numel < 1. */
+nf4_status nf4_sizes(int64_t numel, size_t* packed_bytes, int64_t* nblocks, int64_t* ngroups);
+
+/* Quantize a bf16 weight W [rows, cols] (device, row-major) to NF4 with
+ * double quantization ([P2] §2.1 steps 1-3, §2.2):
+ *   blocks are 64 consecutive elements of the row-major flattening, groups
+ *   256 consecutive blocks (the last block and group may be short);
+ *   scale1 = max |w| per block; code = nearest NF4 value to w / scale1,
+ *   ties to the lower code (all-zero block -> the 0.0 code);
+ *   c2 = fp32(max scale1 of the group / 448);
+ *   c1q = FP8 E4M3 of fp32(scale1 / c2), nearest even, saturating at 448
+ *   (0 for scale1 = 0);
+ *   packed: element e in byte e/2, even e in the low nibble, pad nibble 0.
+ * Outputs: packed, c1q, c2 (device, sizes from nf4_sizes).  d_status
+ * (device int32, may be NULL) gets bit 0 OR-ed in when W holds NaN/Inf. */
+nf4_status nf4_quantize_dq(const uint16_t* W, int64_t rows, int64_t cols, uint8_t* packed, uint8_t* c1q,
+                           float* c2, int32_t* d_status, void* stream);
+
+/* Double dequantization to bf16, reverse order ([P2] §2.2):
+ * scale1' = fp32(E4M3 value of c1q * c2), out = bf16(fp32(code * scale1'))
+ * (one fp32 multiply each, one round-to-nearest-even to bf16).
+ * out: device bf16 [rows, cols]. */
+nf4_status nf4_dequant_bf16(nf4_weight w, uint16_t* out, void* stream);
+
+/* Device workspace bytes needed by qlora_linear_fwd / qlora_linear_bwd for
+ * M tokens, W [N, K] and rank r on the current device (0 on bad sizes). */
+size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t r);
+
+/* QLoRA linear forward ([P4] §3.4; [P1] §3.1):
+ *   T = bf16(X A),  Y = bf16(X Wd^T + s T B),  Wd = dequant(w) in bf16,
+ * with X [M, K], A [K, r], B [r, N], Y [M, N], T [M, r] (T_out may be NULL),
+ * all device bf16; s = alpha / r computed by the caller.  Wd is formed on
+ * chip and never written to memory.  ws: device workspace of at least
+ * qlora_workspace_bytes(M, N, K, r) bytes; its first 4 bytes are the status
+ * word (zeroed by the call).  Requires K % 64 == 0, N % 8 == 0 and
+ * r % 8 == 0 (NF4_ERR_UNSUPPORTED otherwise); 1 <= r <= 256. */
+nf4_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight w, const uint16_t* A, const uint16_t* B,
+                            int32_t r, float s, uint16_t* Y, uint16_t* T_out, void* ws, size_t ws_bytes,
+                            void* stream);
+
+/* QLoRA linear backward ([P1] §3.1: the frozen weight gets no gradient; it
+ * is dequantized again on chip):
+ *   G = s dY B^T,  dX = bf16(dY Wd + G A^T),  dA = X^T G,  dB = s T^T dY,
+ * dY [M, N] bf16, X [M, K] bf16, T [M, r] bf16 from the forward (NULL: the
+ * call recomputes it), dX [M, K] bf16, dA [K, r] fp32, dB [r, N] fp32 (all
+ * device).  Same workspace and shape rules as qlora_linear_fwd. */
+nf4_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, nf4_weight w, const uint16_t* A,
+                            const uint16_t* B, int32_t r, float s, const uint16_t* T, uint16_t* dX, float* dA,
+                            float* dB, void* ws, size_t ws_bytes, void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* nf4_status_str(nf4_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_NF4_H */
