@@ -284,6 +284,34 @@ def config_dict(wl, n):
             "l2": "step working set ~1.3 GB > 126 MB L2; no flush between steps"}
 
 
+def kernel_case(case, n):
+    """n launches of one call on the 7B q matrix (4096x4096, 2048 tokens, r=64),
+    or on the 28672x8192 decode weight at M=16: a small case for ncu."""
+    from bit_nf4_quantized_12_b200 import binding
+    dev = torch.device("cuda", 0)
+    wl = workloads.WORKLOADS["llama7b"]
+    M, r, s = wl.tokens, wl.r, wl.s
+    N, K = 4096, 4096
+    if case == "decode":
+        M, r, s, N, K = 16, 16, 1.0, 28672, 8192
+    W = workloads.weight(N, K, 0.02, seed=0, device=dev)
+    io = workloads.layer_inputs(M, N, K, r, seed=0, device=dev)
+    qw = binding.quantize(W)
+    Wd = torch.empty_like(W)
+    ws = binding.workspace(M, N, K, r, dev)
+    Y, T = binding.linear_fwd(io["X"], qw, io["A"], io["B"], s, ws=ws)
+    for _ in range(n):
+        if case == "quantize":
+            binding.quantize(W, out=qw)
+        elif case == "dequant":
+            binding.dequant(qw, out=Wd)
+        elif case in ("fwd", "decode"):
+            binding.linear_fwd(io["X"], qw, io["A"], io["B"], s, ws=ws, Y=Y, T=T)
+        else:
+            binding.linear_bwd(io["dY"], io["X"], qw, io["A"], io["B"], s, T=T, ws=ws)
+    torch.cuda.synchronize()
+
+
 # ------------------------------------------------------------------ main
 def main():
     ap = argparse.ArgumentParser()
@@ -292,6 +320,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-components", action="store_true")
+    ap.add_argument("--kernel-case", default=None, choices=["quantize", "dequant", "fwd", "bwd", "decode"],
+                    help="run a few launches of one call on one 7B-shaped matrix (for ncu), print nothing")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -305,6 +335,9 @@ def main():
 
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device")
+    if args.kernel_case:
+        kernel_case(args.kernel_case, args.steps)
+        return
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     pg = None

@@ -24,15 +24,13 @@ int device_sms() {
 
 int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 
-// Workspace: [status word + split counters | low-rank hi/lo | T scratch | split partials]
+// Workspace: [status word (256 B) | low-rank hi/lo pair [M, 2rp] bf16 | T scratch [M, r] bf16]
 struct WsLayout {
-  size_t counters = 16;      // 1023 counters after the 16-byte status slot
-  size_t hilo = 0, t_scratch = 0, partial = 0, total = 0;
-  size_t partial_bytes = 0;
+  size_t hilo = 0, t_scratch = 0, total = 0;
 };
-constexpr size_t kHeaderBytes = 4096;
+constexpr size_t kHeaderBytes = 256;
 
-WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int r, int sms) {
+WsLayout ws_layout(int64_t M, int64_t /*N*/, int64_t /*K*/, int r, int /*sms*/) {
   WsLayout L;
   const int64_t rp = round_up(r, 64);
   size_t off = kHeaderBytes;
@@ -40,14 +38,6 @@ WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int r, int sms) {
   off += size_t(round_up(M * 2 * rp * 2, 256));
   L.t_scratch = off;
   off += size_t(round_up(M * r * 2, 256));
-  L.partial = off;
-  size_t pb = 0;
-  auto upd = [&](size_t b) { if (b > pb) pb = b; };
-  upd(plan_nf4_gemm(0, M, N, K, r, sms).partial_bytes);
-  upd(plan_nf4_gemm(1, M, N, K, r, sms).partial_bytes);
-  for (int kind = 0; kind < 4; ++kind) upd(plan_skinny(kind, M, N, K, r, sms).partial_bytes);
-  L.partial_bytes = pb;
-  off += size_t(round_up(int64_t(pb), 256));
   L.total = off;
   return L;
 }
@@ -122,10 +112,8 @@ nf4_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight w, const ui
   cudaStream_t strm = static_cast<cudaStream_t>(stream);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   uint32_t* status = reinterpret_cast<uint32_t*>(wsb);
-  uint32_t* counters = reinterpret_cast<uint32_t*>(wsb + L.counters);
   uint16_t* hilo = reinterpret_cast<uint16_t*>(wsb + L.hilo);
   uint16_t* t_dst = T_out ? T_out : reinterpret_cast<uint16_t*>(wsb + L.t_scratch);
-  float* partial = reinterpret_cast<float*>(wsb + L.partial);
   const int rp = int(round_up(r, 64));
 
   if (cudaMemsetAsync(ws, 0, kHeaderBytes, strm) != cudaSuccess) return NF4_ERR_CUDA;
@@ -134,14 +122,14 @@ nf4_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight w, const ui
   sa.M = M; sa.N = N; sa.K = K; sa.r = r; sa.rp = rp; sa.s = s;
   sa.X = X; sa.A = A; sa.B = B;
   sa.T_out = t_dst; sa.hilo_out = hilo;
-  sa.partial = partial; sa.counters = counters; sa.status = status;
+  sa.status = status;
   if (launch_skinny(plan_skinny(kSkinnyT, M, N, K, r, sms), sa, strm) != cudaSuccess) return NF4_ERR_CUDA;
 
   Nf4GemmArgs ga{};
   ga.M = M; ga.N = N; ga.K = K; ga.r = r; ga.rp = rp;
   ga.packed = w.packed; ga.c1q = w.c1q; ga.c2 = w.c2;
   ga.act = X; ga.lora_w = B; ga.lora_act = hilo; ga.out = Y;
-  ga.partial = partial; ga.counters = counters; ga.status = status;
+  ga.status = status;
   if (launch_nf4_gemm(plan_nf4_gemm(0, M, N, K, r, sms), ga, strm) != cudaSuccess) return NF4_ERR_CUDA;
   return NF4_OK;
 }
@@ -163,9 +151,7 @@ nf4_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, nf
   cudaStream_t strm = static_cast<cudaStream_t>(stream);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   uint32_t* status = reinterpret_cast<uint32_t*>(wsb);
-  uint32_t* counters = reinterpret_cast<uint32_t*>(wsb + L.counters);
   uint16_t* hilo = reinterpret_cast<uint16_t*>(wsb + L.hilo);
-  float* partial = reinterpret_cast<float*>(wsb + L.partial);
   const int rp = int(round_up(r, 64));
 
   if (cudaMemsetAsync(ws, 0, kHeaderBytes, strm) != cudaSuccess) return NF4_ERR_CUDA;
@@ -173,7 +159,7 @@ nf4_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, nf
   SkinnyArgs sa{};
   sa.M = M; sa.N = N; sa.K = K; sa.r = r; sa.rp = rp; sa.s = s;
   sa.X = X; sa.dY = dY; sa.A = A; sa.B = B;
-  sa.partial = partial; sa.counters = counters; sa.status = status;
+  sa.status = status;
 
   const uint16_t* Tin = T;
   if (!Tin) {  // recompute T = bf16(X A) into scratch (the hi/lo output is overwritten by G below)
@@ -193,7 +179,7 @@ nf4_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, nf
   ga.M = M; ga.N = N; ga.K = K; ga.r = r; ga.rp = rp;
   ga.packed = w.packed; ga.c1q = w.c1q; ga.c2 = w.c2;
   ga.act = dY; ga.lora_w = A; ga.lora_act = hilo; ga.out = dX;
-  ga.partial = partial; ga.counters = counters; ga.status = status;
+  ga.status = status;
   if (launch_nf4_gemm(plan_nf4_gemm(1, M, N, K, r, sms), ga, strm) != cudaSuccess) return NF4_ERR_CUDA;
 
   // dA = X^T G  (G hi + G lo)

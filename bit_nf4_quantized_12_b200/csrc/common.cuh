@@ -208,6 +208,29 @@ NF4_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: 
 NF4_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // ----------------------------------------------------------------------------
+// thread-block clusters: rank, hardware barrier, distributed shared memory
+// ----------------------------------------------------------------------------
+NF4_DEV uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Every thread of every CTA in the cluster must call this (hardware barrier,
+// release/acquire ordering of shared::cluster accesses around it).
+NF4_DEV void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+// fp32 load from the shared memory of CTA `rank` of this cluster, at the
+// address that `local` has in this CTA.
+NF4_DEV float ld_dsmem_f32(const void* local, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
+}
+
+// ----------------------------------------------------------------------------
 // small numeric helpers
 // ----------------------------------------------------------------------------
 NF4_DEV float bf16lo_to_f32(uint32_t two) { return __uint_as_float(two << 16); }

@@ -119,9 +119,6 @@ __device__ __forceinline__ float block_scale(const Nf4GemmArgs& a, int64_t b) {
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
-__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
 // Wait ignoring the abort flag (used only to drain in-flight copies/MMAs).
 __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
@@ -152,7 +149,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
   uint64_t* accf = bars + 3 * kStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* last_flag = abort_flag + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t tile_w = blockIdx.x, tile_t = blockIdx.y;
@@ -177,7 +173,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
     }
     mbar_init(accf, 1);
     *abort_flag = 0;
-    *last_flag = 0;
     fence_mbar_init();
   }
   if (warp == 2) {
@@ -328,57 +323,59 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
 
     // ------------------------------------------------------------ epilogue
     const int64_t wdim = BWD ? a.K : a.N;       // extent of the W dimension of the output
-    const int64_t ld = wdim;                    // Y [M,N] / dX [M,K] row length
     const int64_t i = w0 + t;
     const int nchunks = bt / 32;
-    const int64_t tile_lin = tile_t * gridDim.x + tile_w;
     const bool got_acc = ok && mbar_wait(accf, 0, a.status, abort_flag);
-    if (got_acc) {
-      tc_fence_after();
-      for (int c = wg; c < nchunks; c += 2) {
-        uint32_t v[32];
+    if (got_acc) tc_fence_after();
+    float* red = reinterpret_cast<float*>(act_s);   // split partial [bt][128] (stages are free now)
+    for (int c = wg; c < nchunks; c += 2) {
+      uint32_t v[32];
+      if (got_acc) {
         tmem_ld_32x32b_x32(tmem_base + lane_base + c * 32, v);
         tmem_wait_ld();
-        if (P.splits == 1) {
-          if (i < wdim) {
+      } else {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int64_t m = m0 + c * 32 + j;
-              if (m < a.M) {
-                const uint32_t b = pack_bf16x2(__uint_as_float(v[j]), 0.0f);
-                a.out[m * ld + i] = uint16_t(b & 0xFFFFu);
-              }
-            }
-          }
-        } else {
-          float* dst = a.partial + ((tile_lin * P.splits + split) * bt + c * 32) * 128 + t;
+        for (int j = 0; j < 32; ++j) v[j] = 0u;
+      }
+      if (P.splits == 1) {
+        if (i < wdim) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) dst[j * 128] = __uint_as_float(v[j]);
-        }
-      }
-    }
-    if (P.splits > 1) {
-      __threadfence();
-      named_bar_sync(1, 256);
-      if (threadIdx.x == 128) {
-        const uint32_t old = atomicAdd(a.counters + tile_lin, 1u);
-        *last_flag = (old == uint32_t(P.splits - 1)) ? 1 : 0;
-      }
-      named_bar_sync(1, 256);
-      if (*last_flag) {
-        __threadfence();
-        for (int c = wg; c < nchunks; c += 2) {
           for (int j = 0; j < 32; ++j) {
-            float acc = 0.0f;
-            for (int sp = 0; sp < P.splits; ++sp)
-              acc += __ldcg(a.partial + ((tile_lin * P.splits + sp) * bt + c * 32 + j) * 128 + t);
             const int64_t m = m0 + c * 32 + j;
-            if (i < wdim && m < a.M) a.out[m * ld + i] = uint16_t(pack_bf16x2(acc, 0.0f) & 0xFFFFu);
+            if (m < a.M) a.out[m * wdim + i] = uint16_t(pack_bf16x2(__uint_as_float(v[j]), 0.0f) & 0xFFFFu);
           }
         }
-        if (threadIdx.x == 128) a.counters[tile_lin] = 0u;
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) red[(c * 32 + j) * 128 + t] = __uint_as_float(v[j]);
       }
     }
+  }
+
+  // ------------------------------------------------------------ split reduction
+  // The CTAs of one output tile form a cluster along z; each sums a slice of
+  // the tile's columns over every CTA's partial (distributed shared memory,
+  // fixed order, so results do not depend on timing).
+  if (P.splits > 1) {
+    cluster_sync_all();
+    if (warp >= 4) {
+      const int wg = (warp - 4) >> 2;
+      const int t = threadIdx.x - 128 - 128 * wg;
+      const int64_t wdim = BWD ? a.K : a.N;
+      const int64_t i = w0 + t;
+      const float* red = reinterpret_cast<const float*>(act_s);
+      const int cps = bt / P.splits;
+      const int c0 = int(cluster_ctarank()) * cps;
+      for (int col = c0 + wg; col < c0 + cps; col += 2) {
+        float acc = 0.0f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (q < P.splits) acc += ld_dsmem_f32(red + col * 128 + t, uint32_t(q));
+        const int64_t m = m0 + col;
+        if (i < wdim && m < a.M) a.out[m * wdim + i] = uint16_t(pack_bf16x2(acc, 0.0f) & 0xFFFFu);
+      }
+    }
+    cluster_sync_all();
   }
 
   tc_fence_before();
@@ -452,7 +449,6 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1) skinny_gemm_kernel(const __
   uint64_t* accf = bars + 2 * kSkinnyStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* last_flag = abort_flag + 1;
 
   const int warp = threadIdx.x >> 5;
   const int64_t tile = blockIdx.x;
@@ -471,7 +467,6 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1) skinny_gemm_kernel(const __
     }
     mbar_init(accf, 1);
     *abort_flag = 0;
-    *last_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -552,42 +547,44 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1) skinny_gemm_kernel(const __
     const uint32_t lane_base = uint32_t(q * 32) << 16;
     const int64_t i = i0 + t;
     const bool got = nsteps > 0 && mbar_wait(accf, 0, a.status, abort_flag);
-    if (got) {
-      tc_fence_after();
-      for (int c = 0; c < rp / 32; ++c) {
-        uint32_t v[32];
+    if (got) tc_fence_after();
+    float* red = reinterpret_cast<float*>(smem);   // split partial [rp][128]
+    for (int c = 0; c < rp / 32; ++c) {
+      uint32_t v[32];
+      if (got) {
         tmem_ld_32x32b_x32(tmem_base + lane_base + c * 32, v);
         tmem_wait_ld();
-        if (P.splits == 1) {
-          for (int j = 0; j < 32; ++j) skinny_finish(P, i, c * 32 + j, __uint_as_float(v[j]));
-        } else {
-          float* dst = a.partial + ((tile * P.splits + split) * int64_t(rp) + c * 32) * 128 + t;
-          for (int j = 0; j < 32; ++j) dst[j * 128] = __uint_as_float(v[j]);
-        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = 0u;
       }
-    } else if (P.splits > 1 && nsteps == 0) {
-      // an empty split contributes zeros
-      for (int j = 0; j < rp; ++j) a.partial[((tile * P.splits + split) * int64_t(rp) + j) * 128 + t] = 0.0f;
-    }
-    if (P.splits > 1) {
-      __threadfence();
-      named_bar_sync(1, 128);
-      if (threadIdx.x == 64) {
-        const uint32_t old = atomicAdd(a.counters + tile, 1u);
-        *last_flag = (old == uint32_t(P.splits - 1)) ? 1 : 0;
-      }
-      named_bar_sync(1, 128);
-      if (*last_flag) {
-        __threadfence();
-        for (int j = 0; j < rp; ++j) {
-          float acc = 0.0f;
-          for (int sp = 0; sp < P.splits; ++sp)
-            acc += __ldcg(a.partial + ((tile * P.splits + sp) * int64_t(rp) + j) * 128 + t);
-          skinny_finish(P, i, j, acc);
-        }
-        if (threadIdx.x == 64) a.counters[tile] = 0u;
+      if (P.splits == 1) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) skinny_finish(P, i, c * 32 + j, __uint_as_float(v[j]));
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) red[(c * 32 + j) * 128 + t] = __uint_as_float(v[j]);
       }
     }
+  }
+
+  if (P.splits > 1) {
+    cluster_sync_all();
+    if (warp >= 2) {
+      const int t = (warp & 3) * 32 + (threadIdx.x & 31);
+      const int64_t i = i0 + t;
+      const float* red = reinterpret_cast<const float*>(smem);
+      const int jps = rp / P.splits;
+      const int j0 = int(cluster_ctarank()) * jps;
+      for (int j = j0; j < j0 + jps; ++j) {
+        float acc = 0.0f;
+#pragma unroll
+        for (int qq = 0; qq < 8; ++qq)
+          if (qq < P.splits) acc += ld_dsmem_f32(red + j * 128 + t, uint32_t(qq));
+        skinny_finish(P, i, j, acc);
+      }
+    }
+    cluster_sync_all();
   }
 
   tc_fence_before();
@@ -634,24 +631,16 @@ bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* bas
   return r == CUDA_SUCCESS;
 }
 
-// Split counters live in the 4 KB workspace header after a 16-byte status slot.
-constexpr int64_t kMaxCounters = 1000;
-
-static int choose_splits(int64_t base_ctas, int64_t steps, int num_sms, int min_steps) {
+// Split of the reduction: 1, 2, 4 or 8 CTAs per output tile, launched as one
+// thread-block cluster (portable size <= 8) that reduces through distributed
+// shared memory.  Used only when the tile grid alone leaves SMs idle.
+static int choose_splits(int64_t base_ctas, int64_t steps, int num_sms, int min_steps, int64_t cap8) {
   if (base_ctas >= num_sms) return 1;
-  int best = 1;
-  double best_eff = 0.0;
-  for (int s = 1; s <= 32; ++s) {
-    if (steps / s < min_steps && s > 1) break;
-    const int64_t ctas = base_ctas * s;
-    const int64_t waves = cdiv(ctas, num_sms);
-    const double eff = double(ctas) / double(waves * num_sms);
-    if (eff > best_eff + 1e-9) {
-      best_eff = eff;
-      best = s;
-    }
+  for (int s : {8, 4, 2}) {
+    const int64_t cap = (s == 8) ? cap8 : num_sms;
+    if (base_ctas * s <= cap && steps / s >= min_steps) return s;
   }
-  return best;
+  return 1;
 }
 
 Nf4GemmPlan plan_nf4_gemm(int backward, int64_t M, int64_t N, int64_t K, int r, int num_sms) {
@@ -664,10 +653,7 @@ Nf4GemmPlan plan_nf4_gemm(int backward, int64_t M, int64_t N, int64_t K, int r, 
   p.main_steps = backward ? cdiv(N, 64) : K / 64;
   const int rp = int(cdiv(r, 64) * 64);
   p.lora_steps = 2 * (rp / 64);
-  p.splits = choose_splits(p.tiles_w * p.tiles_t, p.main_steps, num_sms, 4);
-  if (p.tiles_w * p.tiles_t > kMaxCounters) p.splits = 1;
-  p.splits = int(cdiv(p.main_steps, cdiv(p.main_steps, p.splits)));   // no empty split
-  p.partial_bytes = p.splits > 1 ? size_t(p.tiles_w * p.tiles_t * p.splits) * p.bt * 128 * 4 : 0;
+  p.splits = choose_splits(p.tiles_w * p.tiles_t, p.main_steps, num_sms, 4, (num_sms * 7) / 8);
   return p;
 }
 
@@ -681,12 +667,26 @@ SkinnyPlan plan_skinny(int kind, int64_t M, int64_t N, int64_t K, int r, int num
     default: p.rows = N; p.red = M; p.steps = cdiv(M, 64); break;
   }
   p.tiles = cdiv(p.rows, 128);
-  p.splits = choose_splits(p.tiles, p.steps, num_sms, 2);
-  if (p.tiles > kMaxCounters) p.splits = 1;
-  p.splits = int(cdiv(p.steps, cdiv(p.steps, p.splits)));   // no empty split
-  const int rp = int(cdiv(r, 64) * 64);
-  p.partial_bytes = p.splits > 1 ? size_t(p.tiles * p.splits) * rp * 128 * 4 : 0;
+  p.splits = choose_splits(p.tiles, p.steps, num_sms, 2, (num_sms * 7) / 8);
   return p;
+}
+
+template <class Params>
+static cudaError_t launch_clustered(void (*kern)(const Params), dim3 grid, dim3 block, size_t smem,
+                                    cudaStream_t stream, dim3 cluster, const Params& P) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cluster.x;
+  attr[0].val.clusterDim.y = cluster.y;
+  attr[0].val.clusterDim.z = cluster.z;
+  cfg.attrs = attr;
+  cfg.numAttrs = (cluster.x * cluster.y * cluster.z > 1) ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, P);
 }
 
 static size_t nf4_gemm_smem(int backward, int bt) {
@@ -723,17 +723,10 @@ cudaError_t launch_nf4_gemm(const Nf4GemmPlan& plan, const Nf4GemmArgs& a, cudaS
   if (!ok) return cudaErrorInvalidValue;
   const size_t smem = nf4_gemm_smem(plan.backward, plan.bt);
   dim3 grid(unsigned(plan.tiles_w), unsigned(plan.tiles_t), unsigned(plan.splits));
-  cudaError_t e;
-  if (plan.backward) {
-    e = cudaFuncSetAttribute(nf4_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (e != cudaSuccess) return e;
-    nf4_gemm_kernel<true><<<grid, kGemmThreads, smem, stream>>>(P);
-  } else {
-    e = cudaFuncSetAttribute(nf4_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (e != cudaSuccess) return e;
-    nf4_gemm_kernel<false><<<grid, kGemmThreads, smem, stream>>>(P);
-  }
-  return cudaGetLastError();
+  void (*kern)(const Nf4GemmParams) = plan.backward ? nf4_gemm_kernel<true> : nf4_gemm_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  return launch_clustered(kern, grid, dim3(kGemmThreads), smem, stream, dim3(1, 1, unsigned(plan.splits)), P);
 }
 
 cudaError_t launch_skinny(const SkinnyPlan& plan, const SkinnyArgs& a, cudaStream_t stream) {
@@ -777,8 +770,8 @@ cudaError_t launch_skinny(const SkinnyPlan& plan, const SkinnyArgs& a, cudaStrea
   cudaError_t e = cudaFuncSetAttribute(skinny_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(unsigned(plan.tiles), unsigned(plan.splits));
-  skinny_gemm_kernel<<<grid, kSkinnyThreads, smem, stream>>>(P);
-  return cudaGetLastError();
+  return launch_clustered(skinny_gemm_kernel, grid, dim3(kSkinnyThreads), smem, stream,
+                          dim3(1, unsigned(plan.splits), 1), P);
 }
 
 }  // namespace nf4

@@ -18,7 +18,8 @@ bool quantize_table_ok();
 //   backward: dX[m, k] = sum_n dY[m,n] Wd[n,k] + sum_j G[m,j]  A[k,j]
 // with Wd dequantized on chip from (packed, c1q, c2); the low-rank operand
 // (sT or G) arrives as a bf16 hi/lo pair [M, 2*rp] (columns [0,rp) hi,
-// [rp,2rp) lo).
+// [rp,2rp) lo).  When the tile grid is small the reduction is split over a
+// cluster of up to 8 CTAs that sum through distributed shared memory.
 struct Nf4GemmPlan {
   int backward;      // 0 forward, 1 backward
   int bt;            // token tile (MMA N): 16..256, multiple of 16
@@ -27,7 +28,6 @@ struct Nf4GemmPlan {
   int64_t tiles_t;   // tiles along tokens
   int64_t main_steps;  // 64-wide reduction steps of the main product
   int lora_steps;    // 64-wide steps of the low-rank product (hi and lo)
-  size_t partial_bytes;  // fp32 split partials (0 when splits == 1)
 };
 Nf4GemmPlan plan_nf4_gemm(int backward, int64_t M, int64_t N, int64_t K, int r, int num_sms);
 
@@ -42,8 +42,6 @@ struct Nf4GemmArgs {
   const uint16_t* lora_w;    // B [r, N] (forward; read by the dequant warps) or A [K, r] (backward)
   const uint16_t* lora_act;  // sT hi/lo (forward) or G hi/lo (backward), [M, 2*rp] bf16
   uint16_t* out;             // Y [M, N] or dX [M, K], bf16
-  float* partial;            // split partials
-  uint32_t* counters;        // one per output tile (split reduction)
   uint32_t* status;          // kStatusTimeout on a failed wait
 };
 cudaError_t launch_nf4_gemm(const Nf4GemmPlan& plan, const Nf4GemmArgs& a, cudaStream_t stream);
@@ -63,7 +61,6 @@ struct SkinnyPlan {
   int64_t tiles;       // 128-row tiles of i
   int64_t steps;       // 64-wide reduction steps (total, all passes)
   int splits;
-  size_t partial_bytes;
 };
 SkinnyPlan plan_skinny(int kind, int64_t M, int64_t N, int64_t K, int r, int num_sms);
 
@@ -80,8 +77,6 @@ struct SkinnyArgs {
   uint16_t* T_out;          // kSkinnyT
   uint16_t* hilo_out;       // kSkinnyT (sT) / kSkinnyG (G)
   float* f32_out;           // kSkinnyDA / kSkinnyDB
-  float* partial;
-  uint32_t* counters;
   uint32_t* status;
 };
 cudaError_t launch_skinny(const SkinnyPlan& plan, const SkinnyArgs& a, cudaStream_t stream);
