@@ -316,7 +316,7 @@ def kernel_case(case, n):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-components", action="store_true")
@@ -350,14 +350,21 @@ def main():
 
     step = Step(device, wl, host_copy=True)
     step_launches = step.launches_per_step
-    for _ in range(max(3, args.warmup)):
+    # warm-up: at least W steps and at least ~1.5 s of load, with the clock
+    # sampler already running so that its samples cover the loaded GPU
+    clocks = ClockSampler(local)
+    clocks.start()
+    t_w = time.perf_counter()
+    nw = 0
+    while nw < max(3, args.warmup) or time.perf_counter() - t_w < 1.5:
         step.run()
+        nw += 1
+        if nw % 8 == 0:
+            torch.cuda.synchronize()
     torch.cuda.synchronize()
 
     # ---- timed region: K device-resident steps
     ev = {k: ([], []) for k in ("q", "dq", "fwd", "bwd")}
-    clocks = ClockSampler(local)
-    clocks.start()
     if pg:
         pg.barrier()
     torch.cuda.synchronize()
