@@ -38,7 +38,8 @@ namespace nf4 {
 namespace {
 
 constexpr int kStages = 4;
-constexpr int kGemmThreads = 384;
+constexpr int kDequantWGs = 4;                          // dequant / epilogue warpgroups
+constexpr int kGemmThreads = 128 + 128 * kDequantWGs;   // + producer, MMA, allocator, spare warp
 constexpr int kSkinnyThreads = 192;
 constexpr int kSkinnyStages = 4;
 
@@ -111,9 +112,6 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, ui
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-__device__ __forceinline__ float block_scale(const Nf4GemmArgs& a, int64_t b) {
-  return e4m3_to_f32(__ldg(a.c1q + b)) * __ldg(a.c2 + (b >> 8));
-}
 
 // ---------------------------------------------------------------- kernel
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -262,62 +260,95 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------ dequant warpgroups
+    // Warpgroup wg takes reduction steps wg, wg + kDequantWGs, ...; the block
+    // scales (c1q, c2) of its next four steps are loaded one window ahead so
+    // their global-memory latency is off the critical path.
     const int wg = (warp - 4) >> 2;
     const int t = threadIdx.x - 128 - 128 * wg;               // TMEM lane 0..127
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    auto block_of = [&](int64_t ks) -> int64_t {              // NF4 block index used at step ks, or -1
+      if (ks >= my_main) return -1;
+      const int64_t g = g_begin + ks;
+      if (!BWD) {
+        const int64_t n = w0 + t;
+        return n < a.N ? n * KB + g : -1;
+      }
+      const int64_t n = g * 64 + (t & 63);
+      const int64_t kblk = w0 / 64 + (t >> 6);
+      return (n < a.N && kblk < KB) ? n * KB + kblk : -1;
+    };
+    uint32_t cq[4], nq[4];
+    float cc[4], nc[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int64_t b = block_of(wg + int64_t(j) * kDequantWGs);
+      cq[j] = b >= 0 ? uint32_t(__ldg(a.c1q + b)) : 0u;
+      cc[j] = b >= 0 ? __ldg(a.c2 + (b >> 8)) : 0.0f;
+    }
     bool ok = true;
-    for (int64_t ks = wg; ks < nsteps && ok; ks += 2) {
-      const int s = int(ks % kStages);
-      const uint32_t ph = uint32_t(ks / kStages) & 1u;
-      if (ks < my_main) {
-        const int64_t g = g_begin + ks;
-        uint32_t o[32];
-        if (!BWD) {
-          const int64_t n = w0 + t;
-          const float s1 = (n < a.N) ? block_scale(a, n * KB + g) : 0.0f;
+    for (int64_t base = wg; base < nsteps && ok; base += 4 * kDequantWGs) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int64_t b = block_of(base + int64_t(4 + j) * kDequantWGs);
+        nq[j] = b >= 0 ? uint32_t(__ldg(a.c1q + b)) : 0u;
+        nc[j] = b >= 0 ? __ldg(a.c2 + (b >> 8)) : 0.0f;
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int64_t ks = base + int64_t(j) * kDequantWGs;
+        if (!ok || ks >= nsteps) break;
+        const int s = int(ks % kStages);
+        const uint32_t ph = uint32_t(ks / kStages) & 1u;
+        if (ks < my_main) {
+          const float s1 = e4m3_to_f32(cq[j]) * cc[j];
+          uint32_t o[32];
           if (!(ok = mbar_wait(&full[s], ph, a.status, abort_flag))) break;
-          const uint32_t pa = smem_u32(pk_s + s * 4096 + t * 32);
-          const uint4 p0 = lds128(pa), p1 = lds128(pa + 16);
-          dequant64(make_table(P.code, s1), p0, p1, o);
+          if (!BWD) {
+            const uint32_t pa = smem_u32(pk_s + s * 4096 + t * 32);
+            const uint4 p0 = lds128(pa), p1 = lds128(pa + 16);
+            dequant64(make_table(P.code, s1), p0, p1, o);
+            tmem_st_32x32b_x32(tmem_base + lane_base + a_col0 + s * 32, o);
+            tmem_wait_st();
+          } else {
+            const int nl = t & 63, kb = t >> 6;
+            const uint32_t pa = smem_u32(pk_s + s * 4096 + nl * 64 + kb * 32);
+            const uint4 p0 = lds128(pa), p1 = lds128(pa + 16);
+            dequant64(make_table(P.code, s1), p0, p1, o);
+            const uint32_t row = smem_u32(a_s + s * 16384) + kb * 8192 + (nl >> 3) * 1024 + (nl & 7) * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              sts128(row + ((c ^ (nl & 7)) << 4), o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+            fence_proxy_async_smem();
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&afull[s]);
+        } else if (!BWD) {
+          // low-rank step: column n of B (rank chunk c) is row n of the A operand
+          const int l = int(ks - my_main);
+          const int c = l % (a.rp / 64);
+          const int64_t n = w0 + t;
+          uint32_t o[32];
+#pragma unroll 8
+          for (int i = 0; i < 32; ++i) {
+            const int j0 = c * 64 + 2 * i;
+            const uint32_t lo = (n < a.N && j0 < a.r) ? uint32_t(__ldg(a.lora_w + int64_t(j0) * a.N + n)) : 0u;
+            const uint32_t hi =
+                (n < a.N && j0 + 1 < a.r) ? uint32_t(__ldg(a.lora_w + int64_t(j0 + 1) * a.N + n)) : 0u;
+            o[i] = lo | (hi << 16);
+          }
+          if (!(ok = mbar_wait(&full[s], ph, a.status, abort_flag))) break;
           tmem_st_32x32b_x32(tmem_base + lane_base + a_col0 + s * 32, o);
           tmem_wait_st();
-        } else {
-          const int nl = t & 63, kb = t >> 6;
-          const int64_t n = g * 64 + nl;
-          const int64_t kblk = w0 / 64 + kb;
-          const float s1 = (n < a.N && kblk < KB) ? block_scale(a, n * KB + kblk) : 0.0f;
-          if (!(ok = mbar_wait(&full[s], ph, a.status, abort_flag))) break;
-          const uint32_t pa = smem_u32(pk_s + s * 4096 + nl * 64 + kb * 32);
-          const uint4 p0 = lds128(pa), p1 = lds128(pa + 16);
-          dequant64(make_table(P.code, s1), p0, p1, o);
-          const uint32_t row = smem_u32(a_s + s * 16384) + kb * 8192 + (nl >> 3) * 1024 + (nl & 7) * 128;
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&afull[s]);
+        }
+      }
 #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            sts128(row + ((c ^ (nl & 7)) << 4), o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
-          fence_proxy_async_smem();
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&afull[s]);
-      } else if (!BWD) {
-        // low-rank step: column n of B (rank chunk c) is row n of the A operand
-        const int l = int(ks - my_main);
-        const int c = l % (a.rp / 64);
-        const int64_t n = w0 + t;
-        uint32_t o[32];
-#pragma unroll 8
-        for (int i = 0; i < 32; ++i) {
-          const int j0 = c * 64 + 2 * i;
-          const uint32_t lo = (n < a.N && j0 < a.r) ? uint32_t(__ldg(a.lora_w + int64_t(j0) * a.N + n)) : 0u;
-          const uint32_t hi = (n < a.N && j0 + 1 < a.r) ? uint32_t(__ldg(a.lora_w + int64_t(j0 + 1) * a.N + n)) : 0u;
-          o[i] = lo | (hi << 16);
-        }
-        if (!(ok = mbar_wait(&full[s], ph, a.status, abort_flag))) break;
-        tmem_st_32x32b_x32(tmem_base + lane_base + a_col0 + s * 32, o);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&afull[s]);
+      for (int j = 0; j < 4; ++j) {
+        cq[j] = nq[j];
+        cc[j] = nc[j];
       }
     }
 
@@ -328,7 +359,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
     const bool got_acc = ok && mbar_wait(accf, 0, a.status, abort_flag);
     if (got_acc) tc_fence_after();
     float* red = reinterpret_cast<float*>(act_s);   // split partial [bt][128] (stages are free now)
-    for (int c = wg; c < nchunks; c += 2) {
+    for (int c = wg; c < nchunks; c += kDequantWGs) {
       uint32_t v[32];
       if (got_acc) {
         tmem_ld_32x32b_x32(tmem_base + lane_base + c * 32, v);
@@ -366,7 +397,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
       const float* red = reinterpret_cast<const float*>(act_s);
       const int cps = bt / P.splits;
       const int c0 = int(cluster_ctarank()) * cps;
-      for (int col = c0 + wg; col < c0 + cps; col += 2) {
+      for (int col = c0 + wg; col < c0 + cps; col += kDequantWGs) {
         float acc = 0.0f;
 #pragma unroll
         for (int q = 0; q < 8; ++q)

@@ -21,6 +21,7 @@
 // and the code decision as one shared-memory table lookup plus one compare.
 #include <cstdint>
 #include <cuda_runtime.h>
+#include <cuda_bf16.h>
 #include "common.cuh"
 #include "kernels.h"
 
@@ -84,12 +85,16 @@ __device__ __forceinline__ uint32_t quantize8_scaled(const uint2* lut, const uin
   return out;
 }
 
+__device__ __forceinline__ __nv_bfloat162 as_bf162(uint32_t u) {
+  return *reinterpret_cast<const __nv_bfloat162*>(&u);
+}
+// Largest |w| of 8 bf16 as a bf16 bit pattern (NaN propagates, so Inf/NaN
+// inputs give a pattern >= 0x7F80).
 __device__ __forceinline__ uint32_t absmax_bits8(const uint4& v) {
-  // |bf16| as 15-bit integers: their order is the order of magnitudes, and
-  // Inf/NaN patterns (>= 0x7F80) come out on top.
-  const uint32_t m = __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
-                              __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
-  return max(m & 0xFFFFu, m >> 16);
+  const __nv_bfloat162 m = __hmax2_nan(__hmax2_nan(__habs2(as_bf162(v.x)), __habs2(as_bf162(v.y))),
+                                       __hmax2_nan(__habs2(as_bf162(v.z)), __habs2(as_bf162(v.w))));
+  const uint32_t u = *reinterpret_cast<const uint32_t*>(&m);
+  return max(u & 0xFFFFu, u >> 16);
 }
 
 struct QuantArgs {
@@ -169,29 +174,35 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const __gri
     for (int w = 1; w < kQuantThreads / 32; ++w) gm = max(gm, warp_max[parity][w]);
     if (gm >= 0x7F80u) bad = 1;
 
-    // second level: fp32 scale2 for the group, E4M3 codes of scale1/scale2
+    // second level: fp32 scale2 for the group, E4M3 codes of scale1/scale2.
+    // Lane j of each 8-lane block group owns round j: it computes that
+    // block's code and reciprocal once; the others receive it by shuffle.
     const float gmax = __uint_as_float(gm << 16);
     const float s2 = __fdiv_rn(gmax, 448.0f);
     if (tid == 0) p.c2[g] = s2;
-    if ((tid & 7) == 0) {
+    const int j = lane & 7;
+    uint32_t my_bm = bm[0];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int64_t b = g * kGroup + i * 32 + (tid >> 3);
-        if (b < nblk_total) {
-          const float c1 = __uint_as_float(bm[i] << 16);
-          p.c1q[b] = (c1 == 0.0f) ? uint8_t(0) : uint8_t(f32_to_e4m3_satfinite(__fdiv_rn(c1, s2)));
-        }
-      }
+    for (int i = 1; i < 8; ++i) my_bm = (j == i) ? bm[i] : my_bm;
+    const float my_c1 = __uint_as_float(my_bm << 16);
+    {
+      const int64_t b = g * kGroup + j * 32 + (tid >> 3);
+      if (b < nblk_total)
+        p.c1q[b] = (my_c1 == 0.0f) ? uint8_t(0) : uint8_t(f32_to_e4m3_satfinite(__fdiv_rn(my_c1, s2)));
     }
+    const bool normal = (my_c1 >= 0x1p-126f && my_c1 <= 0x1p125f) || my_c1 == 0.0f;
+    const float my_inv = (my_c1 == 0.0f) ? 0.0f : (normal ? __frcp_rn(my_c1) : 0.0f);
+    const bool fast = __all_sync(0xffffffffu, normal);
     // 4-bit codes
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int64_t e0 = gbase + i * 2048 + tid * 8;
+      const float inv = __shfl_sync(0xffffffffu, my_inv, (lane & ~7) | i);
       if (e0 >= p.numel) continue;
       const float c1 = __uint_as_float(bm[i] << 16);
       uint32_t q8;
-      if (c1 >= 0x1p-126f && c1 <= 0x1p125f) {
-        q8 = quantize8(lut, v[i], __frcp_rn(c1));
+      if (fast || (c1 >= 0x1p-126f && c1 <= 0x1p125f)) {
+        q8 = (c1 == 0.0f) ? 0x77777777u : quantize8(lut, v[i], fast ? inv : __frcp_rn(c1));
       } else if (c1 == 0.0f) {
         q8 = 0x77777777u;                        // all-zero block: the 0.0 code
       } else {                                   // keep 1/c1 a normal number
@@ -204,11 +215,11 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const __gri
       } else {
         const int valid = int(p.numel - e0);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          if (2 * j < valid) {
-            uint32_t byte = (q8 >> (8 * j)) & 0xFFu;
-            if (2 * j + 1 >= valid) byte &= 0x0Fu;   // pad nibble of an odd tail
-            dst[j] = uint8_t(byte);
+        for (int jj = 0; jj < 4; ++jj) {
+          if (2 * jj < valid) {
+            uint32_t byte = (q8 >> (8 * jj)) & 0xFFu;
+            if (2 * jj + 1 >= valid) byte &= 0x0Fu;   // pad nibble of an odd tail
+            dst[jj] = uint8_t(byte);
           }
         }
       }
@@ -229,77 +240,55 @@ struct DequantArgs {
   float code[16];
 };
 
-// Per-block table: the 16 values bf16(code[q] * scale1), split into low- and
-// high-byte planes so that 4 lookups take a few byte permutes (prmt).
-struct DqTable {
-  uint32_t lo[4], hi[4];
-};
-__device__ __forceinline__ DqTable dq_table(const float (&code)[16], float s1) {
-  uint32_t pr[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) pr[i] = pack_bf16x2(code[2 * i] * s1, code[2 * i + 1] * s1);
-  DqTable t;
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    t.lo[k] = prmt(pr[2 * k], pr[2 * k + 1], 0x6420);
-    t.hi[k] = prmt(pr[2 * k], pr[2 * k + 1], 0x7531);
-  }
-  return t;
-}
-// nibbles j = 0..3 of s -> bf16 pairs (elements 0,1) and (2,3)
-__device__ __forceinline__ void dq_lookup4(const DqTable& t, uint32_t s, uint32_t& o01, uint32_t& o23) {
-  const uint32_t sel2 = ((s >> 1) & 0x4444u) | 0x3210u;
-  const uint32_t lo = prmt(prmt(t.lo[0], t.lo[1], s), prmt(t.lo[2], t.lo[3], s ^ 0x8888u), sel2);
-  const uint32_t hi = prmt(prmt(t.hi[0], t.hi[1], s), prmt(t.hi[2], t.hi[3], s ^ 0x8888u), sel2);
-  o01 = prmt(lo, hi, 0x5140);
-  o23 = prmt(lo, hi, 0x7362);
-}
-
-// One thread expands whole 64-weight blocks: two 16-byte loads of codes, one
-// table per block, eight 16-byte stores; two blocks per iteration.
+// Eight lanes per 64-weight block, eight weights (four packed bytes) per
+// lane and unit, so that every warp load covers 128 contiguous packed bytes
+// and every warp store 512 contiguous bytes of bf16; four units per lane per
+// iteration keep enough bytes in flight.  code[q] comes from a 16-word shared
+// table (one bank per entry), times the block scale in fp32, rounded to bf16.
+constexpr int kDqUnits = 4;
 __global__ void __launch_bounds__(256) nf4_dequant_kernel(const __grid_constant__ DequantArgs p) {
-  float code[16];
+  __shared__ float code_s[16];
+  if (threadIdx.x < 16) code_s[threadIdx.x] = p.code[threadIdx.x];
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int64_t nunits = p.numel / 8;                        // complete 8-weight units
+  const int64_t warp_id = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t base = warp_id * (32 * kDqUnits); base < nunits; base += nwarps * (32 * kDqUnits)) {
+    uint32_t w[kDqUnits];
+    float s1[kDqUnits];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) code[i] = p.code[i];
-  const int64_t nfull = p.numel / kBlock;                  // complete blocks
-  const int64_t stride = int64_t(gridDim.x) * blockDim.x;
-  for (int64_t b0 = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; b0 < nfull; b0 += 2 * stride) {
-    const int64_t b1 = b0 + stride;
-    const bool has1 = b1 < nfull;
-    const uint4* src0 = reinterpret_cast<const uint4*>(p.packed + b0 * 32);
-    const uint4 a0 = __ldcs(src0), a1 = __ldcs(src0 + 1);
-    uint4 c0 = make_uint4(0, 0, 0, 0), c1 = c0;
-    if (has1) {
-      const uint4* src1 = reinterpret_cast<const uint4*>(p.packed + b1 * 32);
-      c0 = __ldcs(src1);
-      c1 = __ldcs(src1 + 1);
-    }
-    const float s0 = e4m3_to_f32(__ldg(p.c1q + b0)) * __ldg(p.c2 + (b0 >> 8));
-    const float s1 = has1 ? e4m3_to_f32(__ldg(p.c1q + b1)) * __ldg(p.c2 + (b1 >> 8)) : 0.0f;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      if (h == 1 && !has1) break;
-      const DqTable t = dq_table(code, h ? s1 : s0);
-      const uint4 q0 = h ? c0 : a0, q1 = h ? c1 : a1;
-      const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-      uint4* dst = reinterpret_cast<uint4*>(p.out + (h ? b1 : b0) * kBlock);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        uint4 o;
-        dq_lookup4(t, w[i] & 0xFFFFu, o.x, o.y);
-        dq_lookup4(t, w[i] >> 16, o.z, o.w);
-        __stcs(dst + i, o);
+    for (int i = 0; i < kDqUnits; ++i) {
+      const int64_t u = base + i * 32 + lane;
+      if (u < nunits) {
+        w[i] = __ldcs(reinterpret_cast<const unsigned int*>(p.packed) + u);
+        const int64_t b = u >> 3;
+        s1[i] = e4m3_to_f32(__ldg(p.c1q + b)) * __ldg(p.c2 + (b >> 8));
+      } else {
+        w[i] = 0u;
+        s1[i] = 0.0f;
       }
     }
+#pragma unroll
+    for (int i = 0; i < kDqUnits; ++i) {
+      const int64_t u = base + i * 32 + lane;
+      if (u >= nunits) break;
+      uint4 o;
+      o.x = pack_bf16x2(code_s[w[i] & 0xFu] * s1[i], code_s[(w[i] >> 4) & 0xFu] * s1[i]);
+      o.y = pack_bf16x2(code_s[(w[i] >> 8) & 0xFu] * s1[i], code_s[(w[i] >> 12) & 0xFu] * s1[i]);
+      o.z = pack_bf16x2(code_s[(w[i] >> 16) & 0xFu] * s1[i], code_s[(w[i] >> 20) & 0xFu] * s1[i]);
+      o.w = pack_bf16x2(code_s[(w[i] >> 24) & 0xFu] * s1[i], code_s[w[i] >> 28] * s1[i]);
+      __stcs(reinterpret_cast<uint4*>(p.out) + u, o);
+    }
   }
-  // ragged tail: the last, short block (numel % 64 weights), one thread
-  if (blockIdx.x == 0 && threadIdx.x == 0 && p.numel % kBlock != 0) {
-    const int64_t b = nfull;
-    const float s1 = e4m3_to_f32(p.c1q[b]) * p.c2[b >> 8];
-    for (int64_t e = b * kBlock; e < p.numel; ++e) {
+  // ragged tail: the last numel % 8 weights, one thread
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    for (int64_t e = nunits * 8; e < p.numel; ++e) {
+      const int64_t b = e / kBlock;
+      const float s = e4m3_to_f32(p.c1q[b]) * p.c2[b >> 8];
       const uint32_t byte = p.packed[e >> 1];
       const uint32_t q = (e & 1) ? (byte >> 4) : (byte & 0xFu);
-      p.out[e] = uint16_t(pack_bf16x2(code[q] * s1, 0.0f) & 0xFFFFu);
+      p.out[e] = uint16_t(pack_bf16x2(code_s[q] * s, 0.0f) & 0xFFFFu);
     }
   }
 }
@@ -336,8 +325,8 @@ cudaError_t launch_dequant(const uint8_t* packed, const uint8_t* c1q, const floa
   a.numel = numel;
   const Codebook& cb = host_codebook();
   for (int i = 0; i < 16; ++i) a.code[i] = cb.code[i];
-  const int64_t nfull = numel / kBlock;
-  int64_t grid = (nfull / 2 + 255) / 256;
+  const int64_t nunits = numel / 8;
+  int64_t grid = (nunits / (32 * kDqUnits) + 7) / 8;   // 8 warps per CTA
   const int64_t cap = int64_t(num_sms) * 8;
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
