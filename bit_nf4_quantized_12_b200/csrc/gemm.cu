@@ -37,7 +37,6 @@
 namespace nf4 {
 namespace {
 
-constexpr int kStages = 4;
 constexpr int kDequantWGs = 4;                          // dequant / epilogue warpgroups
 constexpr int kGemmThreads = 128 + 128 * kDequantWGs;   // + producer, MMA, allocator, spare warp
 constexpr int kSkinnyThreads = 192;
@@ -125,26 +124,39 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
   }
 }
 
-// Forward tensor-memory layout: accumulator in columns [0, acc), the four
-// 32-column A stages after it.
+// Ring depths.  X: the activation tile ring (TMA), P: packed NF4 tiles (TMA,
+// 4 KB each, recycled as soon as a dequant warpgroup has read them), A: the
+// dequantized weight operand (tensor memory in the forward pass, shared
+// memory in the backward pass).  The dequant warps compute a step before they
+// wait for its A slot, so they run ahead of the tensor core by up to SA steps.
+template <bool BWD> struct Rings;
+template <> struct Rings<false> { static constexpr int SX = 5, SP = 12, SA = 8; };
+template <> struct Rings<true>  { static constexpr int SX = 4, SP = 8,  SA = 4; };
+
+// Forward tensor memory: accumulator in columns [0, a_col0), the SA
+// 32-column A slots after it.
 __host__ __device__ constexpr int fwd_a_col0(int bt) { return bt <= 128 ? 128 : 256; }
-__host__ __device__ constexpr uint32_t fwd_tmem_cols(int bt) { return bt <= 128 ? 256u : 512u; }
+constexpr uint32_t kFwdTmemCols = 512;
 
 template <bool BWD>
 __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_constant__ Nf4GemmParams P) {
+  constexpr int SX = Rings<BWD>::SX, SP = Rings<BWD>::SP, SA = Rings<BWD>::SA;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const Nf4GemmArgs& a = P.a;
   const int bt = P.bt;
   const uint32_t act_bytes = uint32_t(bt) * 128u;
-  uint8_t* act_s = smem;                                   // kStages x act_bytes
-  uint8_t* pk_s = act_s + kStages * act_bytes;             // kStages x 4096
-  uint8_t* a_s = pk_s + kStages * 4096;                    // backward: kStages x 16384
-  uint64_t* bars = reinterpret_cast<uint64_t*>(a_s + (BWD ? kStages * 16384 : 0));
-  uint64_t* full = bars;
-  uint64_t* afull = bars + kStages;
-  uint64_t* empty = bars + 2 * kStages;
-  uint64_t* accf = bars + 3 * kStages;
+  uint8_t* act_s = smem;                                   // SX x act_bytes
+  uint8_t* pk_s = act_s + SX * act_bytes;                  // SP x 4096
+  uint8_t* a_s = pk_s + SP * 4096;                         // backward: SA x 16384
+  uint64_t* bars = reinterpret_cast<uint64_t*>(a_s + (BWD ? SA * 16384 : 0));
+  uint64_t* x_full = bars;
+  uint64_t* x_empty = x_full + SX;
+  uint64_t* p_full = x_empty + SX;
+  uint64_t* p_empty = p_full + SP;
+  uint64_t* a_full = p_empty + SP;
+  uint64_t* a_empty = a_full + SA;
+  uint64_t* accf = a_empty + SA;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -160,15 +172,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
   const int my_lora = (split == 0) ? P.lora_steps : 0;
   const int64_t nsteps = my_main + my_lora;
   const int64_t KB = a.K / kBlock;          // NF4 blocks per W row
-  const uint32_t tmem_cols = BWD ? uint32_t(bt < 32 ? 32 : bt) : fwd_tmem_cols(bt);
+  const uint32_t tmem_cols = BWD ? uint32_t(bt < 32 ? 32 : bt) : kFwdTmemCols;
   const uint32_t a_col0 = uint32_t(fwd_a_col0(bt));
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&afull[s], 4);
-      mbar_init(&empty[s], 1);
-    }
+    for (int s = 0; s < SX; ++s) { mbar_init(&x_full[s], 1); mbar_init(&x_empty[s], 1); }
+    for (int s = 0; s < SP; ++s) { mbar_init(&p_full[s], 1); mbar_init(&p_empty[s], 4); }
+    for (int s = 0; s < SA; ++s) { mbar_init(&a_full[s], 4); mbar_init(&a_empty[s], 1); }
     mbar_init(accf, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -183,43 +193,51 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ X producer
     if (elect_one()) {
       tma_prefetch_desc(&P.tm_act);
-      tma_prefetch_desc(&P.tm_pk);
       tma_prefetch_desc(&P.tm_lact);
-      if (BWD) tma_prefetch_desc(&P.tm_lw);
       int64_t issued = 0;
       for (int64_t ks = 0; ks < nsteps; ++ks) {
-        const int s = int(ks % kStages);
-        const uint32_t ph = uint32_t(ks / kStages) & 1u;
-        if (ks >= kStages && !mbar_wait(&empty[s], ph ^ 1u, a.status, abort_flag)) break;
-        uint8_t* act_dst = act_s + s * act_bytes;
+        const int s = int(ks % SX);
+        const uint32_t ph = uint32_t(ks / SX) & 1u;
+        if (ks >= SX && !mbar_wait(&x_empty[s], ph ^ 1u, a.status, abort_flag)) break;
+        uint8_t* dst = act_s + s * act_bytes;
+        mbar_arrive_expect_tx(&x_full[s], act_bytes);
         if (ks < my_main) {
-          const int64_t g = g_begin + ks;
-          mbar_arrive_expect_tx(&full[s], act_bytes + 4096u);
-          tma_load_2d(act_dst, &P.tm_act, &full[s], int32_t(g * 64), int32_t(m0));
-          if (!BWD) tma_load_2d(pk_s + s * 4096, &P.tm_pk, &full[s], int32_t(g * 32), int32_t(w0));
-          else      tma_load_2d(pk_s + s * 4096, &P.tm_pk, &full[s], int32_t(w0 / 2), int32_t(g * 64));
+          tma_load_2d(dst, &P.tm_act, &x_full[s], int32_t((g_begin + ks) * 64), int32_t(m0));
         } else {
           const int l = int(ks - my_main);
           const int nchunk = a.rp / 64;
-          const int part = l / nchunk, c = l % nchunk;
-          const int32_t col = int32_t(part * a.rp + c * 64);
-          if (!BWD) {
-            mbar_arrive_expect_tx(&full[s], act_bytes);
-            tma_load_2d(act_dst, &P.tm_lact, &full[s], col, int32_t(m0));
-          } else {
-            mbar_arrive_expect_tx(&full[s], act_bytes + 16384u);
-            tma_load_2d(act_dst, &P.tm_lact, &full[s], col, int32_t(m0));
-            tma_load_2d(a_s + s * 16384, &P.tm_lw, &full[s], int32_t(c * 64), int32_t(w0));
-          }
+          tma_load_2d(dst, &P.tm_lact, &x_full[s], int32_t((l / nchunk) * a.rp + (l % nchunk) * 64),
+                      int32_t(m0));
         }
         issued = ks + 1;
       }
       if (*abort_flag) {   // let copies already in flight land before the CTA exits
-        for (int64_t ks = (issued > kStages ? issued - kStages : 0); ks < issued; ++ks)
-          mbar_drain(&full[ks % kStages], uint32_t(ks / kStages) & 1u);
+        for (int64_t ks = (issued > SX ? issued - SX : 0); ks < issued; ++ks)
+          mbar_drain(&x_full[ks % SX], uint32_t(ks / SX) & 1u);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ packed-W producer
+    if (elect_one()) {
+      tma_prefetch_desc(&P.tm_pk);
+      int64_t issued = 0;
+      for (int64_t ks = 0; ks < my_main; ++ks) {
+        const int s = int(ks % SP);
+        const uint32_t ph = uint32_t(ks / SP) & 1u;
+        if (ks >= SP && !mbar_wait(&p_empty[s], ph ^ 1u, a.status, abort_flag)) break;
+        const int64_t g = g_begin + ks;
+        mbar_arrive_expect_tx(&p_full[s], 4096u);
+        if (!BWD) tma_load_2d(pk_s + s * 4096, &P.tm_pk, &p_full[s], int32_t(g * 32), int32_t(w0));
+        else      tma_load_2d(pk_s + s * 4096, &P.tm_pk, &p_full[s], int32_t(w0 / 2), int32_t(g * 64));
+        issued = ks + 1;
+      }
+      if (*abort_flag) {
+        for (int64_t ks = (issued > SP ? issued - SP : 0); ks < issued; ++ks)
+          mbar_drain(&p_full[ks % SP], uint32_t(ks / SP) & 1u);
       }
     }
     __syncwarp();
@@ -228,28 +246,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
     const uint32_t idesc_main = make_idesc_bf16(128, bt, BWD ? 1 : 0, 0);
     const uint32_t idesc_lora = make_idesc_bf16(128, bt, 0, 0);
     for (int64_t ks = 0; ks < nsteps; ++ks) {
-      const int s = int(ks % kStages);
-      const uint32_t ph = uint32_t(ks / kStages) & 1u;
-      if (!mbar_wait(&full[s], ph, a.status, abort_flag)) break;
-      const bool need_a = !BWD || ks < my_main;
-      if (need_a && !mbar_wait(&afull[s], ph, a.status, abort_flag)) break;
+      const int sx = int(ks % SX), sa = int(ks % SA);
+      if (!mbar_wait(&x_full[sx], uint32_t(ks / SX) & 1u, a.status, abort_flag)) break;
+      if (!mbar_wait(&a_full[sa], uint32_t(ks / SA) & 1u, a.status, abort_flag)) break;
       tc_fence_after();
       if (elect_one()) {
-        const uint32_t act_addr = smem_u32(act_s + s * act_bytes);
-        const uint32_t a_addr = smem_u32(a_s + s * 16384);
+        const uint32_t act_addr = smem_u32(act_s + sx * act_bytes);
+        const uint32_t a_addr = smem_u32(a_s + sa * 16384);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t bdesc = make_sdesc_sw128(act_addr + kk * 32, 16, 1024);
           const uint32_t acc = (ks > 0 || kk > 0) ? 1u : 0u;
           if (!BWD) {
-            mma_ts(tmem_base, tmem_base + a_col0 + s * 32 + kk * 8, bdesc, idesc_main, acc);
+            mma_ts(tmem_base, tmem_base + a_col0 + sa * 32 + kk * 8, bdesc, idesc_main, acc);
           } else if (ks < my_main) {
             mma_ss(tmem_base, make_sdesc_sw128(a_addr + kk * 2048, 8192, 1024), bdesc, idesc_main, acc);
           } else {
             mma_ss(tmem_base, make_sdesc_sw128(a_addr + kk * 32, 16, 1024), bdesc, idesc_lora, acc);
           }
         }
-        mma_commit(&empty[s]);
+        mma_commit(&x_empty[sx]);
+        mma_commit(&a_empty[sa]);
       }
       __syncwarp();
     }
@@ -297,38 +314,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
       for (int j = 0; j < 4; ++j) {
         const int64_t ks = base + int64_t(j) * kDequantWGs;
         if (!ok || ks >= nsteps) break;
-        const int s = int(ks % kStages);
-        const uint32_t ph = uint32_t(ks / kStages) & 1u;
+        const int sa = int(ks % SA);
+        const uint32_t a_ph = uint32_t(ks / SA) & 1u;
+        uint32_t o[32];
         if (ks < my_main) {
-          const float s1 = e4m3_to_f32(cq[j]) * cc[j];
-          uint32_t o[32];
-          if (!(ok = mbar_wait(&full[s], ph, a.status, abort_flag))) break;
-          if (!BWD) {
-            const uint32_t pa = smem_u32(pk_s + s * 4096 + t * 32);
-            const uint4 p0 = lds128(pa), p1 = lds128(pa + 16);
-            dequant64(make_table(P.code, s1), p0, p1, o);
-            tmem_st_32x32b_x32(tmem_base + lane_base + a_col0 + s * 32, o);
-            tmem_wait_st();
-          } else {
-            const int nl = t & 63, kb = t >> 6;
-            const uint32_t pa = smem_u32(pk_s + s * 4096 + nl * 64 + kb * 32);
-            const uint4 p0 = lds128(pa), p1 = lds128(pa + 16);
-            dequant64(make_table(P.code, s1), p0, p1, o);
-            const uint32_t row = smem_u32(a_s + s * 16384) + kb * 8192 + (nl >> 3) * 1024 + (nl & 7) * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-              sts128(row + ((c ^ (nl & 7)) << 4), o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
-            fence_proxy_async_smem();
-          }
-          tc_fence_before();
+          const int sp = int(ks % SP);
+          if (!(ok = mbar_wait(&p_full[sp], uint32_t(ks / SP) & 1u, a.status, abort_flag))) break;
+          const uint32_t pa = BWD ? smem_u32(pk_s + sp * 4096 + (t & 63) * 64 + (t >> 6) * 32)
+                                  : smem_u32(pk_s + sp * 4096 + t * 32);
+          const uint4 p0 = lds128(pa), p1 = lds128(pa + 16);
           __syncwarp();
-          if (lane == 0) mbar_arrive(&afull[s]);
+          if (lane == 0) mbar_arrive(&p_empty[sp]);
+          dequant64(make_table(P.code, e4m3_to_f32(cq[j]) * cc[j]), p0, p1, o);
         } else if (!BWD) {
           // low-rank step: column n of B (rank chunk c) is row n of the A operand
-          const int l = int(ks - my_main);
-          const int c = l % (a.rp / 64);
+          const int c = int(ks - my_main) % (a.rp / 64);
           const int64_t n = w0 + t;
-          uint32_t o[32];
 #pragma unroll 8
           for (int i = 0; i < 32; ++i) {
             const int j0 = c * 64 + 2 * i;
@@ -337,12 +338,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
                 (n < a.N && j0 + 1 < a.r) ? uint32_t(__ldg(a.lora_w + int64_t(j0 + 1) * a.N + n)) : 0u;
             o[i] = lo | (hi << 16);
           }
-          if (!(ok = mbar_wait(&full[s], ph, a.status, abort_flag))) break;
-          tmem_st_32x32b_x32(tmem_base + lane_base + a_col0 + s * 32, o);
+        }
+        // the A slot must have been released by the MMA of step ks - SA
+        if (ks >= SA && !(ok = mbar_wait(&a_empty[sa], a_ph ^ 1u, a.status, abort_flag))) break;
+        if (!BWD) {
+          tmem_st_32x32b_x32(tmem_base + lane_base + a_col0 + sa * 32, o);
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&afull[s]);
+          if (lane == 0) mbar_arrive(&a_full[sa]);
+        } else if (ks < my_main) {
+          const int nl = t & 63, kb = t >> 6;
+          const uint32_t row = smem_u32(a_s + sa * 16384) + kb * 8192 + (nl >> 3) * 1024 + (nl & 7) * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            sts128(row + ((c ^ (nl & 7)) << 4), o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&a_full[sa]);
+        } else {
+          // backward low-rank step: the A-factor tile A[k0:k0+128, chunk] by TMA
+          __syncwarp();
+          if (lane == 0) {
+            if ((warp & 3) == 0) {
+              const int c = int(ks - my_main) % (a.rp / 64);
+              mbar_arrive_expect_tx(&a_full[sa], 16384u);
+              tma_load_2d(a_s + sa * 16384, &P.tm_lw, &a_full[sa], int32_t(c * 64), int32_t(w0));
+            } else {
+              mbar_arrive(&a_full[sa]);
+            }
+          }
         }
       }
 #pragma unroll
@@ -358,7 +383,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
     const int nchunks = bt / 32;
     const bool got_acc = ok && mbar_wait(accf, 0, a.status, abort_flag);
     if (got_acc) tc_fence_after();
-    float* red = reinterpret_cast<float*>(act_s);   // split partial [bt][128] (stages are free now)
+    float* red = reinterpret_cast<float*>(act_s);   // split partial [bt][128] (the X ring is free now)
     for (int c = wg; c < nchunks; c += kDequantWGs) {
       uint32_t v[32];
       if (got_acc) {
@@ -721,7 +746,10 @@ static cudaError_t launch_clustered(void (*kern)(const Params), dim3 grid, dim3 
 }
 
 static size_t nf4_gemm_smem(int backward, int bt) {
-  return 1024 + size_t(kStages) * (size_t(bt) * 128 + 4096 + (backward ? 16384 : 0)) + 256;
+  const size_t x = size_t(bt) * 128;
+  if (backward)
+    return 1024 + Rings<true>::SX * x + Rings<true>::SP * 4096 + Rings<true>::SA * 16384 + 512;
+  return 1024 + Rings<false>::SX * x + Rings<false>::SP * 4096 + 512;
 }
 static size_t skinny_smem() { return 1024 + size_t(kSkinnyStages) * (16384 + 32768) + 256; }
 
