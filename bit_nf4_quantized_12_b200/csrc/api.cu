@@ -4,7 +4,7 @@
 #include <cstring>
 #include <cuda_runtime.h>
 
-#include "../../include/qlora_nf4.h"
+#include "qlora_nf4.h"
 #include "format.h"
 #include "kernels.h"
 

@@ -19,7 +19,6 @@ namespace nf4 {
 // ----------------------------------------------------------------------------
 constexpr uint32_t kStatusNonfinite = 1u;   // quantize saw NaN or Inf in W
 constexpr uint32_t kStatusTimeout   = 2u;   // a bounded wait gave up
-constexpr uint64_t kWaitLimitNs     = 2000000000ull;  // 2 s per wait
 
 NF4_DEV uint64_t globaltimer_ns() {
   uint64_t t;
@@ -69,18 +68,25 @@ NF4_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 // Wait for the phase with the given parity to complete.  Gives up after
-// kWaitLimitNs, sets kStatusTimeout in *err (if any) and returns false, so a
-// lost arrival can never hang the GPU.  Once any wait has failed (*abort set
-// in shared memory), later waits return false at once.
+// about kWaitLimitCycles SM cycles (~2 s), sets kStatusTimeout in *err (if
+// any) and returns false, so a lost arrival can never hang the GPU.  Once any
+// wait has failed (*abort set in shared memory), later waits return false at
+// once.  The time bound uses the SM cycle counter, read only every 1024
+// polls, so a wait that succeeds within a few microseconds costs no timer
+// reads.
+constexpr long long kWaitLimitCycles = 4000000000ll;
 NF4_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err, volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
+  long long t0 = -1;
   uint32_t spins = 0;
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (((++spins) & 255u) == 0u) {
+    if (((++spins) & 1023u) == 0u) {
       if (abort_flag != nullptr && *abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      const long long now = clock64();
+      if (t0 < 0) {
+        t0 = now;
+      } else if (now - t0 > kWaitLimitCycles) {
         if (err) atomicOr(err, kStatusTimeout);
         if (abort_flag) *abort_flag = 1;
         return false;
@@ -219,6 +225,15 @@ NF4_DEV uint32_t cluster_ctarank() {
 // release/acquire ordering of shared::cluster accesses around it).
 NF4_DEV void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+// Address of `local`'s counterpart in the shared memory of CTA `rank`.
+NF4_DEV uint32_t dsmem_addr(const void* local, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+  return remote;
+}
+NF4_DEV void st_dsmem_f32(uint32_t remote, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
 }
 // fp32 load from the shared memory of CTA `rank` of this cluster, at the
 // address that `local` has in this CTA.

@@ -50,7 +50,7 @@ struct Nf4GemmParams {
   CUtensorMap tm_act;   // X [M,K] / dY [M,N], bf16, box {64, bt}, 128B swizzle
   CUtensorMap tm_pk;    // packed [N, K/2] bytes; box {32,128} fwd, {64,64} bwd
   CUtensorMap tm_lact;  // hi/lo [M, 2rp] bf16, box {64, bt}, 128B swizzle
-  CUtensorMap tm_lw;    // backward: A [K, r] bf16, box {64, 128}, 128B swizzle
+  CUtensorMap tm_lw;    // forward: B [r, N], box {64, 64}; backward: A [K, r], box {64, 128}; 128B swizzle
   Nf4GemmArgs a;
   CodeTable code;
   int bt;
@@ -116,31 +116,24 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, ui
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
-// Wait ignoring the abort flag (used only to drain in-flight copies/MMAs).
+// Wait ignoring the abort flag (used only to drain in-flight copies/MMAs),
+// bounded to ~100 ms of SM cycles.
 __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
-  const uint64_t t0 = globaltimer_ns();
+  const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > 100000000ull) break;   // 100 ms
+    if (clock64() - t0 > 200000000ll) break;
   }
 }
 
 // Ring depths.  X: the activation tile ring (TMA), P: packed NF4 tiles (TMA,
 // 4 KB each, recycled as soon as a dequant warpgroup has read them), A: the
-// dequantized weight operand (tensor memory in the forward pass, shared
-// memory in the backward pass).  The dequant warps compute a step before they
-// wait for its A slot, so they run ahead of the tensor core by up to SA steps.
-template <bool BWD> struct Rings;
-template <> struct Rings<false> { static constexpr int SX = 5, SP = 12, SA = 8; };
-template <> struct Rings<true>  { static constexpr int SX = 4, SP = 8,  SA = 4; };
-
-// Forward tensor memory: accumulator in columns [0, a_col0), the SA
-// 32-column A slots after it.
-__host__ __device__ constexpr int fwd_a_col0(int bt) { return bt <= 128 ? 128 : 256; }
-constexpr uint32_t kFwdTmemCols = 512;
+// dequantized weight operand in shared memory (16 KB per step).  The dequant
+// warps compute a step before they wait for its A slot, so they run ahead of
+// the tensor core by up to SA steps.
+constexpr int SX = 4, SP = 8, SA = 4;
 
 template <bool BWD>
 __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_constant__ Nf4GemmParams P) {
-  constexpr int SX = Rings<BWD>::SX, SP = Rings<BWD>::SP, SA = Rings<BWD>::SA;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const Nf4GemmArgs& a = P.a;
@@ -148,8 +141,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
   const uint32_t act_bytes = uint32_t(bt) * 128u;
   uint8_t* act_s = smem;                                   // SX x act_bytes
   uint8_t* pk_s = act_s + SX * act_bytes;                  // SP x 4096
-  uint8_t* a_s = pk_s + SP * 4096;                         // backward: SA x 16384
-  uint64_t* bars = reinterpret_cast<uint64_t*>(a_s + (BWD ? SA * 16384 : 0));
+  uint8_t* a_s = pk_s + SP * 4096;                         // SA x 16384
+  uint64_t* bars = reinterpret_cast<uint64_t*>(a_s + SA * 16384);
   uint64_t* x_full = bars;
   uint64_t* x_empty = x_full + SX;
   uint64_t* p_full = x_empty + SX;
@@ -172,8 +165,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
   const int my_lora = (split == 0) ? P.lora_steps : 0;
   const int64_t nsteps = my_main + my_lora;
   const int64_t KB = a.K / kBlock;          // NF4 blocks per W row
-  const uint32_t tmem_cols = BWD ? uint32_t(bt < 32 ? 32 : bt) : kFwdTmemCols;
-  const uint32_t a_col0 = uint32_t(fwd_a_col0(bt));
+  const uint32_t tmem_cols = uint32_t(bt < 32 ? 32 : bt);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < SX; ++s) { mbar_init(&x_full[s], 1); mbar_init(&x_empty[s], 1); }
@@ -224,6 +216,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
     // ------------------------------------------------------------ packed-W producer
     if (elect_one()) {
       tma_prefetch_desc(&P.tm_pk);
+      tma_prefetch_desc(&P.tm_lw);
       int64_t issued = 0;
       for (int64_t ks = 0; ks < my_main; ++ks) {
         const int s = int(ks % SP);
@@ -243,8 +236,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    const uint32_t idesc_main = make_idesc_bf16(128, bt, BWD ? 1 : 0, 0);
-    const uint32_t idesc_lora = make_idesc_bf16(128, bt, 0, 0);
+    // A operand layouts: forward main steps K-major (rows of W), backward
+    // main steps MN-major (columns of W), forward low-rank steps MN-major
+    // (B^T by TMA), backward low-rank steps K-major (A by TMA).
+    const uint32_t idesc_k = make_idesc_bf16(128, bt, 0, 0);
+    const uint32_t idesc_mn = make_idesc_bf16(128, bt, 1, 0);
     for (int64_t ks = 0; ks < nsteps; ++ks) {
       const int sx = int(ks % SX), sa = int(ks % SA);
       if (!mbar_wait(&x_full[sx], uint32_t(ks / SX) & 1u, a.status, abort_flag)) break;
@@ -253,17 +249,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
       if (elect_one()) {
         const uint32_t act_addr = smem_u32(act_s + sx * act_bytes);
         const uint32_t a_addr = smem_u32(a_s + sa * 16384);
+        const bool a_mn = (ks < my_main) == BWD;
+        const uint32_t idesc = a_mn ? idesc_mn : idesc_k;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t bdesc = make_sdesc_sw128(act_addr + kk * 32, 16, 1024);
-          const uint32_t acc = (ks > 0 || kk > 0) ? 1u : 0u;
-          if (!BWD) {
-            mma_ts(tmem_base, tmem_base + a_col0 + sa * 32 + kk * 8, bdesc, idesc_main, acc);
-          } else if (ks < my_main) {
-            mma_ss(tmem_base, make_sdesc_sw128(a_addr + kk * 2048, 8192, 1024), bdesc, idesc_main, acc);
-          } else {
-            mma_ss(tmem_base, make_sdesc_sw128(a_addr + kk * 32, 16, 1024), bdesc, idesc_lora, acc);
-          }
+          const uint64_t adesc = a_mn ? make_sdesc_sw128(a_addr + kk * 2048, 8192, 1024)
+                                      : make_sdesc_sw128(a_addr + kk * 32, 16, 1024);
+          mma_ss(tmem_base, adesc, bdesc, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(&x_empty[sx]);
         mma_commit(&a_empty[sa]);
@@ -281,8 +274,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
     // scales (c1q, c2) of its next four steps are loaded one window ahead so
     // their global-memory latency is off the critical path.
     const int wg = (warp - 4) >> 2;
-    const int t = threadIdx.x - 128 - 128 * wg;               // TMEM lane 0..127
-    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    const int t = threadIdx.x - 128 - 128 * wg;               // 0..127
     auto block_of = [&](int64_t ks) -> int64_t {              // NF4 block index used at step ks, or -1
       if (ks >= my_main) return -1;
       const int64_t g = g_begin + ks;
@@ -316,7 +308,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
         if (!ok || ks >= nsteps) break;
         const int sa = int(ks % SA);
         const uint32_t a_ph = uint32_t(ks / SA) & 1u;
-        uint32_t o[32];
         if (ks < my_main) {
           const int sp = int(ks % SP);
           if (!(ok = mbar_wait(&p_full[sp], uint32_t(ks / SP) & 1u, a.status, abort_flag))) break;
@@ -325,45 +316,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
           const uint4 p0 = lds128(pa), p1 = lds128(pa + 16);
           __syncwarp();
           if (lane == 0) mbar_arrive(&p_empty[sp]);
+          uint32_t o[32];
           dequant64(make_table(P.code, e4m3_to_f32(cq[j]) * cc[j]), p0, p1, o);
-        } else if (!BWD) {
-          // low-rank step: column n of B (rank chunk c) is row n of the A operand
-          const int c = int(ks - my_main) % (a.rp / 64);
-          const int64_t n = w0 + t;
-#pragma unroll 8
-          for (int i = 0; i < 32; ++i) {
-            const int j0 = c * 64 + 2 * i;
-            const uint32_t lo = (n < a.N && j0 < a.r) ? uint32_t(__ldg(a.lora_w + int64_t(j0) * a.N + n)) : 0u;
-            const uint32_t hi =
-                (n < a.N && j0 + 1 < a.r) ? uint32_t(__ldg(a.lora_w + int64_t(j0 + 1) * a.N + n)) : 0u;
-            o[i] = lo | (hi << 16);
-          }
-        }
-        // the A slot must have been released by the MMA of step ks - SA
-        if (ks >= SA && !(ok = mbar_wait(&a_empty[sa], a_ph ^ 1u, a.status, abort_flag))) break;
-        if (!BWD) {
-          tmem_st_32x32b_x32(tmem_base + lane_base + a_col0 + sa * 32, o);
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&a_full[sa]);
-        } else if (ks < my_main) {
-          const int nl = t & 63, kb = t >> 6;
-          const uint32_t row = smem_u32(a_s + sa * 16384) + kb * 8192 + (nl >> 3) * 1024 + (nl & 7) * 128;
+          // the A slot must have been released by the MMA of step ks - SA
+          if (ks >= SA && !(ok = mbar_wait(&a_empty[sa], a_ph ^ 1u, a.status, abort_flag))) break;
+          // forward: row t of Wd (K-major, 128-byte rows); backward: row
+          // t%64 of the MN atom t/64 (64 weights along k)
+          const int row_i = BWD ? (t & 63) : t;
+          const uint32_t row = smem_u32(a_s + sa * 16384) + (BWD ? (t >> 6) * 8192 : 0) + (row_i >> 3) * 1024 +
+                               (row_i & 7) * 128;
 #pragma unroll
           for (int c = 0; c < 8; ++c)
-            sts128(row + ((c ^ (nl & 7)) << 4), o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+            sts128(row + ((c ^ (row_i & 7)) << 4), o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive(&a_full[sa]);
         } else {
-          // backward low-rank step: the A-factor tile A[k0:k0+128, chunk] by TMA
+          // low-rank step: the A operand is a tile of a LoRA factor, by TMA
+          // (forward: B^T [128 features x 64 ranks], two MN-major boxes;
+          //  backward: A [128 inputs x 64 ranks], one K-major box)
+          if (ks >= SA && !(ok = mbar_wait(&a_empty[sa], a_ph ^ 1u, a.status, abort_flag))) break;
           __syncwarp();
           if (lane == 0) {
             if ((warp & 3) == 0) {
               const int c = int(ks - my_main) % (a.rp / 64);
+              uint8_t* dst = a_s + sa * 16384;
               mbar_arrive_expect_tx(&a_full[sa], 16384u);
-              tma_load_2d(a_s + sa * 16384, &P.tm_lw, &a_full[sa], int32_t(c * 64), int32_t(w0));
+              if (!BWD) {
+                tma_load_2d(dst, &P.tm_lw, &a_full[sa], int32_t(w0), int32_t(c * 64));
+                tma_load_2d(dst + 8192, &P.tm_lw, &a_full[sa], int32_t(w0 + 64), int32_t(c * 64));
+              } else {
+                tma_load_2d(dst, &P.tm_lw, &a_full[sa], int32_t(c * 64), int32_t(w0));
+              }
             } else {
               mbar_arrive(&a_full[sa]);
             }
@@ -378,6 +362,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
     }
 
     // ------------------------------------------------------------ epilogue
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     const int64_t wdim = BWD ? a.K : a.N;       // extent of the W dimension of the output
     const int64_t i = w0 + t;
     const int nchunks = bt / 32;
@@ -491,14 +476,14 @@ __device__ __forceinline__ void skinny_finish(const SkinnyParams& P, int64_t i, 
   }
 }
 
-__global__ void __launch_bounds__(kSkinnyThreads, 1) skinny_gemm_kernel(const __grid_constant__ SkinnyParams P) {
+__global__ void __launch_bounds__(kSkinnyThreads, 2) skinny_gemm_kernel(const __grid_constant__ SkinnyParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const SkinnyArgs& a = P.a;
   const int rp = a.rp;
   const uint32_t b_bytes = uint32_t(rp) * 128u;
   constexpr uint32_t a_bytes = 16384u;
-  const uint32_t stage_bytes = a_bytes + 32768u;
+  const uint32_t stage_bytes = a_bytes + b_bytes;   // multiple of 8 KB: stages stay 1024-aligned
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSkinnyStages * stage_bytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + kSkinnyStages;
@@ -604,7 +589,11 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1) skinny_gemm_kernel(const __
     const int64_t i = i0 + t;
     const bool got = nsteps > 0 && mbar_wait(accf, 0, a.status, abort_flag);
     if (got) tc_fence_after();
-    float* red = reinterpret_cast<float*>(smem);   // split partial [rp][128]
+    // Split partials stay in this CTA's shared memory ([rp][128] floats over
+    // the now idle stage ring); after one cluster barrier each CTA pulls its
+    // slice of columns from every CTA of the cluster, 8 columns x 8 CTAs of
+    // loads in flight at a time, and sums them in a fixed order.
+    float* red = reinterpret_cast<float*>(smem);
     for (int c = 0; c < rp / 32; ++c) {
       uint32_t v[32];
       if (got) {
@@ -630,14 +619,22 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1) skinny_gemm_kernel(const __
       const int t = (warp & 3) * 32 + (threadIdx.x & 31);
       const int64_t i = i0 + t;
       const float* red = reinterpret_cast<const float*>(smem);
-      const int jps = rp / P.splits;
+      const int jps = rp / P.splits;                 // multiple of 8 (rp % 64 == 0, splits <= 8)
       const int j0 = int(cluster_ctarank()) * jps;
-      for (int j = j0; j < j0 + jps; ++j) {
-        float acc = 0.0f;
+      for (int jb = 0; jb < jps; jb += 8) {
+        float part[8][8];
 #pragma unroll
-        for (int qq = 0; qq < 8; ++qq)
-          if (qq < P.splits) acc += ld_dsmem_f32(red + j * 128 + t, uint32_t(qq));
-        skinny_finish(P, i, j, acc);
+        for (int jj = 0; jj < 8; ++jj)
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            part[jj][q] = (q < P.splits) ? ld_dsmem_f32(red + (j0 + jb + jj) * 128 + t, uint32_t(q)) : 0.0f;
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          float acc = 0.0f;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) acc += part[jj][q];
+          skinny_finish(P, i, j0 + jb + jj, acc);
+        }
       }
     }
     cluster_sync_all();
@@ -723,7 +720,7 @@ SkinnyPlan plan_skinny(int kind, int64_t M, int64_t N, int64_t K, int r, int num
     default: p.rows = N; p.red = M; p.steps = cdiv(M, 64); break;
   }
   p.tiles = cdiv(p.rows, 128);
-  p.splits = choose_splits(p.tiles, p.steps, num_sms, 2, (num_sms * 7) / 8);
+  p.splits = choose_splits(p.tiles, p.steps, 2 * num_sms, 2, (2 * num_sms * 7) / 8);
   return p;
 }
 
@@ -745,13 +742,10 @@ static cudaError_t launch_clustered(void (*kern)(const Params), dim3 grid, dim3 
   return cudaLaunchKernelEx(&cfg, kern, P);
 }
 
-static size_t nf4_gemm_smem(int backward, int bt) {
-  const size_t x = size_t(bt) * 128;
-  if (backward)
-    return 1024 + Rings<true>::SX * x + Rings<true>::SP * 4096 + Rings<true>::SA * 16384 + 512;
-  return 1024 + Rings<false>::SX * x + Rings<false>::SP * 4096 + 512;
+static size_t nf4_gemm_smem(int /*backward*/, int bt) {
+  return 1024 + size_t(SX) * bt * 128 + size_t(SP) * 4096 + size_t(SA) * 16384 + 512;
 }
-static size_t skinny_smem() { return 1024 + size_t(kSkinnyStages) * (16384 + 32768) + 256; }
+static size_t skinny_smem(int rp) { return 1024 + size_t(kSkinnyStages) * (16384 + size_t(rp) * 128) + 256; }
 
 cudaError_t launch_nf4_gemm(const Nf4GemmPlan& plan, const Nf4GemmArgs& a, cudaStream_t stream) {
   Nf4GemmParams P;
@@ -773,6 +767,7 @@ cudaError_t launch_nf4_gemm(const Nf4GemmPlan& plan, const Nf4GemmArgs& a, cudaS
   if (!plan.backward) {
     ok &= encode_tmap_2d(&P.tm_act, BF, a.act, K, M, K * 2, 64, plan.bt, SW);
     ok &= encode_tmap_2d(&P.tm_pk, U8, a.packed, K / 2, N, K / 2, 32, 128, NOSW);
+    ok &= encode_tmap_2d(&P.tm_lw, BF, a.lora_w, N, uint64_t(a.r), N * 2, 64, 64, SW);
   } else {
     ok &= encode_tmap_2d(&P.tm_act, BF, a.act, N, M, N * 2, 64, plan.bt, SW);
     ok &= encode_tmap_2d(&P.tm_pk, U8, a.packed, K / 2, N, K / 2, 64, 64, NOSW);
@@ -825,7 +820,7 @@ cudaError_t launch_skinny(const SkinnyPlan& plan, const SkinnyArgs& a, cudaStrea
       break;
   }
   if (!ok) return cudaErrorInvalidValue;
-  const size_t smem = skinny_smem();
+  const size_t smem = skinny_smem(a.rp);
   cudaError_t e = cudaFuncSetAttribute(skinny_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(unsigned(plan.tiles), unsigned(plan.splits));
