@@ -232,8 +232,9 @@ NF4_DEV uint32_t dsmem_addr(const void* local, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
   return remote;
 }
-NF4_DEV void st_dsmem_f32(uint32_t remote, float v) {
-  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
+NF4_DEV void st_dsmem_f32x4(uint32_t remote, float a, float b, float c, float d) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(remote), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
 }
 // fp32 load from the shared memory of CTA `rank` of this cluster, at the
 // address that `local` has in this CTA.

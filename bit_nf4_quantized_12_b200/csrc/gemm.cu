@@ -40,7 +40,7 @@ namespace {
 constexpr int kDequantWGs = 4;                          // dequant / epilogue warpgroups
 constexpr int kGemmThreads = 128 + 128 * kDequantWGs;   // + producer, MMA, allocator, spare warp
 constexpr int kSkinnyThreads = 192;
-constexpr int kSkinnyStages = 4;
+constexpr int kSkinnyStages = 2;
 
 struct CodeTable {
   float v[16];
@@ -167,6 +167,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
   const int64_t KB = a.K / kBlock;          // NF4 blocks per W row
   const uint32_t tmem_cols = uint32_t(bt < 32 ? 32 : bt);
 
+  if (threadIdx.x == 32) {   // descriptor fetches overlap the setup below
+    tma_prefetch_desc(&P.tm_act);
+    tma_prefetch_desc(&P.tm_lact);
+    tma_prefetch_desc(&P.tm_pk);
+    tma_prefetch_desc(&P.tm_lw);
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < SX; ++s) { mbar_init(&x_full[s], 1); mbar_init(&x_empty[s], 1); }
     for (int s = 0; s < SP; ++s) { mbar_init(&p_full[s], 1); mbar_init(&p_empty[s], 4); }
@@ -187,8 +193,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
   if (warp == 0) {
     // ------------------------------------------------------------ X producer
     if (elect_one()) {
-      tma_prefetch_desc(&P.tm_act);
-      tma_prefetch_desc(&P.tm_lact);
       int64_t issued = 0;
       for (int64_t ks = 0; ks < nsteps; ++ks) {
         const int s = int(ks % SX);
@@ -215,8 +219,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
   } else if (warp == 3) {
     // ------------------------------------------------------------ packed-W producer
     if (elect_one()) {
-      tma_prefetch_desc(&P.tm_pk);
-      tma_prefetch_desc(&P.tm_lw);
       int64_t issued = 0;
       for (int64_t ks = 0; ks < my_main; ++ks) {
         const int s = int(ks % SP);
@@ -407,13 +409,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
       const float* red = reinterpret_cast<const float*>(act_s);
       const int cps = bt / P.splits;
       const int c0 = int(cluster_ctarank()) * cps;
-      for (int col = c0 + wg; col < c0 + cps; col += kDequantWGs) {
-        float acc = 0.0f;
+      for (int col = c0 + wg; col < c0 + cps; col += 4 * kDequantWGs) {
+        float part[4][8];
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          if (q < P.splits) acc += ld_dsmem_f32(red + col * 128 + t, uint32_t(q));
-        const int64_t m = m0 + col;
-        if (i < wdim && m < a.M) a.out[m * wdim + i] = uint16_t(pack_bf16x2(acc, 0.0f) & 0xFFFFu);
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int cu = col + u * kDequantWGs;
+            part[u][q] = (q < P.splits && cu < c0 + cps) ? ld_dsmem_f32(red + cu * 128 + t, uint32_t(q)) : 0.0f;
+          }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          float acc = 0.0f;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) acc += part[u][q];
+          const int cu = col + u * kDequantWGs;
+          const int64_t m = m0 + cu;
+          if (cu < c0 + cps && i < wdim && m < a.M) a.out[m * wdim + i] = uint16_t(pack_bf16x2(acc, 0.0f) & 0xFFFFu);
+        }
       }
     }
     cluster_sync_all();
@@ -444,34 +457,62 @@ struct SkinnyParams {
 
 __device__ __forceinline__ uint32_t bf16_bits(float x) { return pack_bf16x2(x, 0.0f) & 0xFFFFu; }
 
-__device__ __forceinline__ void skinny_finish(const SkinnyParams& P, int64_t i, int j, float acc) {
+// Final values of eight consecutive columns j0..j0+7 of row i (j0 % 8 == 0):
+// one 16-byte store per output row segment where the row holds all eight.
+__device__ __forceinline__ void skinny_finish8(const SkinnyParams& P, int64_t i, int j0, const float (&acc)[8]) {
   const SkinnyArgs& a = P.a;
   switch (P.kind) {
-    case kSkinnyT: {
-      if (i >= a.M) return;
-      const uint32_t tb = bf16_bits(acc);                 // T in the bf16 compute type
-      if (j < a.r && a.T_out) a.T_out[i * a.r + j] = uint16_t(tb);
-      const float v = (j < a.r) ? a.s * __uint_as_float(tb << 16) : 0.0f;
-      const uint32_t hi = bf16_bits(v);
-      const uint32_t lo = bf16_bits(v - __uint_as_float(hi << 16));
-      a.hilo_out[i * 2 * a.rp + j] = uint16_t(hi);
-      a.hilo_out[i * 2 * a.rp + a.rp + j] = uint16_t(lo);
-      break;
-    }
+    case kSkinnyT:
     case kSkinnyG: {
       if (i >= a.M) return;
-      const float v = (j < a.r) ? a.s * acc : 0.0f;
-      const uint32_t hi = bf16_bits(v);
-      const uint32_t lo = bf16_bits(v - __uint_as_float(hi << 16));
-      a.hilo_out[i * 2 * a.rp + j] = uint16_t(hi);
-      a.hilo_out[i * 2 * a.rp + a.rp + j] = uint16_t(lo);
+      uint32_t hi[4], lo[4], tb[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        float v[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int j = j0 + 2 * u + h;
+          if (P.kind == kSkinnyT) {
+            const float tval = __uint_as_float(bf16_bits(acc[2 * u + h]) << 16);   // T in bf16
+            v[h] = (j < a.r) ? a.s * tval : 0.0f;
+          } else {
+            v[h] = (j < a.r) ? a.s * acc[2 * u + h] : 0.0f;
+          }
+        }
+        tb[u] = pack_bf16x2(acc[2 * u], acc[2 * u + 1]);
+        hi[u] = pack_bf16x2(v[0], v[1]);
+        const float h0 = __uint_as_float(hi[u] << 16), h1 = __uint_as_float(hi[u] & 0xFFFF0000u);
+        lo[u] = pack_bf16x2(v[0] - h0, v[1] - h1);
+      }
+      uint16_t* row = a.hilo_out + i * 2 * a.rp;
+      *reinterpret_cast<uint4*>(row + j0) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(row + a.rp + j0) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      if (P.kind == kSkinnyT && a.T_out != nullptr) {
+        if (j0 + 8 <= a.r) {
+          *reinterpret_cast<uint4*>(a.T_out + i * a.r + j0) = make_uint4(tb[0], tb[1], tb[2], tb[3]);
+        } else {
+          for (int u = 0; u < 8 && j0 + u < a.r; ++u)
+            a.T_out[i * a.r + j0 + u] = uint16_t((u & 1) ? (tb[u >> 1] >> 16) : (tb[u >> 1] & 0xFFFFu));
+        }
+      }
       break;
     }
-    case kSkinnyDA:
-      if (i < a.K && j < a.r) a.f32_out[i * a.r + j] = acc;
+    case kSkinnyDA: {
+      if (i >= a.K) return;
+      float* row = a.f32_out + i * a.r;
+      if (j0 + 8 <= a.r) {
+        *reinterpret_cast<float4*>(row + j0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *reinterpret_cast<float4*>(row + j0 + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+      } else {
+        for (int u = 0; u < 8 && j0 + u < a.r; ++u) row[j0 + u] = acc[u];
+      }
       break;
-    default:  // kSkinnyDB: computed as dB^T
-      if (i < a.N && j < a.r) a.f32_out[int64_t(j) * a.N + i] = a.s * acc;
+    }
+    default:  // kSkinnyDB, computed as dB^T: column j of dB^T is row j of dB
+      if (i >= a.N) return;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (j0 + u < a.r) a.f32_out[int64_t(j0 + u) * a.N + i] = a.s * acc[u];
       break;
   }
 }
@@ -484,7 +525,9 @@ __global__ void __launch_bounds__(kSkinnyThreads, 2) skinny_gemm_kernel(const __
   const uint32_t b_bytes = uint32_t(rp) * 128u;
   constexpr uint32_t a_bytes = 16384u;
   const uint32_t stage_bytes = a_bytes + b_bytes;   // multiple of 8 KB: stages stay 1024-aligned
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSkinnyStages * stage_bytes);
+  float* recv = reinterpret_cast<float*>(smem + kSkinnyStages * stage_bytes);   // [splits][128][rp/splits]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSkinnyStages * stage_bytes +
+                                               (P.splits > 1 ? uint32_t(rp) * 512u : 0u));
   uint64_t* full = bars;
   uint64_t* empty = bars + kSkinnyStages;
   uint64_t* accf = bars + 2 * kSkinnyStages;
@@ -501,6 +544,10 @@ __global__ void __launch_bounds__(kSkinnyThreads, 2) skinny_gemm_kernel(const __
   const int64_t nsteps = g_end > g_begin ? g_end - g_begin : 0;
   const uint32_t tmem_cols = rp <= 32 ? 32u : (rp <= 64 ? 64u : (rp <= 128 ? 128u : 256u));
 
+  if (threadIdx.x == 32) {
+    tma_prefetch_desc(&P.tm_a);
+    tma_prefetch_desc(&P.tm_b);
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSkinnyStages; ++s) {
       mbar_init(&full[s], 1);
@@ -521,8 +568,6 @@ __global__ void __launch_bounds__(kSkinnyThreads, 2) skinny_gemm_kernel(const __
 
   if (warp == 0) {
     if (elect_one()) {
-      tma_prefetch_desc(&P.tm_a);
-      tma_prefetch_desc(&P.tm_b);
       int64_t issued = 0;
       for (int64_t ks = 0; ks < nsteps; ++ks) {
         const int s = int(ks % kSkinnyStages);
@@ -589,11 +634,12 @@ __global__ void __launch_bounds__(kSkinnyThreads, 2) skinny_gemm_kernel(const __
     const int64_t i = i0 + t;
     const bool got = nsteps > 0 && mbar_wait(accf, 0, a.status, abort_flag);
     if (got) tc_fence_after();
-    // Split partials stay in this CTA's shared memory ([rp][128] floats over
-    // the now idle stage ring); after one cluster barrier each CTA pulls its
-    // slice of columns from every CTA of the cluster, 8 columns x 8 CTAs of
-    // loads in flight at a time, and sums them in a fixed order.
-    float* red = reinterpret_cast<float*>(smem);
+    // Split partials: each CTA of the cluster owns rp/splits columns; every
+    // CTA pushes its partial of those columns into the owner's receive
+    // buffer with 16-byte remote stores (no round trips), then one cluster
+    // barrier, then the owner sums the slices in a fixed order.
+    const int jps = rp / P.splits;
+    const uint32_t me = P.splits > 1 ? cluster_ctarank() : 0u;
     for (int c = 0; c < rp / 32; ++c) {
       uint32_t v[32];
       if (got) {
@@ -605,10 +651,21 @@ __global__ void __launch_bounds__(kSkinnyThreads, 2) skinny_gemm_kernel(const __
       }
       if (P.splits == 1) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) skinny_finish(P, i, c * 32 + j, __uint_as_float(v[j]));
+        for (int j8 = 0; j8 < 32; j8 += 8) {
+          float acc[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) acc[u] = __uint_as_float(v[j8 + u]);
+          skinny_finish8(P, i, c * 32 + j8, acc);
+        }
       } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) red[(c * 32 + j) * 128 + t] = __uint_as_float(v[j]);
+        for (int j = 0; j < 32; j += 4) {
+          const int jj = c * 32 + j;
+          const int owner = jj / jps;
+          float* slot = recv + (int(me) * 128 + t) * jps + (jj - owner * jps);
+          st_dsmem_f32x4(dsmem_addr(slot, uint32_t(owner)), __uint_as_float(v[j]), __uint_as_float(v[j + 1]),
+                         __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+        }
       }
     }
   }
@@ -618,26 +675,21 @@ __global__ void __launch_bounds__(kSkinnyThreads, 2) skinny_gemm_kernel(const __
     if (warp >= 2) {
       const int t = (warp & 3) * 32 + (threadIdx.x & 31);
       const int64_t i = i0 + t;
-      const float* red = reinterpret_cast<const float*>(smem);
-      const int jps = rp / P.splits;                 // multiple of 8 (rp % 64 == 0, splits <= 8)
+      const int jps = rp / P.splits;
       const int j0 = int(cluster_ctarank()) * jps;
-      for (int jb = 0; jb < jps; jb += 8) {
-        float part[8][8];
+      for (int jj = 0; jj < jps; jj += 8) {
+        float acc[8];
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj)
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            part[jj][q] = (q < P.splits) ? ld_dsmem_f32(red + (j0 + jb + jj) * 128 + t, uint32_t(q)) : 0.0f;
-#pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-          float acc = 0.0f;
-#pragma unroll
-          for (int q = 0; q < 8; ++q) acc += part[jj][q];
-          skinny_finish(P, i, j0 + jb + jj, acc);
+        for (int u = 0; u < 8; ++u) acc[u] = 0.0f;
+        for (int q = 0; q < P.splits; ++q) {
+          const float4* src = reinterpret_cast<const float4*>(recv + (q * 128 + t) * jps + jj);
+          const float4 x0 = src[0], x1 = src[1];
+          acc[0] += x0.x; acc[1] += x0.y; acc[2] += x0.z; acc[3] += x0.w;
+          acc[4] += x1.x; acc[5] += x1.y; acc[6] += x1.z; acc[7] += x1.w;
         }
+        skinny_finish8(P, i, j0 + jj, acc);
       }
     }
-    cluster_sync_all();
   }
 
   tc_fence_before();
@@ -745,7 +797,9 @@ static cudaError_t launch_clustered(void (*kern)(const Params), dim3 grid, dim3 
 static size_t nf4_gemm_smem(int /*backward*/, int bt) {
   return 1024 + size_t(SX) * bt * 128 + size_t(SP) * 4096 + size_t(SA) * 16384 + 512;
 }
-static size_t skinny_smem(int rp) { return 1024 + size_t(kSkinnyStages) * (16384 + size_t(rp) * 128) + 256; }
+static size_t skinny_smem(int rp, int splits) {
+  return 1024 + size_t(kSkinnyStages) * (16384 + size_t(rp) * 128) + (splits > 1 ? size_t(rp) * 512 : 0) + 256;
+}
 
 cudaError_t launch_nf4_gemm(const Nf4GemmPlan& plan, const Nf4GemmArgs& a, cudaStream_t stream) {
   Nf4GemmParams P;
@@ -820,7 +874,7 @@ cudaError_t launch_skinny(const SkinnyPlan& plan, const SkinnyArgs& a, cudaStrea
       break;
   }
   if (!ok) return cudaErrorInvalidValue;
-  const size_t smem = skinny_smem(a.rp);
+  const size_t smem = skinny_smem(a.rp, plan.splits);
   cudaError_t e = cudaFuncSetAttribute(skinny_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   dim3 grid(unsigned(plan.tiles), unsigned(plan.splits));
