@@ -67,21 +67,34 @@ NF4_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Same, but the thread may sleep in hardware until the phase completes (or
+// about `hint_ns` passes), so waiting warps leave the issue slots to others.
+NF4_DEV bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2, %3;\n\t"
+      "selp.b32 %0, 1, 0, P;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
 // Wait for the phase with the given parity to complete.  Gives up after
 // about kWaitLimitCycles SM cycles (~2 s), sets kStatusTimeout in *err (if
 // any) and returns false, so a lost arrival can never hang the GPU.  Once any
 // wait has failed (*abort set in shared memory), later waits return false at
-// once.  The time bound uses the SM cycle counter, read only every 1024
-// polls, so a wait that succeeds within a few microseconds costs no timer
-// reads.
+// once.  Each poll lets the thread sleep in hardware until the phase completes
+// (at most ~20 us), and the cycle counter is read every 16 polls, so waiting
+// costs almost no issue slots and the bound stays coarse but finite.
 constexpr long long kWaitLimitCycles = 4000000000ll;
 NF4_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err, volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   long long t0 = -1;
   uint32_t spins = 0;
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (((++spins) & 1023u) == 0u) {
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    if (((++spins) & 15u) == 0u) {
       if (abort_flag != nullptr && *abort_flag) return false;
       const long long now = clock64();
       if (t0 < 0) {

@@ -131,6 +131,11 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
 // warps compute a step before they wait for its A slot, so they run ahead of
 // the tensor core by up to SA steps.
 constexpr int SX = 4, SP = 8, SA = 4;
+// Each packed and operand slot must belong to a single dequant warpgroup
+// (slot = step mod ring size, warpgroup = step mod kDequantWGs).  Otherwise two
+// warpgroups share a slot, one can run two barrier phases ahead, and a parity
+// wait would pass on the wrong phase.
+static_assert(SP % kDequantWGs == 0 && SA % kDequantWGs == 0, "ring slots must map to one dequant warpgroup");
 
 template <bool BWD>
 __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_constant__ Nf4GemmParams P) {
