@@ -823,16 +823,17 @@ cudaError_t launch_nf4_gemm(const Nf4GemmPlan& plan, const Nf4GemmArgs& a, cudaS
   bool ok = true;
   const uint64_t M = a.M, N = a.N, K = a.K;
   const uint64_t hw = 2 * uint64_t(a.rp);
+  const uint32_t act_box = uint32_t(plan.bt);
   if (!plan.backward) {
-    ok &= encode_tmap_2d(&P.tm_act, BF, a.act, K, M, K * 2, 64, plan.bt, SW);
+    ok &= encode_tmap_2d(&P.tm_act, BF, a.act, K, M, K * 2, 64, act_box, SW);
     ok &= encode_tmap_2d(&P.tm_pk, U8, a.packed, K / 2, N, K / 2, 32, 128, NOSW);
     ok &= encode_tmap_2d(&P.tm_lw, BF, a.lora_w, N, uint64_t(a.r), N * 2, 64, 64, SW);
   } else {
-    ok &= encode_tmap_2d(&P.tm_act, BF, a.act, N, M, N * 2, 64, plan.bt, SW);
+    ok &= encode_tmap_2d(&P.tm_act, BF, a.act, N, M, N * 2, 64, act_box, SW);
     ok &= encode_tmap_2d(&P.tm_pk, U8, a.packed, K / 2, N, K / 2, 64, 64, NOSW);
     ok &= encode_tmap_2d(&P.tm_lw, BF, a.lora_w, uint64_t(a.r), K, uint64_t(a.r) * 2, 64, 128, SW);
   }
-  ok &= encode_tmap_2d(&P.tm_lact, BF, a.lora_act, hw, M, hw * 2, 64, plan.bt, SW);
+  ok &= encode_tmap_2d(&P.tm_lact, BF, a.lora_act, hw, M, hw * 2, 64, act_box, SW);
   if (!ok) return cudaErrorInvalidValue;
   const size_t smem = nf4_gemm_smem(plan.backward, plan.bt);
   dim3 grid(unsigned(plan.tiles_w), unsigned(plan.tiles_t), unsigned(plan.splits));
