@@ -41,6 +41,7 @@ SIGNATURES = {
     "qlora_linear_fwd": (ctypes.c_int, [_P, _I64, NF4Weight, _P, _P, _I32, _F, _P, _P, _P, _SZ, _P]),
     "qlora_linear_bwd": (ctypes.c_int, [_P, _P, _I64, NF4Weight, _P, _P, _I32, _F, _P, _P, _P, _P, _P,
                                         _SZ, _P]),
+    "qlora_linear_fwd_noalloc": (ctypes.c_int, [_P, _I64, NF4Weight, _P, _P, _I32, _F, _P, _P, _P]),
     "nf4_status_str": (ctypes.c_char_p, [ctypes.c_int]),
 }
 
@@ -154,6 +155,21 @@ def linear_fwd(X, qw: QuantizedWeight, A, B, s, ws=None, Y=None, T=None, want_T=
                                   _dev(B, torch.bfloat16, "B"), r, float(s), _dev(Y, torch.bfloat16, "Y"),
                                   None if T is None else _dev(T, torch.bfloat16, "T"),
                                   _dev(ws, torch.uint8, "ws"), ws.numel(), _stream()))
+    return Y, T
+
+
+def linear_fwd_noalloc(X, qw: QuantizedWeight, A, B, s, Y=None, T=None, want_T=True):
+    """linear_fwd with the library's fixed scratch array instead of a workspace;
+    returns (Y, T).  Y and T are allocated here unless given."""
+    M, K = X.shape
+    r = A.shape[1]
+    if Y is None:
+        Y = torch.empty(M, qw.rows, dtype=torch.bfloat16, device=X.device)
+    if T is None and want_T:
+        T = torch.empty(M, r, dtype=torch.bfloat16, device=X.device)
+    _check(lib().qlora_linear_fwd_noalloc(_dev(X, torch.bfloat16, "X"), M, qw.abi(), _dev(A, torch.bfloat16, "A"),
+                                          _dev(B, torch.bfloat16, "B"), r, float(s), _dev(Y, torch.bfloat16, "Y"),
+                                          None if T is None else _dev(T, torch.bfloat16, "T"), _stream()))
     return Y, T
 
 

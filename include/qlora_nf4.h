@@ -118,6 +118,33 @@ nf4_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, nf
                             const uint16_t* B, int32_t r, float s, const uint16_t* T, uint16_t* dX, float* dA,
                             float* dB, void* ws, size_t ws_bytes, void* stream);
 
+/* Size of the fixed scratch array behind qlora_linear_fwd_noalloc (4 MiB per
+ * device, part of the library's device image). */
+#define QLORA_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/* qlora_linear_fwd with no workspace argument and no allocation.  The pages
+ * have no counterpart: this is an integration entry point, not part of the
+ * method.  Results equal those of qlora_linear_fwd with the same arguments.
+ * Who needs it: callers that cannot allocate device memory at the point of
+ * the call.  Examples are a decode loop driven from C with a device-memory
+ * budget fixed at start-up (cudaMalloc / cudaFree would synchronize the
+ * device between tokens and can fail once the budget is committed), and
+ * hosts that only hand out input and output buffers.  The scratch is a
+ * fixed device array of QLORA_NOALLOC_SCRATCH_BYTES per device:
+ *  - the first call on a device, with that device current, does a one-time
+ *    set-up (looks up the array's device address); make it before any
+ *    stream capture begins;
+ *  - when qlora_workspace_bytes(M, N, K, r) exceeds
+ *    QLORA_NOALLOC_SCRATCH_BYTES the call returns NF4_ERR_WORKSPACE and
+ *    launches nothing (at r = 64 that allows M up to 10922 tokens);
+ *  - the status word is cleared on the stream by each call;
+ *  - calls that overlap in time on one device (other streams, other host
+ *    threads) share the array and race: the caller orders them.
+ * Same arguments and shape rules as qlora_linear_fwd, without ws/ws_bytes. */
+nf4_status qlora_linear_fwd_noalloc(const uint16_t* X, int64_t M, nf4_weight w, const uint16_t* A,
+                                    const uint16_t* B, int32_t r, float s, uint16_t* Y, uint16_t* T_out,
+                                    void* stream);
+
 /* Human-readable name of a status code (static string). */
 const char* nf4_status_str(nf4_status status);
 

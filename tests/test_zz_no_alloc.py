@@ -1,0 +1,50 @@
+"""qlora_linear_fwd_noalloc (scratch from the library's fixed device array)
+against qlora_linear_fwd (caller workspace), through the C ABI, on two calls
+in a row with different shapes, plus the rejection of a request larger than
+the fixed array.  Kept last in collection order so that it also runs after
+every other test has used the library in the same process."""
+import pytest
+import torch
+
+from bit_nf4_quantized_12_b200 import binding, workloads
+from gpu_helpers import f64, gpu_quantize, tol_check
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+SCRATCH_BYTES = 4 << 20   # QLORA_NOALLOC_SCRATCH_BYTES
+
+
+def _layer(M, N, K, r, seed):
+    W = workloads.weight(N, K, 0.02, seed=seed, device=DEV)
+    io = workloads.layer_inputs(M, N, K, r, seed=seed, device=DEV)
+    qw, st = gpu_quantize(W)
+    assert st == 0
+    return qw, io
+
+
+def test_noalloc_matches_workspace_entry_point_two_calls():
+    # the second call has a different shape and rank, so a stale status word
+    # or stale scratch from the first would show
+    cases = [(300, 384, 1024, 64, 0.25, 3), (37, 520, 640, 8, 4.0, 5)]
+    for M, N, K, r, s, seed in cases:
+        assert binding.workspace_bytes(M, N, K, r) <= SCRATCH_BYTES
+        qw, io = _layer(M, N, K, r, seed)
+        Yn, Tn = binding.linear_fwd_noalloc(io["X"], qw, io["A"], io["B"], s)
+        torch.cuda.synchronize()
+        ws = binding.workspace(M, N, K, r, DEV)
+        Yw, Tw = binding.linear_fwd(io["X"], qw, io["A"], io["B"], s, ws=ws)
+        torch.cuda.synchronize()
+        assert binding.workspace_status(ws) == 0
+        tol_check(f64(Yn), f64(Yw), f"Y {M}x{N}x{K} r{r}")
+        tol_check(f64(Tn), f64(Tw), f"T {M}x{N}x{K} r{r}")
+        # same kernels, same launch plan: the results are the same bits
+        assert torch.equal(Yn, Yw) and torch.equal(Tn, Tw)
+
+
+def test_noalloc_rejects_oversize_request():
+    M, N, K, r = 12000, 256, 512, 64
+    assert binding.workspace_bytes(M, N, K, r) > SCRATCH_BYTES
+    qw, io = _layer(M, N, K, r, 7)
+    with pytest.raises(binding.NF4Error, match="NF4_ERR_WORKSPACE"):
+        binding.linear_fwd_noalloc(io["X"], qw, io["A"], io["B"], 1.0)
