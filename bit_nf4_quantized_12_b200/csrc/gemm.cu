@@ -110,6 +110,16 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
 __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
+__device__ __forceinline__ void sts16(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(uint16_t(v)) : "memory");
+}
+__device__ __forceinline__ void stg128(void* p, const uint4& v) {
+  asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+// Barrier over the 128 threads of one warpgroup (ids 1..4; 0 is __syncthreads).
+__device__ __forceinline__ void warpgroup_sync(int id) {
+  asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory");
+}
 
 
 // ---------------------------------------------------------------- kernel
@@ -371,7 +381,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
     // ------------------------------------------------------------ epilogue
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     const int64_t wdim = BWD ? a.K : a.N;       // extent of the W dimension of the output
-    const int64_t i = w0 + t;
     const int nchunks = bt / 32;
     const bool got_acc = ok && mbar_wait(accf, 0, a.status, abort_flag);
     if (got_acc) tc_fence_after();
@@ -386,12 +395,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
         for (int j = 0; j < 32; ++j) v[j] = 0u;
       }
       if (P.splits == 1) {
-        if (i < wdim) {
+        // Stage the chunk as bf16 [32 tokens][128 rows of W] in the idle X
+        // ring, then write whole 16-byte pieces of output rows.
+        const uint32_t stg = smem_u32(act_s) + uint32_t(c) * (32 * 256);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int64_t m = m0 + c * 32 + j;
-            if (m < a.M) a.out[m * wdim + i] = uint16_t(pack_bf16x2(__uint_as_float(v[j]), 0.0f) & 0xFFFFu);
-          }
+        for (int j = 0; j < 32; ++j) sts16(stg + j * 256 + t * 2, pack_bf16x2(__uint_as_float(v[j]), 0.0f));
+        warpgroup_sync(1 + wg);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int e = q * 128 + t;                 // 16-byte piece: token row e / 16, columns (e % 16) * 8 ...
+          const int64_t m = m0 + c * 32 + (e >> 4);
+          const int64_t col = w0 + (e & 15) * 8;     // wdim % 8 == 0, so the piece is whole or absent
+          if (m < a.M && col < wdim) stg128(a.out + m * wdim + col, lds128(stg + uint32_t(e) * 16));
         }
       } else {
 #pragma unroll
