@@ -123,14 +123,18 @@ nf4_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight w, const ui
   sa.X = X; sa.A = A; sa.B = B;
   sa.T_out = t_dst; sa.hilo_out = hilo;
   sa.status = status;
-  if (launch_skinny(plan_skinny(kSkinnyT, M, N, K, r, sms), sa, strm) != cudaSuccess) return NF4_ERR_CUDA;
+  sa.pdl_mode = kPdlWaitFirst;
+  if (launch_skinny(plan_skinny(kSkinnyT, M, N, K, r, sms), sa, strm, false) != cudaSuccess) return NF4_ERR_CUDA;
 
+  // The fused GEMM may start while T is still being computed: its main
+  // product does not need T, and it waits for T before the low-rank steps.
   Nf4GemmArgs ga{};
   ga.M = M; ga.N = N; ga.K = K; ga.r = r; ga.rp = rp;
   ga.packed = w.packed; ga.c1q = w.c1q; ga.c2 = w.c2;
   ga.act = X; ga.lora_w = B; ga.lora_act = hilo; ga.out = Y;
   ga.status = status;
-  if (launch_nf4_gemm(plan_nf4_gemm(0, M, N, K, r, sms), ga, strm) != cudaSuccess) return NF4_ERR_CUDA;
+  ga.pdl_mode = kPdlWaitLowRank;
+  if (launch_nf4_gemm(plan_nf4_gemm(0, M, N, K, r, sms), ga, strm, true) != cudaSuccess) return NF4_ERR_CUDA;
   return NF4_OK;
 }
 
@@ -161,18 +165,28 @@ nf4_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, nf
   sa.X = X; sa.dY = dY; sa.A = A; sa.B = B;
   sa.status = status;
 
+  // Launch order and overlap: the first kernel waits for all earlier work of
+  // the stream; each later one is a programmatic dependent of the one before.
+  // G waits for the T recompute (both write the hi/lo buffer).  The fused
+  // GEMM waits for G at its start and then lets dA and dB start: they read
+  // only G and the inputs, so they fill the SMs the GEMM's last wave leaves
+  // idle, and wait for the GEMM only before they exit.
   const uint16_t* Tin = T;
+  bool after_kernel = false;
+  sa.pdl_mode = kPdlWaitFirst;
   if (!Tin) {  // recompute T = bf16(X A) into scratch (the hi/lo output is overwritten by G below)
     uint16_t* tw = reinterpret_cast<uint16_t*>(wsb + L.t_scratch);
     sa.T_out = tw;
     sa.hilo_out = hilo;
-    if (launch_skinny(plan_skinny(kSkinnyT, M, N, K, r, sms), sa, strm) != cudaSuccess) return NF4_ERR_CUDA;
+    if (launch_skinny(plan_skinny(kSkinnyT, M, N, K, r, sms), sa, strm, false) != cudaSuccess) return NF4_ERR_CUDA;
     Tin = tw;
+    after_kernel = true;
   }
   // G = s dY B^T as a bf16 hi/lo pair
   sa.T_out = nullptr;
   sa.hilo_out = hilo;
-  if (launch_skinny(plan_skinny(kSkinnyG, M, N, K, r, sms), sa, strm) != cudaSuccess) return NF4_ERR_CUDA;
+  if (launch_skinny(plan_skinny(kSkinnyG, M, N, K, r, sms), sa, strm, after_kernel) != cudaSuccess)
+    return NF4_ERR_CUDA;
 
   // dX = dY Wd + G A^T
   Nf4GemmArgs ga{};
@@ -180,16 +194,18 @@ nf4_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, nf
   ga.packed = w.packed; ga.c1q = w.c1q; ga.c2 = w.c2;
   ga.act = dY; ga.lora_w = A; ga.lora_act = hilo; ga.out = dX;
   ga.status = status;
-  if (launch_nf4_gemm(plan_nf4_gemm(1, M, N, K, r, sms), ga, strm) != cudaSuccess) return NF4_ERR_CUDA;
+  ga.pdl_mode = kPdlWaitFirst;
+  if (launch_nf4_gemm(plan_nf4_gemm(1, M, N, K, r, sms), ga, strm, true) != cudaSuccess) return NF4_ERR_CUDA;
 
   // dA = X^T G  (G hi + G lo)
   sa.hilo_in = hilo;
   sa.f32_out = dA;
-  if (launch_skinny(plan_skinny(kSkinnyDA, M, N, K, r, sms), sa, strm) != cudaSuccess) return NF4_ERR_CUDA;
+  sa.pdl_mode = kPdlWaitLast;
+  if (launch_skinny(plan_skinny(kSkinnyDA, M, N, K, r, sms), sa, strm, true) != cudaSuccess) return NF4_ERR_CUDA;
   // dB = s T^T dY
   sa.T = Tin;
   sa.f32_out = dB;
-  if (launch_skinny(plan_skinny(kSkinnyDB, M, N, K, r, sms), sa, strm) != cudaSuccess) return NF4_ERR_CUDA;
+  if (launch_skinny(plan_skinny(kSkinnyDB, M, N, K, r, sms), sa, strm, true) != cudaSuccess) return NF4_ERR_CUDA;
   return NF4_OK;
 }
 

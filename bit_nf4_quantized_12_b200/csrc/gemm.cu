@@ -204,6 +204,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  if (a.pdl_mode == kPdlWaitFirst) griddep_wait();
+  griddep_launch();
 
   if (warp == 0) {
     // ------------------------------------------------------------ X producer
@@ -218,6 +220,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
         if (ks < my_main) {
           tma_load_2d(dst, &P.tm_act, &x_full[s], int32_t((g_begin + ks) * 64), int32_t(m0));
         } else {
+          if (ks == my_main && a.pdl_mode == kPdlWaitLowRank) griddep_wait();   // s*T / G come from the previous kernel
           const int l = int(ks - my_main);
           const int nchunk = a.rp / 64;
           tma_load_2d(dst, &P.tm_lact, &x_full[s], int32_t((l / nchunk) * a.rp + (l % nchunk) * 64),
@@ -331,6 +334,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
           const uint32_t pa = BWD ? smem_u32(pk_s + sp * 4096 + (t & 63) * 64 + (t >> 6) * 32)
                                   : smem_u32(pk_s + sp * 4096 + t * 32);
           const uint4 p0 = lds128(pa), p1 = lds128(pa + 16);
+          // The slot is refilled by TMA, an async-proxy write: order these
+          // generic-proxy reads before it, or the refill can land first.
+          fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive(&p_empty[sp]);
           uint32_t o[32];
@@ -388,8 +394,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
     for (int c = wg; c < nchunks; c += kDequantWGs) {
       uint32_t v[32];
       if (got_acc) {
-        tmem_ld_32x32b_x32(tmem_base + lane_base + c * 32, v);
-        tmem_wait_ld();
+        tmem_ld_32x32b_x32(tmem_base + lane_base + c * 32, v);   // waits for the data
       } else {
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = 0u;
@@ -452,6 +457,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
     cluster_sync_all();
   }
 
+  if (a.pdl_mode != kPdlWaitFirst) griddep_wait();   // complete only after the previous kernel
   tc_fence_before();
   __syncthreads();
   if (warp == 2) {
@@ -585,6 +591,8 @@ __global__ void __launch_bounds__(kSkinnyThreads, 2) skinny_gemm_kernel(const __
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  if (a.pdl_mode == kPdlWaitFirst) griddep_wait();
+  griddep_launch();
 
   if (warp == 0) {
     if (elect_one()) {
@@ -663,8 +671,7 @@ __global__ void __launch_bounds__(kSkinnyThreads, 2) skinny_gemm_kernel(const __
     for (int c = 0; c < rp / 32; ++c) {
       uint32_t v[32];
       if (got) {
-        tmem_ld_32x32b_x32(tmem_base + lane_base + c * 32, v);
-        tmem_wait_ld();
+        tmem_ld_32x32b_x32(tmem_base + lane_base + c * 32, v);   // waits for the data
       } else {
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = 0u;
@@ -712,6 +719,7 @@ __global__ void __launch_bounds__(kSkinnyThreads, 2) skinny_gemm_kernel(const __
     }
   }
 
+  if (a.pdl_mode != kPdlWaitFirst) griddep_wait();   // complete only after the previous kernel
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -798,19 +806,28 @@ SkinnyPlan plan_skinny(int kind, int64_t M, int64_t N, int64_t K, int r, int num
 
 template <class Params>
 static cudaError_t launch_clustered(void (*kern)(const Params), dim3 grid, dim3 block, size_t smem,
-                                    cudaStream_t stream, dim3 cluster, const Params& P) {
+                                    cudaStream_t stream, dim3 cluster, bool pdl, const Params& P) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = cluster.x;
-  attr[0].val.clusterDim.y = cluster.y;
-  attr[0].val.clusterDim.z = cluster.z;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  if (cluster.x * cluster.y * cluster.z > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster.x;
+    attr[n].val.clusterDim.y = cluster.y;
+    attr[n].val.clusterDim.z = cluster.z;
+    ++n;
+  }
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = (cluster.x * cluster.y * cluster.z > 1) ? 1 : 0;
+  cfg.numAttrs = n;
   return cudaLaunchKernelEx(&cfg, kern, P);
 }
 
@@ -821,7 +838,7 @@ static size_t skinny_smem(int rp, int splits) {
   return 1024 + size_t(kSkinnyStages) * (16384 + size_t(rp) * 128) + (splits > 1 ? size_t(rp) * 512 : 0) + 256;
 }
 
-cudaError_t launch_nf4_gemm(const Nf4GemmPlan& plan, const Nf4GemmArgs& a, cudaStream_t stream) {
+cudaError_t launch_nf4_gemm(const Nf4GemmPlan& plan, const Nf4GemmArgs& a, cudaStream_t stream, bool pdl) {
   Nf4GemmParams P;
   memset(&P, 0, sizeof(P));
   P.a = a;
@@ -855,10 +872,10 @@ cudaError_t launch_nf4_gemm(const Nf4GemmPlan& plan, const Nf4GemmArgs& a, cudaS
   void (*kern)(const Nf4GemmParams) = plan.backward ? nf4_gemm_kernel<true> : nf4_gemm_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  return launch_clustered(kern, grid, dim3(kGemmThreads), smem, stream, dim3(1, 1, unsigned(plan.splits)), P);
+  return launch_clustered(kern, grid, dim3(kGemmThreads), smem, stream, dim3(1, 1, unsigned(plan.splits)), pdl, P);
 }
 
-cudaError_t launch_skinny(const SkinnyPlan& plan, const SkinnyArgs& a, cudaStream_t stream) {
+cudaError_t launch_skinny(const SkinnyPlan& plan, const SkinnyArgs& a, cudaStream_t stream, bool pdl) {
   SkinnyParams P;
   memset(&P, 0, sizeof(P));
   P.a = a;
@@ -900,7 +917,7 @@ cudaError_t launch_skinny(const SkinnyPlan& plan, const SkinnyArgs& a, cudaStrea
   if (e != cudaSuccess) return e;
   dim3 grid(unsigned(plan.tiles), unsigned(plan.splits));
   return launch_clustered(skinny_gemm_kernel, grid, dim3(kSkinnyThreads), smem, stream,
-                          dim3(1, unsigned(plan.splits), 1), P);
+                          dim3(1, unsigned(plan.splits), 1), pdl, P);
 }
 
 }  // namespace nf4

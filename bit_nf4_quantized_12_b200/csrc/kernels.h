@@ -6,6 +6,14 @@
 
 namespace nf4 {
 
+// How a kernel orders itself against the previous kernel of its stream when
+// it is launched as a programmatic dependent (see griddep_wait in common.cuh).
+enum PdlMode : int {
+  kPdlWaitFirst = 0,    // wait for the previous kernel, then let the next one start
+  kPdlWaitLast = 1,     // let the next kernel start, work, wait before exiting
+  kPdlWaitLowRank = 2,  // fused GEMM: main product first, wait before the low-rank operand
+};
+
 cudaError_t launch_quantize(const uint16_t* W, int64_t numel, uint8_t* packed, uint8_t* c1q, float* c2,
                             uint32_t* status, int num_sms, cudaStream_t stream);
 cudaError_t launch_dequant(const uint8_t* packed, const uint8_t* c1q, const float* c2, int64_t numel,
@@ -43,8 +51,10 @@ struct Nf4GemmArgs {
   const uint16_t* lora_act;  // sT hi/lo (forward) or G hi/lo (backward), [M, 2*rp] bf16
   uint16_t* out;             // Y [M, N] or dX [M, K], bf16
   uint32_t* status;          // kStatusTimeout on a failed wait
+  int pdl_mode;              // PdlMode
 };
-cudaError_t launch_nf4_gemm(const Nf4GemmPlan& plan, const Nf4GemmArgs& a, cudaStream_t stream);
+// pdl: launch as a programmatic dependent of the previous kernel of the stream
+cudaError_t launch_nf4_gemm(const Nf4GemmPlan& plan, const Nf4GemmArgs& a, cudaStream_t stream, bool pdl);
 
 // ---------------------------------------------------------------- skinny GEMM
 // D[i, j] = sum_k Aop[i,k] Bop[j,k] for the low-rank products, j < rp <= 256.
@@ -78,8 +88,9 @@ struct SkinnyArgs {
   uint16_t* hilo_out;       // kSkinnyT (sT) / kSkinnyG (G)
   float* f32_out;           // kSkinnyDA / kSkinnyDB
   uint32_t* status;
+  int pdl_mode;             // PdlMode (kPdlWaitFirst or kPdlWaitLast)
 };
-cudaError_t launch_skinny(const SkinnyPlan& plan, const SkinnyArgs& a, cudaStream_t stream);
+cudaError_t launch_skinny(const SkinnyPlan& plan, const SkinnyArgs& a, cudaStream_t stream, bool pdl);
 
 // Tensor-map helper (driver entry point resolved through the runtime).
 bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
