@@ -126,6 +126,18 @@ nf4_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight w, const ui
   sa.pdl_mode = kPdlWaitFirst;
   if (launch_skinny(plan_skinny(kSkinnyT, M, N, K, r, sms), sa, strm, false) != cudaSuccess) return NF4_ERR_CUDA;
 
+  if (gemv_supported(M, K)) {
+    // one token: a matrix-vector product bound by reading the packed weight,
+    // on CUDA cores; it overlaps T and waits for it only before the low-rank
+    // term
+    Nf4GemvArgs va{};
+    va.M = M; va.N = N; va.K = K; va.r = r; va.s = s;
+    va.X = X; va.packed = w.packed; va.c1q = w.c1q; va.c2 = w.c2;
+    va.T = t_dst; va.B = B; va.Y = Y; va.status = status;
+    if (launch_nf4_gemv(va, host_codebook().code, sms, strm, true) != cudaSuccess) return NF4_ERR_CUDA;
+    return NF4_OK;
+  }
+
   // The fused GEMM may start while T is still being computed: its main
   // product does not need T, and it waits for T before the low-rank steps.
   Nf4GemmArgs ga{};

@@ -143,6 +143,14 @@ NF4_DEV void tma_store_commit() { asm volatile("cp.async.bulk.commit_group;" :::
 NF4_DEV void tma_store_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 NF4_DEV void tma_store_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 // Generic-proxy shared-memory writes -> visible to the async proxy (TMA, MMA).
+// Contiguous global -> shared copy by the bulk-copy engine, completing on an
+// mbarrier; both addresses and the size are multiples of 16 bytes.
+NF4_DEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
 NF4_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // ----------------------------------------------------------------------------

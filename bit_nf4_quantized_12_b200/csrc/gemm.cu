@@ -8,24 +8,25 @@
 //
 // nf4_gemm_kernel: the two products with the frozen weight (Y and dX).  Both
 // are computed transposed, with the W dimension as the 128-row MMA "M" and
-// tokens as the MMA "N", so that the dequantized weight tile is the A operand:
-//   forward : A = Wd[n0:n0+128, k:k+64]  written by the dequant warps straight
-//             into tensor memory (tcgen05.st), one 64-weight block per thread;
-//   backward: A = Wd[n:n+64, k0:k0+128]^T written into shared memory in the
-//             MN-major 128-byte-swizzled layout the MMA reads (the NF4 blocks
-//             run along k, which is the MN dimension there).
+// tokens as the MMA "N" (bt <= 256), so that the dequantized weight tile is
+// the A operand, written into shared memory by the dequant warps:
+//   forward : A = Wd[n0:n0+128, k:k+64], K-major 128-byte-swizzled rows;
+//   backward: A = Wd[n:n+64, k0:k0+128]^T, MN-major (the NF4 blocks run along
+//             k, which is the MN dimension there).
 // The activation operand (X or dY) is staged by TMA.  The low-rank term is
 // appended as extra 64-wide reduction steps into the same fp32 accumulator,
 // using a bf16 hi/lo split of s*T (forward) or G (backward) so the low-rank
-// product carries ~16 significant bits.  A fixed split of the reduction with
-// a deterministic last-CTA reduction serves small grids (decode, k/v).
+// product carries ~16 significant bits.  Small grids (k/v, few tokens) split
+// the reduction over a cluster of up to 8 CTAs that sum their partials
+// through distributed shared memory in a fixed order.
 //
 // skinny_gemm_kernel: the rank-r products T, G, dA, dB (N = r padded to 64),
-// both operands by TMA, split reduction with the same last-CTA scheme.
+// both operands by TMA, split reduction over a cluster in the same way.
 //
-// Warp roles (nf4_gemm, 384 threads): warp 0 TMA producer, warp 1 MMA issuer,
-// warp 2 tensor-memory allocator, warps 4-11 two dequant warpgroups that take
-// alternate reduction steps and then run the epilogue.  Every wait is bounded
+// Warp roles (nf4_gemm, 640 threads): warp 0 activation TMA producer, warp 1
+// MMA issuer, warp 2 tensor-memory allocator, warp 3 packed-weight TMA
+// producer, warps 4-19 four dequant warpgroups that take every fourth
+// reduction step and then run the epilogue.  Every wait is bounded
 // (common.cuh) and reports kStatusTimeout instead of hanging.
 #include <cstdint>
 #include <cstring>
@@ -33,6 +34,7 @@
 #include <cuda_runtime.h>
 #include "common.cuh"
 #include "kernels.h"
+#include "nf4_lut.cuh"
 
 namespace nf4 {
 namespace {
@@ -41,10 +43,6 @@ constexpr int kDequantWGs = 4;                          // dequant / epilogue wa
 constexpr int kGemmThreads = 128 + 128 * kDequantWGs;   // + producer, MMA, allocator, spare warp
 constexpr int kSkinnyThreads = 192;
 constexpr int kSkinnyStages = 2;
-
-struct CodeTable {
-  float v[16];
-};
 
 struct Nf4GemmParams {
   CUtensorMap tm_act;   // X [M,K] / dY [M,N], bf16, box {64, bt}, 128B swizzle
@@ -58,49 +56,6 @@ struct Nf4GemmParams {
   int64_t main_steps;   // total 64-wide steps of the main reduction
   int lora_steps;
 };
-
-// ---------------------------------------------------------------- dequant
-// 16-entry bf16 table of one block (code[q] * scale1, each an fp32 multiply
-// rounded to bf16) split into low-byte and high-byte planes so that four
-// lookups are a handful of byte permutes.
-struct BlockTable {
-  uint32_t lo[4], hi[4];
-};
-
-__device__ __forceinline__ BlockTable make_table(const CodeTable& code, float s1) {
-  uint32_t pr[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) pr[i] = pack_bf16x2(code.v[2 * i] * s1, code.v[2 * i + 1] * s1);
-  BlockTable t;
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    t.lo[k] = prmt(pr[2 * k], pr[2 * k + 1], 0x6420);
-    t.hi[k] = prmt(pr[2 * k], pr[2 * k + 1], 0x7531);
-  }
-  return t;
-}
-
-// Four nibbles (bits 0-15 of s, element j in nibble j) -> two bf16x2 words.
-__device__ __forceinline__ void lookup4(const BlockTable& t, uint32_t s, uint32_t& o01, uint32_t& o23) {
-  const uint32_t sel_a = s;                   // entries 0-7 (bit 3 clear)
-  const uint32_t sel_b = s ^ 0x8888u;         // entries 8-15
-  const uint32_t sel2 = ((s >> 1) & 0x4444u) | 0x3210u;   // pick a or b per byte by bit 3
-  const uint32_t lo = prmt(prmt(t.lo[0], t.lo[1], sel_a), prmt(t.lo[2], t.lo[3], sel_b), sel2);
-  const uint32_t hi = prmt(prmt(t.hi[0], t.hi[1], sel_a), prmt(t.hi[2], t.hi[3], sel_b), sel2);
-  o01 = prmt(lo, hi, 0x5140);
-  o23 = prmt(lo, hi, 0x7362);
-}
-
-// 32 packed bytes (64 weights) -> 32 bf16x2 words in element order.
-__device__ __forceinline__ void dequant64(const BlockTable& t, const uint4& p0, const uint4& p1,
-                                          uint32_t (&o)[32]) {
-  const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    lookup4(t, w[i] & 0xFFFFu, o[4 * i + 0], o[4 * i + 1]);
-    lookup4(t, w[i] >> 16, o[4 * i + 2], o[4 * i + 3]);
-  }
-}
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;

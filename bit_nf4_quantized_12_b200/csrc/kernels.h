@@ -92,6 +92,28 @@ struct SkinnyArgs {
 };
 cudaError_t launch_skinny(const SkinnyPlan& plan, const SkinnyArgs& a, cudaStream_t stream, bool pdl);
 
+// ---------------------------------------------------------------- decode GEMV
+// Forward of the linear layer for one token on CUDA cores:
+//   y[n] = bf16(sum_k x[k] Wd[n,k] + s sum_j T[j] B[j,n]),
+// with T = bf16(x A) produced by the previous kernel of the stream (the
+// kernel waits for it only before the low-rank term).
+struct Nf4GemvArgs {
+  int64_t M, N, K;
+  int r;
+  float s;
+  const uint16_t* X;         // [M, K] bf16
+  const uint8_t* packed;
+  const uint8_t* c1q;
+  const float* c2;
+  const uint16_t* T;         // [M, r] bf16
+  const uint16_t* B;         // [r, N] bf16
+  uint16_t* Y;               // [M, N] bf16
+  uint32_t* status;          // kStatusTimeout on a failed wait
+};
+// Whether the GEMV takes this problem (one token, K within its shared memory).
+bool gemv_supported(int64_t M, int64_t K);
+cudaError_t launch_nf4_gemv(const Nf4GemvArgs& a, const float code[16], int num_sms, cudaStream_t stream, bool pdl);
+
 // Tensor-map helper (driver entry point resolved through the runtime).
 bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
                     uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,

@@ -1,0 +1,60 @@
+// nf4_lut.cuh -- per-block NF4 dequantization by byte permutes, shared by the
+// fused GEMM (operand tiles) and the decode GEMV.
+//
+// A weight is w' = bf16(fp32(code[q] * scale1)) ("QLoRA 原理精讲" §2.2: the
+// block constant is restored first, then each 4-bit code is mapped through the
+// NF4 table and scaled); the 16 possible values of one block are formed once
+// and looked up with prmt.
+#pragma once
+#include <cstdint>
+#include "common.cuh"
+
+namespace nf4 {
+
+struct CodeTable {
+  float v[16];
+};
+
+// 16-entry bf16 table of one block (code[q] * scale1, each an fp32 multiply
+// rounded to bf16) split into low-byte and high-byte planes so that four
+// lookups are a handful of byte permutes.
+struct BlockTable {
+  uint32_t lo[4], hi[4];
+};
+
+__device__ __forceinline__ BlockTable make_table(const CodeTable& code, float s1) {
+  uint32_t pr[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) pr[i] = pack_bf16x2(code.v[2 * i] * s1, code.v[2 * i + 1] * s1);
+  BlockTable t;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    t.lo[k] = prmt(pr[2 * k], pr[2 * k + 1], 0x6420);
+    t.hi[k] = prmt(pr[2 * k], pr[2 * k + 1], 0x7531);
+  }
+  return t;
+}
+
+// Four nibbles (bits 0-15 of s, element j in nibble j) -> two bf16x2 words.
+__device__ __forceinline__ void lookup4(const BlockTable& t, uint32_t s, uint32_t& o01, uint32_t& o23) {
+  const uint32_t sel_a = s;                   // entries 0-7 (bit 3 clear)
+  const uint32_t sel_b = s ^ 0x8888u;         // entries 8-15
+  const uint32_t sel2 = ((s >> 1) & 0x4444u) | 0x3210u;   // pick a or b per byte by bit 3
+  const uint32_t lo = prmt(prmt(t.lo[0], t.lo[1], sel_a), prmt(t.lo[2], t.lo[3], sel_b), sel2);
+  const uint32_t hi = prmt(prmt(t.hi[0], t.hi[1], sel_a), prmt(t.hi[2], t.hi[3], sel_b), sel2);
+  o01 = prmt(lo, hi, 0x5140);
+  o23 = prmt(lo, hi, 0x7362);
+}
+
+// 32 packed bytes (64 weights) -> 32 bf16x2 words in element order.
+__device__ __forceinline__ void dequant64(const BlockTable& t, const uint4& p0, const uint4& p1,
+                                          uint32_t (&o)[32]) {
+  const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    lookup4(t, w[i] & 0xFFFFu, o[4 * i + 0], o[4 * i + 1]);
+    lookup4(t, w[i] >> 16, o[4 * i + 2], o[4 * i + 3]);
+  }
+}
+
+}  // namespace nf4
