@@ -59,6 +59,11 @@ def bwd_flops(M, N, K, r):
     return 2 * M * N * K + 4 * M * N * r + 4 * M * K * r
 
 
+# ncu dram__bytes_read.sum + dram__bytes_write.sum of the forward fused GEMM on the
+# 4096x4096 weight at 2048 tokens, mean of two launches
+GEMM_FWD_Q_DRAM_BYTES = (26552320 + 67840 + 26551296 + 0) // 2
+
+
 def decode_bytes(M, N, K, r):
     numel = N * K
     nb = (numel + 63) // 64
@@ -408,7 +413,12 @@ def main():
     roofline = {"kernel": "qlora_linear_fwd+bwd calls (nf4_gemm_kernel + skinny_gemm_kernel)",
                 "bound": "tensor", "achieved": gemm_tflops, "peak": peaks["bf16_tflops_sustained"],
                 "unit": "TFLOP/s", "frac": gemm_tflops / peaks["bf16_tflops_sustained"],
-                "peak_kind": f"{peak_kind} bf16_tflops_sustained", "traffic": None}
+                "peak_kind": f"{peak_kind} bf16_tflops_sustained",
+                # DRAM read+write of one forward fused-GEMM launch on the 4096x4096
+                # weight at 2048 tokens, from ncu (profiles/dram_traffic_llama7b_q.md);
+                # the kernel has not changed since that capture
+                "traffic": GEMM_FWD_Q_DRAM_BYTES,
+                "traffic_case": "nf4_gemm_kernel<0>, 4096x4096 weight, 2048 tokens, r=64 (ncu, bytes per launch)"}
 
     # ---- end to end through the public API with host buffers
     h2d, d2h = step.e2e_bytes()
