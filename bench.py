@@ -415,8 +415,8 @@ def main():
                 "unit": "TFLOP/s", "frac": gemm_tflops / peaks["bf16_tflops_sustained"],
                 "peak_kind": f"{peak_kind} bf16_tflops_sustained",
                 # DRAM read+write of one forward fused-GEMM launch on the 4096x4096
-                # weight at 2048 tokens, from ncu (profiles/dram_traffic_llama7b_q.md);
-                # the kernel has not changed since that capture
+                # weight at 2048 tokens, from an ncu capture of this kernel as built
+                # here (it has not changed since)
                 "traffic": GEMM_FWD_Q_DRAM_BYTES,
                 "traffic_case": "nf4_gemm_kernel<0>, 4096x4096 weight, 2048 tokens, r=64 (ncu, bytes per launch)"}
 
