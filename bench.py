@@ -254,6 +254,20 @@ def oracle_sample_step(wl, frac_rows, seed=0):
     return flops, secs
 
 
+def max_over_ranks(ms, pg, device):
+    """The slowest rank's time: the job is done when every replica is."""
+    if pg is None:
+        return ms
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(world, step_flops, steps, ms):
+    """Aggregate TFLOP/s of `world` replicas that each ran `steps` steps in `ms`."""
+    return world * step_flops * steps / (ms * 1e-3) / 1e12
+
+
 def run_reference(args, wl, rank, world):
     if rank != 0:
         return
@@ -381,15 +395,11 @@ def main():
     if pg:
         pg.barrier()
     clk = clocks.stop()
-    ms = t0.elapsed_time(t1)
-    if pg:
-        t = torch.tensor([ms], device=device)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(t0.elapsed_time(t1), pg, device)
 
     M, r = wl.tokens, wl.r
     step_flops = sum(fwd_flops(M, N, K, r) + bwd_flops(M, N, K, r) for _, N, K in wl.mats)
-    value = world * step_flops * args.steps / (ms * 1e-3) / 1e12
+    value = whole_job_tflops(world, step_flops, args.steps, ms)
 
     comp = {}
     qb = sum(quant_bytes(N, K) for _, N, K in wl.mats) * args.steps
@@ -432,12 +442,8 @@ def main():
         step.run_e2e()
     e1 = _ev()
     torch.cuda.synchronize()
-    ems = e0.elapsed_time(e1)
-    if pg:
-        t = torch.tensor([ems], device=device)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ems = float(t.item())
-    e2e_value = world * step_flops * args.steps / (ems * 1e-3) / 1e12
+    ems = max_over_ranks(e0.elapsed_time(e1), pg, device)
+    e2e_value = whole_job_tflops(world, step_flops, args.steps, ems)
 
     if not args.no_components and rank == 0:
         del step
