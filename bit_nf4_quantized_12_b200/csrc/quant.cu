@@ -10,15 +10,17 @@
 // block, then one multiply per weight) compared with fp32 midpoints rounded
 // down.  For every pair of bf16 values this yields the same code as the
 // exact quotient (checked exhaustively on the host by the test suite); blocks
-// whose absmax lies outside [2^-126, 2^125] are rescaled by a power of two
-// first so the reciprocal stays a normal number.
+// whose absmax lies outside [2^-122, 2^125] are rescaled by a power of two
+// first so that 16 / absmax (the cells below work on 16 x) stays a normal
+// number.  A power-of-two rescaling leaves the computed x unchanged.
 //
 // Dequantize ("QLoRA 原理精讲" §2.2, reverse order): scale1' = fp32(E4M3 value
 // of c1q * scale2), w' = bf16(fp32(code * scale1')).
 //
 // Both kernels are HBM-bandwidth bound: 16-byte coalesced loads and stores,
 // the per-block absmax by warp shuffles across the 8 lanes that own a block,
-// and the code decision as one shared-memory table lookup plus one compare.
+// and the code decision as one lookup in a 33-cell shared-memory table plus
+// one compare.
 #include <cstdint>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -28,59 +30,58 @@
 namespace nf4 {
 namespace {
 
-constexpr int kQuantThreads = 256;   // one group (16384 weights) per CTA iteration
-constexpr int kLutBits = 11;         // sign(1) | exponent(8) | significand top 2
-constexpr int kLutSize = 1 << kLutBits;
+constexpr int kQuantThreads = 512;   // one group (16384 weights) per CTA iteration
+constexpr int kQuantIters = kGroupElems / (kQuantThreads * 8);   // 16-byte loads per thread per group: 4
+static_assert(kQuantIters * kQuantThreads * 8 == kGroupElems, "a group is an exact number of passes");
+constexpr int kCells = 33;           // cells of 16 x: floor(16 x) = -16 .. 16
 
-// Bucket table over the fp32 bit pattern of the normalized value x: every
-// bucket holds at most one threshold (checked on the host), so
-// code = base + (x > thr).  Built per CTA by binary search over the 15
-// ascending thresholds.
-__device__ __forceinline__ void build_lut(uint2* lut, const float* thr_smem) {
-  for (int idx = threadIdx.x; idx < kLutSize; idx += blockDim.x) {
-    const uint32_t lo_bits = uint32_t(idx) << (32 - kLutBits);
-    const uint32_t hi_bits = lo_bits | ((1u << (32 - kLutBits)) - 1u);
-    uint2 e;
-    if (((lo_bits >> 23) & 0xFF) == 0xFF) {   // NaN / Inf: only with non-finite input
-      e = make_uint2(__float_as_uint(INFINITY), kCodeZero);
-    } else {
-      const float a = __uint_as_float(lo_bits), b = __uint_as_float(hi_bits);
-      const float xmin = fminf(a, b), xmax = fmaxf(a, b);
-      int base = 0;                            // #{thr < xmin}: lower bound in 4 steps
-#pragma unroll
-      for (int step = 8; step >= 1; step >>= 1)
-        if (base + step - 1 < 15 && thr_smem[base + step - 1] < xmin) base += step;
-      const float t_in = (base < 15 && thr_smem[base] <= xmax) ? thr_smem[base] : INFINITY;
-      e = make_uint2(__float_as_uint(t_in), uint32_t(base));
+// Code decision by cells of width 1/16 in x = w / absmax: cell c holds
+// x in [(c-16)/16, (c-15)/16).  Consecutive NF4 thresholds are more than
+// 0.08 apart (checked on the host), so a cell holds at most one threshold
+// and code = #{thresholds below the cell} + (x > that threshold).  The
+// comparison is made on 16 x against 16 T, both exact power-of-two scalings
+// of the fp32 values, so the decision equals x > T.  Most weights fall in a
+// few cells near 0, so the warp's table loads are mostly broadcasts.
+__device__ __forceinline__ void build_cells(uint2* cells, const float* thr_smem) {
+  for (int c = threadIdx.x; c < kCells; c += blockDim.x) {
+    const float lo = float(c - 16) * 0.0625f, hi = float(c - 15) * 0.0625f;
+    uint32_t base = 0;
+    float t_in = INFINITY;
+    for (int i = 0; i < 15; ++i) {
+      if (thr_smem[i] < lo) ++base;
+      else if (thr_smem[i] < hi) t_in = thr_smem[i] * 16.0f;
     }
-    lut[idx] = e;
+    cells[c] = make_uint2(__float_as_uint(t_in), base);
   }
 }
 
-__device__ __forceinline__ uint32_t classify(const uint2* lut, float x) {
-  const uint2 e = lut[__float_as_uint(x) >> (32 - kLutBits)];
-  return e.y + (x > __uint_as_float(e.x) ? 1u : 0u);
+__device__ __forceinline__ uint32_t classify16(const uint2* cells, float x16) {
+  // NaN or |x| > 1 (only with non-finite input) clamps into an end cell
+  const uint32_t idx = min(uint32_t(__float2int_rd(x16) + 16), uint32_t(kCells - 1));
+  const uint2 e = cells[idx];
+  return e.y + (x16 > __uint_as_float(e.x) ? 1u : 0u);
 }
 
-// 8 consecutive bf16 (one uint4) -> 8 nibbles (element 0 in bits 0-3).
-__device__ __forceinline__ uint32_t quantize8(const uint2* lut, const uint4& v, float inv) {
+// 8 consecutive bf16 (one uint4) -> 8 nibbles (element 0 in bits 0-3);
+// inv16 = 16 / scale1.
+__device__ __forceinline__ uint32_t quantize8(const uint2* cells, const uint4& v, float inv16) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   uint32_t out = 0;
 #pragma unroll
   for (int j = 3; j >= 0; --j) {
-    out = (out << 4) | classify(lut, bf16hi_to_f32(w[j]) * inv);
-    out = (out << 4) | classify(lut, bf16lo_to_f32(w[j]) * inv);
+    out = (out << 4) | classify16(cells, bf16hi_to_f32(w[j]) * inv16);
+    out = (out << 4) | classify16(cells, bf16lo_to_f32(w[j]) * inv16);
   }
   return out;
 }
 // Same with the weights first scaled by a power of two (extreme blocks).
-__device__ __forceinline__ uint32_t quantize8_scaled(const uint2* lut, const uint4& v, float inv, float pre) {
+__device__ __forceinline__ uint32_t quantize8_scaled(const uint2* cells, const uint4& v, float inv16, float pre) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   uint32_t out = 0;
 #pragma unroll
   for (int j = 3; j >= 0; --j) {
-    out = (out << 4) | classify(lut, (bf16hi_to_f32(w[j]) * pre) * inv);
-    out = (out << 4) | classify(lut, (bf16lo_to_f32(w[j]) * pre) * inv);
+    out = (out << 4) | classify16(cells, (bf16hi_to_f32(w[j]) * pre) * inv16);
+    out = (out << 4) | classify16(cells, (bf16lo_to_f32(w[j]) * pre) * inv16);
   }
   return out;
 }
@@ -108,12 +109,15 @@ struct QuantArgs {
   float thr[15];
 };
 
-__device__ __forceinline__ void load_group(const QuantArgs& p, int64_t g, uint4 (&v)[8]) {
+// Pass i of a group covers weights i * 4096 .. i * 4096 + 4095; thread tid
+// loads 8 of them (tid * 8 ..), so the 8 lanes tid & ~7 .. tid | 7 hold one
+// 64-weight block.
+__device__ __forceinline__ void load_group(const QuantArgs& p, int64_t g, uint4 (&v)[kQuantIters]) {
   const int64_t gbase = g * kGroupElems;
   const bool full = gbase + kGroupElems <= p.numel;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int64_t e0 = gbase + i * 2048 + threadIdx.x * 8;
+  for (int i = 0; i < kQuantIters; ++i) {
+    const int64_t e0 = gbase + int64_t(i) * (kQuantThreads * 8) + threadIdx.x * 8;
     if (full || e0 + 8 <= p.numel) {
       v[i] = __ldcs(reinterpret_cast<const uint4*>(p.W + e0));
     } else {
@@ -128,13 +132,13 @@ __device__ __forceinline__ void load_group(const QuantArgs& p, int64_t g, uint4 
 
 // Persistent CTAs walk the groups; the next group's 32 KB are loaded while
 // the current one is classified.
-__global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const __grid_constant__ QuantArgs p) {
-  __shared__ uint2 lut[kLutSize];
+__global__ void __launch_bounds__(kQuantThreads, 2) nf4_quantize_kernel(const __grid_constant__ QuantArgs p) {
+  __shared__ uint2 cells[kCells];
   __shared__ float thr_s[16];
   __shared__ uint32_t warp_max[2][kQuantThreads / 32];
   if (threadIdx.x < 15) thr_s[threadIdx.x] = p.thr[threadIdx.x];
   __syncthreads();
-  build_lut(lut, thr_s);
+  build_cells(cells, thr_s);
   __syncthreads();
 
   const int tid = threadIdx.x;
@@ -143,15 +147,15 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const __gri
   uint32_t bad = 0;
 
   int64_t g = blockIdx.x;
-  uint4 v[8];
+  uint4 v[kQuantIters];
   if (g < p.ngroups) load_group(p, g, v);
   for (int parity = 0; g < p.ngroups; g += gridDim.x, parity ^= 1) {
     const int64_t gbase = g * kGroupElems;
     // first level: absmax of each block (8 lanes x 8 weights)
-    uint32_t bm[8];
+    uint32_t bm[kQuantIters];
     uint32_t gm = 0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < kQuantIters; ++i) {
       uint32_t m = absmax_bits8(v[i]);
       m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
       m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
@@ -165,7 +169,7 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const __gri
 
     // prefetch the next group while this one is finished
     const int64_t gn = g + gridDim.x;
-    uint4 vn[8];
+    uint4 vn[kQuantIters];
     if (gn < p.ngroups) load_group(p, gn, vn);
 
     __syncthreads();
@@ -175,39 +179,41 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const __gri
     if (gm >= 0x7F80u) bad = 1;
 
     // second level: fp32 scale2 for the group, E4M3 codes of scale1/scale2.
-    // Lane j of each 8-lane block group owns round j: it computes that
-    // block's code and reciprocal once; the others receive it by shuffle.
+    // Lane j < kQuantIters of each 8-lane block group owns pass j: it
+    // computes that block's code and reciprocal once; the others receive the
+    // reciprocal by shuffle.
     const float gmax = __uint_as_float(gm << 16);
     const float s2 = __fdiv_rn(gmax, 448.0f);
     if (tid == 0) p.c2[g] = s2;
     const int j = lane & 7;
     uint32_t my_bm = bm[0];
 #pragma unroll
-    for (int i = 1; i < 8; ++i) my_bm = (j == i) ? bm[i] : my_bm;
+    for (int i = 1; i < kQuantIters; ++i) my_bm = (j == i) ? bm[i] : my_bm;
     const float my_c1 = __uint_as_float(my_bm << 16);
-    {
-      const int64_t b = g * kGroup + j * 32 + (tid >> 3);
+    if (j < kQuantIters) {
+      const int64_t b = g * kGroup + int64_t(j) * (kQuantThreads / 8) + (tid >> 3);
       if (b < nblk_total)
         p.c1q[b] = (my_c1 == 0.0f) ? uint8_t(0) : uint8_t(f32_to_e4m3_satfinite(__fdiv_rn(my_c1, s2)));
     }
-    const bool normal = (my_c1 >= 0x1p-126f && my_c1 <= 0x1p125f) || my_c1 == 0.0f;
+    // 16 / scale1 must stay a finite normal number: scale1 in [2^-122, 2^125]
+    const bool normal = (my_c1 >= 0x1p-122f && my_c1 <= 0x1p125f) || my_c1 == 0.0f;
     const float my_inv = (my_c1 == 0.0f) ? 0.0f : (normal ? __frcp_rn(my_c1) : 0.0f);
     const bool fast = __all_sync(0xffffffffu, normal);
     // 4-bit codes
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int64_t e0 = gbase + i * 2048 + tid * 8;
+    for (int i = 0; i < kQuantIters; ++i) {
+      const int64_t e0 = gbase + int64_t(i) * (kQuantThreads * 8) + tid * 8;
       const float inv = __shfl_sync(0xffffffffu, my_inv, (lane & ~7) | i);
       if (e0 >= p.numel) continue;
       const float c1 = __uint_as_float(bm[i] << 16);
       uint32_t q8;
-      if (fast || (c1 >= 0x1p-126f && c1 <= 0x1p125f)) {
-        q8 = (c1 == 0.0f) ? 0x77777777u : quantize8(lut, v[i], fast ? inv : __frcp_rn(c1));
+      if (fast || (c1 >= 0x1p-122f && c1 <= 0x1p125f)) {
+        q8 = (c1 == 0.0f) ? 0x77777777u : quantize8(cells, v[i], (fast ? inv : __frcp_rn(c1)) * 16.0f);
       } else if (c1 == 0.0f) {
         q8 = 0x77777777u;                        // all-zero block: the 0.0 code
-      } else {                                   // keep 1/c1 a normal number
+      } else {                                   // keep 16/c1 a normal number
         const float pre = (c1 < 1.0f) ? 0x1p64f : 0x1p-64f;
-        q8 = quantize8_scaled(lut, v[i], __frcp_rn(c1 * pre), pre);
+        q8 = quantize8_scaled(cells, v[i], __frcp_rn(c1 * pre) * 16.0f, pre);
       }
       uint8_t* dst = p.packed + (e0 >> 1);
       if (e0 + 8 <= p.numel) {
@@ -225,7 +231,7 @@ __global__ void __launch_bounds__(kQuantThreads) nf4_quantize_kernel(const __gri
       }
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = vn[i];
+    for (int i = 0; i < kQuantIters; ++i) v[i] = vn[i];
   }
   if (bad && p.status != nullptr && tid == 0) atomicOr(p.status, kStatusNonfinite);
 }
@@ -334,20 +340,14 @@ cudaError_t launch_dequant(const uint8_t* packed, const uint8_t* c1q, const floa
   return cudaGetLastError();
 }
 
-// Host check that the quantize lookup table is well formed: no bucket of
-// x values (fixed sign, exponent and top 3 significand bits) holds two
-// thresholds.
+// Host check that the quantize cell table is well formed: no cell of width
+// 1/16 in x holds two thresholds.
 bool quantize_table_ok() {
   const Codebook& cb = host_codebook();
-  for (uint32_t idx = 0; idx < uint32_t(kLutSize); ++idx) {
-    uint32_t lo_bits = idx << (32 - kLutBits), hi_bits = lo_bits | ((1u << (32 - kLutBits)) - 1u);
-    if (((lo_bits >> 23) & 0xFF) == 0xFF) continue;
-    float a, b;
-    memcpy(&a, &lo_bits, 4);
-    memcpy(&b, &hi_bits, 4);
-    float xmin = a < b ? a : b, xmax = a < b ? b : a;
+  for (int c = 0; c < kCells; ++c) {
+    const float lo = float(c - 16) * 0.0625f, hi = float(c - 15) * 0.0625f;
     int n = 0;
-    for (int i = 0; i < 15; ++i) n += (cb.thr[i] >= xmin && cb.thr[i] <= xmax);
+    for (int i = 0; i < 15; ++i) n += (cb.thr[i] >= lo && cb.thr[i] < hi);
     if (n > 1) return false;
   }
   return true;
