@@ -305,14 +305,15 @@ def config_dict(wl, n):
 
 def kernel_case(case, n):
     """n launches of one call on the 7B q matrix (4096x4096, 2048 tokens, r=64),
-    or on the 28672x8192 decode weight at M=16: a small case for ncu."""
+    or on the 28672x8192 decode weight at M=16 ("decode") or M=1 ("gemv"):
+    a small case for ncu."""
     from bit_nf4_quantized_12_b200 import binding
     dev = torch.device("cuda", 0)
     wl = workloads.WORKLOADS["llama7b"]
     M, r, s = wl.tokens, wl.r, wl.s
     N, K = 4096, 4096
-    if case == "decode":
-        M, r, s, N, K = 16, 16, 1.0, 28672, 8192
+    if case in ("decode", "gemv"):
+        M, r, s, N, K = (16 if case == "decode" else 1), 16, 1.0, 28672, 8192
     W = workloads.weight(N, K, 0.02, seed=0, device=dev)
     io = workloads.layer_inputs(M, N, K, r, seed=0, device=dev)
     qw = binding.quantize(W)
@@ -324,7 +325,7 @@ def kernel_case(case, n):
             binding.quantize(W, out=qw)
         elif case == "dequant":
             binding.dequant(qw, out=Wd)
-        elif case in ("fwd", "decode"):
+        elif case in ("fwd", "decode", "gemv"):
             binding.linear_fwd(io["X"], qw, io["A"], io["B"], s, ws=ws, Y=Y, T=T)
         else:
             binding.linear_bwd(io["dY"], io["X"], qw, io["A"], io["B"], s, T=T, ws=ws)
@@ -339,7 +340,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-components", action="store_true")
-    ap.add_argument("--kernel-case", default=None, choices=["quantize", "dequant", "fwd", "bwd", "decode"],
+    ap.add_argument("--kernel-case", default=None, choices=["quantize", "dequant", "fwd", "bwd", "decode", "gemv"],
                     help="run a few launches of one call on one 7B-shaped matrix (for ncu), print nothing")
     args = ap.parse_args()
 
