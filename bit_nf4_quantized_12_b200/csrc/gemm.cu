@@ -343,7 +343,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     const int64_t wdim = BWD ? a.K : a.N;       // extent of the W dimension of the output
     const int nchunks = bt / 32;
-    const bool got_acc = ok && mbar_wait(accf, 0, a.status, abort_flag);
+    // a CTA whose share of a split reduction is empty issued no MMA: its
+    // accumulator was never written and its partial is zero
+    const bool got_acc = ok && nsteps > 0 && mbar_wait(accf, 0, a.status, abort_flag);
     if (got_acc) tc_fence_after();
     float* red = reinterpret_cast<float*>(act_s);   // split partial [bt][128] (the X ring is free now)
     for (int c = wg; c < nchunks; c += kDequantWGs) {
@@ -726,7 +728,9 @@ static int choose_splits(int64_t base_ctas, int64_t steps, int num_sms, int min_
   if (base_ctas >= num_sms) return 1;
   for (int s : {8, 4, 2}) {
     const int64_t cap = (s == 8) ? cap8 : num_sms;
-    if (base_ctas * s <= cap && steps / s >= min_steps) return s;
+    const int64_t per = (steps + s - 1) / s;
+    // every split gets at least one step (the last one gets steps - (s-1) per)
+    if (base_ctas * s <= cap && steps / s >= min_steps && (s - 1) * per < steps) return s;
   }
   return 1;
 }

@@ -102,6 +102,14 @@ def test_llama7b_layer_sampled_rows(idx):
     _run(wl.tokens, N, K, wl.r, wl.s, seed=seed, rows=rows, W=W, io=io)
 
 
+@pytest.mark.parametrize("N,K,r", [(104, 2112, 8), (4104, 64, 16), (8, 64, 8), (520, 4096, 64), (2056, 640, 256)])
+def test_one_token_gemv_edges(N, K, r):
+    """One token takes the CUDA-core GEMV: a last pass with fewer than 32
+    blocks (K = 2112 is 33 blocks), a single block per row, a row count that
+    leaves warps with fewer rows than the ring holds, and the largest rank."""
+    _run(1, N, K, r, 0.5, seed=N + K)
+
+
 @pytest.mark.parametrize("M", [1, 4, 16])
 @pytest.mark.parametrize("shape", [(28672, 8192), (8192, 28672)])
 def test_decode_shapes_sampled_columns(M, shape):
