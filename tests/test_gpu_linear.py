@@ -102,6 +102,14 @@ def test_llama7b_layer_sampled_rows(idx):
     _run(wl.tokens, N, K, wl.r, wl.s, seed=seed, rows=rows, W=W, io=io)
 
 
+@pytest.mark.parametrize("M,N,K,r", [(2, 8, 4096, 8), (100, 256, 512, 72), (33, 1032, 2112, 16),
+                                     (257, 384, 1024, 24)])
+def test_tile_and_split_edges(M, N, K, r):
+    """A single W tile split 8 ways, padding inside the rank (r = 72 of 128),
+    33 blocks per row with a ragged W tile, and a last token tile of one token."""
+    _run(M, N, K, r, 0.75, seed=M * 7 + N)
+
+
 @pytest.mark.parametrize("N,K,r", [(104, 2112, 8), (4104, 64, 16), (8, 64, 8), (520, 4096, 64), (2056, 640, 256)])
 def test_one_token_gemv_edges(N, K, r):
     """One token takes the CUDA-core GEMV: a last pass with fewer than 32
