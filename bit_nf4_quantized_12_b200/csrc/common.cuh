@@ -1,7 +1,8 @@
 // common.cuh -- sm_100a building blocks shared by the kernels of libqlora_nf4:
 // bf16 helpers, mbarrier waits with a time bound, TMA (cp.async.bulk.tensor)
-// loads/stores, and the tcgen05 (5th-generation tensor core + tensor memory)
-// instructions used by the GEMM kernels.  Inline PTX only; no CUTLASS.
+// and bulk-copy loads, programmatic dependent launch, and the tcgen05
+// (5th-generation tensor core + tensor memory) instructions used by the GEMM
+// kernels.  Inline PTX only; no CUTLASS.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -20,11 +21,6 @@ namespace nf4 {
 constexpr uint32_t kStatusNonfinite = 1u;   // quantize saw NaN or Inf in W
 constexpr uint32_t kStatusTimeout   = 2u;   // a bounded wait gave up
 
-NF4_DEV uint64_t globaltimer_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
 
 NF4_DEV uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -132,17 +128,6 @@ NF4_DEV void tma_load_2d(void* dst, const CUtensorMap* m, uint64_t* bar, int32_t
       "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
 }
-// 2-D tiled store shared -> global (bulk group).
-NF4_DEV void tma_store_2d(const CUtensorMap* m, const void* src, int32_t x, int32_t y) {
-  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-                   reinterpret_cast<uint64_t>(m)),
-               "r"(smem_u32(src)), "r"(x), "r"(y)
-               : "memory");
-}
-NF4_DEV void tma_store_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-NF4_DEV void tma_store_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-NF4_DEV void tma_store_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-// Generic-proxy shared-memory writes -> visible to the async proxy (TMA, MMA).
 // Contiguous global -> shared copy by the bulk-copy engine, completing on an
 // mbarrier; both addresses and the size are multiples of 16 bytes.
 NF4_DEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -151,10 +136,13 @@ NF4_DEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
+// Orders this thread's generic-proxy shared-memory accesses with later
+// async-proxy accesses (TMA, bulk copies, MMA): after writing an operand the
+// MMA will read, and after reading a slot a copy will refill.
 NF4_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // ----------------------------------------------------------------------------
-// tcgen05: tensor memory allocation, MMA, loads/stores.
+// tcgen05: tensor memory allocation, MMA, loads.
 // ----------------------------------------------------------------------------
 NF4_DEV void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {  // whole warp
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
@@ -180,14 +168,6 @@ NF4_DEV void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t 
       : "memory");
 }
 // D(tmem) (+)= A(tmem) * B(smem desc)^T.
-NF4_DEV void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
 // Arrive on *bar once all previously issued MMAs of this thread complete.
 NF4_DEV void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
