@@ -72,6 +72,20 @@ def test_host_validation_before_launch():
         assert L.nf4_status_str(code).startswith(b"NF4_")
 
 
+def test_noalloc_entry_point_validates_on_host():
+    """The allocation-free forward checks its scratch limit and its arguments
+    before any set-up or launch: no device is touched here."""
+    L = binding.lib()
+    fake = ctypes.c_void_p(0x10000)
+    w = binding.NF4Weight(0x10000, 0x10000, 0x10000, 256, 512)
+    limit = 4 << 20                              # QLORA_NOALLOC_SCRATCH_BYTES
+    big_m = 12000                                # needs more than the fixed scratch at r = 64
+    assert L.qlora_workspace_bytes(big_m, 256, 512, 64) > limit
+    assert L.qlora_linear_fwd_noalloc(fake, big_m, w, fake, fake, 64, 1.0, fake, None, None) == 4   # WORKSPACE
+    assert L.qlora_linear_fwd_noalloc(fake, 16, w, fake, fake, 0, 1.0, fake, None, None) == 1       # r out of range
+    assert L.qlora_linear_fwd_noalloc(fake, 0, w, fake, fake, 16, 1.0, fake, None, None) == 1       # no tokens
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(binding.NF4Error):
