@@ -24,16 +24,32 @@ int device_sms() {
 
 int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 
-// Workspace: [status word (256 B) | low-rank hi/lo pair [M, 2rp] bf16 | T scratch [M, r] bf16]
+// Shapes outside the fused tensor-core kernels (W rows not starting on an
+// NF4 block, a W row count or rank off the 8-element store granule) take the
+// generic CUDA-core path of generic.cu.
+bool needs_generic(int64_t N, int64_t K, int r) { return K % 64 != 0 || N % 8 != 0 || r % 8 != 0; }
+
+// Workspace, fused path:   [status word (256 B) | low-rank hi/lo pair [M, 2rp] bf16 | T scratch [M, r] bf16]
+// Workspace, generic path: [status word (256 B) | Wd [N, K] bf16 | T scratch [M, r] bf16 | G [M, r] fp32]
 struct WsLayout {
-  size_t hilo = 0, t_scratch = 0, total = 0;
+  size_t hilo = 0, wd = 0, t_scratch = 0, g = 0, total = 0;
 };
 constexpr size_t kHeaderBytes = 256;
 
-WsLayout ws_layout(int64_t M, int64_t /*N*/, int64_t /*K*/, int r, int /*sms*/) {
+WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int r, int /*sms*/) {
   WsLayout L;
-  const int64_t rp = round_up(r, 64);
   size_t off = kHeaderBytes;
+  if (needs_generic(N, K, r)) {
+    L.wd = off;
+    off += size_t(round_up(N * K * 2, 256));
+    L.t_scratch = off;
+    off += size_t(round_up(M * r * 2, 256));
+    L.g = off;
+    off += size_t(round_up(M * r * 4, 256));
+    L.total = off;
+    return L;
+  }
+  const int64_t rp = round_up(r, 64);
   L.hilo = off;
   off += size_t(round_up(M * 2 * rp * 2, 256));
   L.t_scratch = off;
@@ -42,12 +58,25 @@ WsLayout ws_layout(int64_t M, int64_t /*N*/, int64_t /*K*/, int r, int /*sms*/) 
   return L;
 }
 
+GenericOperand bf16_operand(const uint16_t* base, int64_t si, int64_t sp) { return GenericOperand{base, si, sp, 0}; }
+GenericOperand f32_operand(const float* base, int64_t si, int64_t sp) { return GenericOperand{base, si, sp, 1}; }
+
+// out[I, J] = scale * sum_p a(i, p) b(j, p)
+GenericGemm generic_product(int64_t I, int64_t J, GenericOperand a, GenericOperand b, int64_t P, float scale,
+                            void* out, bool out_fp32) {
+  GenericGemm g{};
+  g.I = I; g.J = J; g.nseg = 1;
+  g.seg[0] = GenericSegment{a, b, P, scale};
+  g.out = out; g.out_fp32 = out_fp32 ? 1 : 0;
+  return g;
+}
+
 nf4_status check_linear_shapes(int64_t M, const nf4_weight& w, int32_t r) {
   if (M < 1 || w.rows < 1 || w.cols < 1 || r < 1 || r > 256) return NF4_ERR_INVALID_ARG;
   if (!w.packed || !w.c1q || !w.c2) return NF4_ERR_INVALID_ARG;
-  if (w.cols % 64 != 0 || w.rows % 8 != 0 || r % 8 != 0) return NF4_ERR_UNSUPPORTED;
   if (w.rows > (int64_t(1) << 31) || w.cols > (int64_t(1) << 31) || M > (int64_t(1) << 31))
     return NF4_ERR_UNSUPPORTED;
+  if (needs_generic(w.rows, w.cols, r) && w.rows > (int64_t(1) << 40) / w.cols) return NF4_ERR_UNSUPPORTED;
   if (!aligned16(w.packed)) return NF4_ERR_MISALIGNED;
   return NF4_OK;
 }
@@ -93,6 +122,8 @@ nf4_status nf4_dequant_bf16(nf4_weight w, uint16_t* out, void* stream) {
 
 size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t r) {
   if (M < 1 || N < 1 || K < 1 || r < 1 || r > 256) return 0;
+  if (N > (int64_t(1) << 31) || K > (int64_t(1) << 31) || M > (int64_t(1) << 31)) return 0;
+  if (needs_generic(N, K, r) && N > (int64_t(1) << 40) / K) return 0;
   return ws_layout(M, N, K, r, device_sms()).total;
 }
 
@@ -117,6 +148,19 @@ nf4_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight w, const ui
   const int rp = int(round_up(r, 64));
 
   if (cudaMemsetAsync(ws, 0, kHeaderBytes, strm) != cudaSuccess) return NF4_ERR_CUDA;
+
+  if (needs_generic(N, K, r)) {
+    // Wd = dequant(W) into the workspace, T = bf16(X A), Y = bf16(X Wd^T + s T B)
+    uint16_t* wd = reinterpret_cast<uint16_t*>(wsb + L.wd);
+    if (launch_dequant(w.packed, w.c1q, w.c2, N * K, wd, sms, strm) != cudaSuccess) return NF4_ERR_CUDA;
+    const GenericGemm gt = generic_product(M, r, bf16_operand(X, K, 1), bf16_operand(A, 1, r), K, 1.0f, t_dst, false);
+    if (launch_generic_gemm(gt, sms, strm) != cudaSuccess) return NF4_ERR_CUDA;
+    GenericGemm gy = generic_product(M, N, bf16_operand(X, K, 1), bf16_operand(wd, K, 1), K, 1.0f, Y, false);
+    gy.nseg = 2;
+    gy.seg[1] = GenericSegment{bf16_operand(t_dst, r, 1), bf16_operand(B, 1, N), r, s};
+    if (launch_generic_gemm(gy, sms, strm) != cudaSuccess) return NF4_ERR_CUDA;
+    return NF4_OK;
+  }
 
   SkinnyArgs sa{};
   sa.M = M; sa.N = N; sa.K = K; sa.r = r; sa.rp = rp; sa.s = s;
@@ -171,6 +215,32 @@ nf4_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, nf
   const int rp = int(round_up(r, 64));
 
   if (cudaMemsetAsync(ws, 0, kHeaderBytes, strm) != cudaSuccess) return NF4_ERR_CUDA;
+
+  if (needs_generic(N, K, r)) {
+    // Wd = dequant(W); [T = bf16(X A)]; G = s dY B^T (fp32);
+    // dX = bf16(dY Wd + G A^T); dA = X^T G; dB = s T^T dY
+    uint16_t* wd = reinterpret_cast<uint16_t*>(wsb + L.wd);
+    float* g = reinterpret_cast<float*>(wsb + L.g);
+    if (launch_dequant(w.packed, w.c1q, w.c2, N * K, wd, sms, strm) != cudaSuccess) return NF4_ERR_CUDA;
+    const uint16_t* Tin = T;
+    if (!Tin) {
+      uint16_t* tw = reinterpret_cast<uint16_t*>(wsb + L.t_scratch);
+      const GenericGemm gt = generic_product(M, r, bf16_operand(X, K, 1), bf16_operand(A, 1, r), K, 1.0f, tw, false);
+      if (launch_generic_gemm(gt, sms, strm) != cudaSuccess) return NF4_ERR_CUDA;
+      Tin = tw;
+    }
+    const GenericGemm gg = generic_product(M, r, bf16_operand(dY, N, 1), bf16_operand(B, N, 1), N, s, g, true);
+    if (launch_generic_gemm(gg, sms, strm) != cudaSuccess) return NF4_ERR_CUDA;
+    GenericGemm gx = generic_product(M, K, bf16_operand(dY, N, 1), bf16_operand(wd, 1, K), N, 1.0f, dX, false);
+    gx.nseg = 2;
+    gx.seg[1] = GenericSegment{f32_operand(g, r, 1), bf16_operand(A, r, 1), r, 1.0f};
+    if (launch_generic_gemm(gx, sms, strm) != cudaSuccess) return NF4_ERR_CUDA;
+    const GenericGemm ga = generic_product(K, r, bf16_operand(X, 1, K), f32_operand(g, 1, r), M, 1.0f, dA, true);
+    if (launch_generic_gemm(ga, sms, strm) != cudaSuccess) return NF4_ERR_CUDA;
+    const GenericGemm gb = generic_product(r, N, bf16_operand(Tin, 1, r), bf16_operand(dY, 1, N), M, s, dB, true);
+    if (launch_generic_gemm(gb, sms, strm) != cudaSuccess) return NF4_ERR_CUDA;
+    return NF4_OK;
+  }
 
   SkinnyArgs sa{};
   sa.M = M; sa.N = N; sa.K = K; sa.r = r; sa.rp = rp; sa.s = s;

@@ -114,6 +114,30 @@ struct Nf4GemvArgs {
 bool gemv_supported(int64_t M, int64_t K);
 cudaError_t launch_nf4_gemv(const Nf4GemvArgs& a, const float code[16], int num_sms, cudaStream_t stream, bool pdl);
 
+// ---------------------------------------------------------------- generic GEMM
+// C[i, j] = sum over segments of scale * sum_p a(i, p) b(j, p), on CUDA cores,
+// for the linear layer's shapes outside the fused kernels.  An operand
+// element (i, p) sits at base[i * si + p * sp] (bf16 or fp32); C is [I, J]
+// row-major, bf16 (round to nearest even) or fp32.
+struct GenericOperand {
+  const void* base;
+  int64_t si, sp;
+  int fp32;
+};
+struct GenericSegment {
+  GenericOperand a, b;
+  int64_t P;       // reduction length
+  float scale;
+};
+struct GenericGemm {
+  int64_t I, J;
+  int nseg;        // 1 or 2
+  GenericSegment seg[2];
+  void* out;
+  int out_fp32;
+};
+cudaError_t launch_generic_gemm(const GenericGemm& g, int num_sms, cudaStream_t stream);
+
 // Tensor-map helper (driver entry point resolved through the runtime).
 bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
                     uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,

@@ -99,11 +99,16 @@ size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t r);
 /* QLoRA linear forward ([P4] §3.4; [P1] §3.1):
  *   T = bf16(X A),  Y = bf16(X Wd^T + s T B),  Wd = dequant(w) in bf16,
  * with X [M, K], A [K, r], B [r, N], Y [M, N], T [M, r] (T_out may be NULL),
- * all device bf16; s = alpha / r computed by the caller.  Wd is formed on
- * chip and never written to memory.  ws: device workspace of at least
- * qlora_workspace_bytes(M, N, K, r) bytes; its first 4 bytes are the status
- * word (zeroed by the call).  Requires K % 64 == 0, N % 8 == 0 and
- * r % 8 == 0 (NF4_ERR_UNSUPPORTED otherwise); 1 <= r <= 256. */
+ * all device bf16; s = alpha / r computed by the caller.  ws: device
+ * workspace of at least qlora_workspace_bytes(M, N, K, r) bytes; its first 4
+ * bytes are the status word (zeroed by the call).  1 <= r <= 256;
+ * M, N, K <= 2^31.
+ * When K % 64 == 0, N % 8 == 0 and r % 8 == 0, Wd is formed on chip inside
+ * the tensor-core product and never written to memory.  Other shapes (rows of
+ * W that do not start on an NF4 block, a row count or rank off the 8-element
+ * granule) take a CUDA-core path that first dequantizes W into the workspace
+ * (which then holds N * K bf16 more; N * K <= 2^40) and accumulates in fp32:
+ * same results within rounding, far lower throughput. */
 nf4_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight w, const uint16_t* A, const uint16_t* B,
                             int32_t r, float s, uint16_t* Y, uint16_t* T_out, void* ws, size_t ws_bytes,
                             void* stream);

@@ -56,12 +56,20 @@ def test_host_validation_before_launch():
     w = binding.NF4Weight(0x10000, 0x10000, 0x10000, 64, 128)
     assert L.nf4_dequant_bf16(w, odd, None) == 2
     assert L.nf4_dequant_bf16(binding.NF4Weight(0, 0x10000, 0x10000, 64, 128), fake, None) == 1
-    # linear layer: rank bounds, unsupported shapes, workspace
+    # linear layer: rank bounds, workspace
     assert L.qlora_linear_fwd(fake, 16, w, fake, fake, 0, 1.0, fake, None, fake, 1 << 30, None) == 1
     assert L.qlora_linear_fwd(fake, 16, w, fake, fake, 300, 1.0, fake, None, fake, 1 << 30, None) == 1
-    w_bad = binding.NF4Weight(0x10000, 0x10000, 0x10000, 64, 100)      # K % 64 != 0
-    assert L.qlora_linear_fwd(fake, 16, w_bad, fake, fake, 16, 1.0, fake, None, fake, 1 << 30, None) == 3
-    assert L.qlora_linear_fwd(fake, 16, w, fake, fake, 12, 1.0, fake, None, fake, 1 << 30, None) == 3
+    # shapes off the fused kernels' granules (K % 64, N % 8, r % 8) take the
+    # generic path, whose workspace also holds the dequantized W
+    w_rag = binding.NF4Weight(0x10000, 0x10000, 0x10000, 64, 100)      # K % 64 != 0
+    need = L.qlora_workspace_bytes(16, 64, 100, 16)
+    assert need >= 256 + 64 * 100 * 2 + 16 * 16 * 2 + 16 * 16 * 4
+    assert L.qlora_linear_fwd(fake, 16, w_rag, fake, fake, 16, 1.0, fake, None, fake, need - 1, None) == 4
+    assert L.qlora_workspace_bytes(16, 64, 128, 12) >= 256 + 64 * 128 * 2          # r % 8 != 0
+    assert L.qlora_workspace_bytes(16, 60, 128, 16) >= 256 + 60 * 128 * 2          # N % 8 != 0
+    assert L.qlora_workspace_bytes(16, 64, 128, 16) < 64 * 128 * 2                 # fused: no Wd copy
+    assert L.qlora_linear_fwd(fake, 16, w, fake, fake, 12, 1.0, fake, None, fake, 16, None) == 4
+    assert L.qlora_workspace_bytes(16, 1 << 31, 1 << 31, 12) == 0                  # Wd copy too large
     assert L.qlora_linear_fwd(fake, 16, w, fake, fake, 16, 1.0, fake, None, fake, 16, None) == 4
     assert L.qlora_linear_fwd(odd, 16, w, fake, fake, 16, 1.0, fake, None, fake, 1 << 30, None) == 2
     assert L.qlora_linear_bwd(fake, fake, 16, w, fake, fake, 16, 1.0, None, fake, fake, None, fake, 1 << 30,

@@ -102,6 +102,26 @@ def test_llama7b_layer_sampled_rows(idx):
     _run(wl.tokens, N, K, wl.r, wl.s, seed=seed, rows=rows, W=W, io=io)
 
 
+@pytest.mark.parametrize("M,N,K,r,s", [(5, 24, 100, 8, 2.0), (33, 40, 1000, 12, 0.5), (17, 13, 64, 8, 1.0),
+                                       (1, 96, 130, 4, 4.0), (70, 100, 257, 3, 1.5), (40, 8, 4095, 16, 0.25)])
+def test_ragged_shapes_generic_path(M, N, K, r, s):
+    """Shapes outside the fused kernels: K % 64 != 0 (rows of W do not start on
+    an NF4 block), N % 8 != 0, r % 8 != 0, and one token with a ragged K."""
+    _run(M, N, K, r, s, seed=M + N + K)
+
+
+def test_robust_weight_layer_sampled_rows():
+    """The 4095 x 11007 Student-t weight with outliers at 4096 tokens, r = 8,
+    alpha = 32 (K = 11007 is not a multiple of the block): 128 sampled token
+    rows for Y and dX, full dA and dB."""
+    wl = workloads.WORKLOADS["robust"]
+    _, N, K = wl.mats[0]
+    W = workloads.weight(N, K, wl.w_std, seed=0, device=DEV, kind=wl.w_kind)
+    io = workloads.layer_inputs(wl.tokens, N, K, wl.r, seed=0, device=DEV)
+    rows = np.sort(np.random.default_rng(5).choice(wl.tokens, 128, replace=False))
+    _run(wl.tokens, N, K, wl.r, wl.s, seed=0, rows=rows, W=W, io=io)
+
+
 @pytest.mark.parametrize("M,N,K,r", [(2, 8, 4096, 8), (100, 256, 512, 72), (33, 1032, 2112, 16),
                                      (257, 384, 1024, 24)])
 def test_tile_and_split_edges(M, N, K, r):
