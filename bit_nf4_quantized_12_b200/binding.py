@@ -30,6 +30,14 @@ class NF4Weight(ctypes.Structure):
                 ("rows", ctypes.c_int64), ("cols", ctypes.c_int64)]
 
 
+class QloraPlan(ctypes.Structure):
+    _fields_ = [("path", ctypes.c_int32), ("token_tile", ctypes.c_int32), ("splits", ctypes.c_int32),
+                ("lora_steps", ctypes.c_int32), ("tiles_w", ctypes.c_int64), ("tiles_t", ctypes.c_int64),
+                ("main_steps", ctypes.c_int64), ("lowrank_splits", ctypes.c_int32 * 4)]
+
+
+PATH_FUSED, PATH_GEMV, PATH_GENERIC = 0, 1, 2
+
 # (name, restype, argtypes) for every symbol of include/qlora_nf4.h
 _P, _I64, _I32, _F, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
 SIGNATURES = {
@@ -42,6 +50,7 @@ SIGNATURES = {
     "qlora_linear_bwd": (ctypes.c_int, [_P, _P, _I64, NF4Weight, _P, _P, _I32, _F, _P, _P, _P, _P, _P,
                                         _SZ, _P]),
     "qlora_linear_fwd_noalloc": (ctypes.c_int, [_P, _I64, NF4Weight, _P, _P, _I32, _F, _P, _P, _P]),
+    "qlora_linear_plan": (ctypes.c_int, [_I64, _I64, _I64, _I32, _I32, _I32, _P]),
     "nf4_status_str": (ctypes.c_char_p, [ctypes.c_int]),
 }
 
@@ -135,6 +144,17 @@ def dequant(qw: QuantizedWeight, out: torch.Tensor = None):
 # ---------------------------------------------------------------- linear layer
 def workspace_bytes(M, N, K, r):
     return int(lib().qlora_workspace_bytes(int(M), int(N), int(K), int(r)))
+
+
+def plan(M, N, K, r, backward=False, num_sms=0):
+    """Launch plan the library picks for a linear call of these sizes (host
+    only).  Returns a dict of the qlora_plan fields."""
+    out = QloraPlan()
+    _check(lib().qlora_linear_plan(int(M), int(N), int(K), int(r), int(bool(backward)), int(num_sms),
+                                   ctypes.byref(out)))
+    d = {name: getattr(out, name) for name, _ in QloraPlan._fields_}
+    d["lowrank_splits"] = list(out.lowrank_splits)
+    return d
 
 
 def workspace(M, N, K, r, device):

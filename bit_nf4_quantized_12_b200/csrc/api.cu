@@ -71,12 +71,24 @@ GenericGemm generic_product(int64_t I, int64_t J, GenericOperand a, GenericOpera
   return g;
 }
 
-nf4_status check_linear_shapes(int64_t M, const nf4_weight& w, int32_t r) {
-  if (M < 1 || w.rows < 1 || w.cols < 1 || r < 1 || r > 256) return NF4_ERR_INVALID_ARG;
-  if (!w.packed || !w.c1q || !w.c2) return NF4_ERR_INVALID_ARG;
-  if (w.rows > (int64_t(1) << 31) || w.cols > (int64_t(1) << 31) || M > (int64_t(1) << 31))
+// The fused GEMM puts token tiles on grid.y (at most 65535 of at most 256).
+constexpr int64_t kMaxFusedTokens = int64_t(65535) * 256;
+
+nf4_status check_sizes(int64_t M, int64_t N, int64_t K, int32_t r) {
+  if (M < 1 || N < 1 || K < 1 || r < 1 || r > 256) return NF4_ERR_INVALID_ARG;
+  if (N > (int64_t(1) << 31) || K > (int64_t(1) << 31) || M > (int64_t(1) << 31)) return NF4_ERR_UNSUPPORTED;
+  if (needs_generic(N, K, r)) {
+    if (N > (int64_t(1) << 40) / K) return NF4_ERR_UNSUPPORTED;
+  } else if (M > kMaxFusedTokens && !gemv_supported(M, K)) {
     return NF4_ERR_UNSUPPORTED;
-  if (needs_generic(w.rows, w.cols, r) && w.rows > (int64_t(1) << 40) / w.cols) return NF4_ERR_UNSUPPORTED;
+  }
+  return NF4_OK;
+}
+
+nf4_status check_linear_shapes(int64_t M, const nf4_weight& w, int32_t r) {
+  const nf4_status st = check_sizes(M, w.rows, w.cols, r);
+  if (st != NF4_OK) return st;
+  if (!w.packed || !w.c1q || !w.c2) return NF4_ERR_INVALID_ARG;
   if (!aligned16(w.packed)) return NF4_ERR_MISALIGNED;
   return NF4_OK;
 }
@@ -121,9 +133,7 @@ nf4_status nf4_dequant_bf16(nf4_weight w, uint16_t* out, void* stream) {
 }
 
 size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t r) {
-  if (M < 1 || N < 1 || K < 1 || r < 1 || r > 256) return 0;
-  if (N > (int64_t(1) << 31) || K > (int64_t(1) << 31) || M > (int64_t(1) << 31)) return 0;
-  if (needs_generic(N, K, r) && N > (int64_t(1) << 40) / K) return 0;
+  if (check_sizes(M, N, K, r) != NF4_OK) return 0;
   return ws_layout(M, N, K, r, device_sms()).total;
 }
 
@@ -288,6 +298,38 @@ nf4_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, nf
   sa.T = Tin;
   sa.f32_out = dB;
   if (launch_skinny(plan_skinny(kSkinnyDB, M, N, K, r, sms), sa, strm, true) != cudaSuccess) return NF4_ERR_CUDA;
+  return NF4_OK;
+}
+
+nf4_status qlora_linear_plan(int64_t M, int64_t N, int64_t K, int32_t r, int32_t backward, int32_t num_sms,
+                             qlora_plan* out) {
+  if (!out) return NF4_ERR_INVALID_ARG;
+  const nf4_status st = check_sizes(M, N, K, r);
+  if (st != NF4_OK) return st;
+  const int sms = num_sms > 0 ? num_sms : device_sms();
+  qlora_plan p;
+  memset(&p, 0, sizeof(p));
+  if (needs_generic(N, K, r)) {
+    p.path = QLORA_PATH_GENERIC;
+  } else if (!backward && gemv_supported(M, K)) {
+    p.path = QLORA_PATH_GEMV;
+    p.lowrank_splits[kSkinnyT] = plan_skinny(kSkinnyT, M, N, K, r, sms).splits;
+  } else {
+    const Nf4GemmPlan g = plan_nf4_gemm(backward ? 1 : 0, M, N, K, r, sms);
+    p.path = QLORA_PATH_FUSED;
+    p.token_tile = g.bt;
+    p.splits = g.splits;
+    p.lora_steps = g.lora_steps;
+    p.tiles_w = g.tiles_w;
+    p.tiles_t = g.tiles_t;
+    p.main_steps = g.main_steps;
+    // the forward computes T; the backward recomputes it when not given
+    p.lowrank_splits[kSkinnyT] = plan_skinny(kSkinnyT, M, N, K, r, sms).splits;
+    if (backward) {
+      for (int kind : {kSkinnyG, kSkinnyDA, kSkinnyDB}) p.lowrank_splits[kind] = plan_skinny(kind, M, N, K, r, sms).splits;
+    }
+  }
+  *out = p;
   return NF4_OK;
 }
 

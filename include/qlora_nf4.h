@@ -102,7 +102,8 @@ size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t r);
  * all device bf16; s = alpha / r computed by the caller.  ws: device
  * workspace of at least qlora_workspace_bytes(M, N, K, r) bytes; its first 4
  * bytes are the status word (zeroed by the call).  1 <= r <= 256;
- * M, N, K <= 2^31.
+ * M, N, K <= 2^31, and M <= 65535 * 256 on the fused path below
+ * (NF4_ERR_UNSUPPORTED otherwise, before anything is launched).
  * When K % 64 == 0, N % 8 == 0 and r % 8 == 0, Wd is formed on chip inside
  * the tensor-core product and never written to memory.  Other shapes (rows of
  * W that do not start on an NF4 block, a row count or rank off the 8-element
@@ -149,6 +150,43 @@ nf4_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, nf
 nf4_status qlora_linear_fwd_noalloc(const uint16_t* X, int64_t M, nf4_weight w, const uint16_t* A,
                                     const uint16_t* B, int32_t r, float s, uint16_t* Y, uint16_t* T_out,
                                     void* stream);
+
+/* Launch plan of a qlora_linear_fwd / qlora_linear_bwd call, as the library
+ * would choose it for these sizes on a device with num_sms SMs (num_sms <= 0:
+ * the current device, or 148 when none is visible).  Host only: launches
+ * nothing and touches no device memory.  The pages have no counterpart; it
+ * exists so that callers and tests can see which kernels a shape runs.
+ *   path        QLORA_PATH_FUSED: tensor-core GEMM with W dequantized on chip;
+ *               QLORA_PATH_GEMV: one-token forward on CUDA cores;
+ *               QLORA_PATH_GENERIC: W dequantized into the workspace, then
+ *               CUDA-core products (shapes off the fused kernels' granules).
+ *   token_tile  fused: tokens per output tile (32, 64, 128 or 256).
+ *   splits      fused: CTAs that share one output tile's reduction (1, 2, 4
+ *               or 8, one thread-block cluster); every split gets >= 1 step.
+ *   tiles_w     fused: 128-row tiles of the W dimension (N forward, K backward).
+ *   tiles_t     fused: token tiles.
+ *   main_steps  fused: 64-wide steps of the main reduction (K forward, N backward).
+ *   lora_steps  fused: 64-wide steps of the low-rank term (hi and lo halves).
+ *   lowrank_splits[4]  splits of the low-rank products T = X A, G = s dY B^T,
+ *               dA = X^T G, dB = s T^T dY (fused and GEMV paths; 0 where the
+ *               call does not run that product).
+ * Returns NF4_ERR_INVALID_ARG / NF4_ERR_UNSUPPORTED for the sizes that
+ * qlora_linear_fwd / qlora_linear_bwd reject with those codes. */
+#define QLORA_PATH_FUSED 0
+#define QLORA_PATH_GEMV 1
+#define QLORA_PATH_GENERIC 2
+typedef struct {
+  int32_t path;
+  int32_t token_tile;
+  int32_t splits;
+  int32_t lora_steps;
+  int64_t tiles_w;
+  int64_t tiles_t;
+  int64_t main_steps;
+  int32_t lowrank_splits[4];
+} qlora_plan;
+nf4_status qlora_linear_plan(int64_t M, int64_t N, int64_t K, int32_t r, int32_t backward, int32_t num_sms,
+                             qlora_plan* out);
 
 /* Human-readable name of a status code (static string). */
 const char* nf4_status_str(nf4_status status);

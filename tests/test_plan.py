@@ -1,0 +1,147 @@
+"""Host-side launch planning of the linear layer (CPU only, no device).
+
+qlora_linear_plan reports the path, tiles and reduction splits the library
+picks for a call.  These tests sweep shapes and SM counts and check what the
+kernels rely on:
+  - the path: generic exactly when K % 64, N % 8 or r % 8 is nonzero; the
+    one-token GEMV only for a forward with M = 1;
+  - the tile grid covers the output exactly once and fits the launch limits;
+  - a split reduction is used only when the tiles leave SMs idle, fits one
+    cluster (<= 8 CTAs) and gives every CTA at least one step of the
+    contiguous partition ceil(steps / splits) the kernels use (an empty
+    split would add an unwritten accumulator);
+  - sizes the calls reject are rejected by the plan query with the same code.
+"""
+import itertools
+
+import pytest
+
+from bit_nf4_quantized_12_b200 import binding
+
+
+def cdiv(a, b):
+    return -(-a // b)
+
+
+def nonempty(steps, s):
+    return s == 1 or (s - 1) * cdiv(steps, s) < steps
+
+
+LOWRANK_STEPS = {  # 64-wide reduction steps of T, G, dA (hi and lo passes), dB
+    0: lambda M, N, K: cdiv(K, 64),
+    1: lambda M, N, K: cdiv(N, 64),
+    2: lambda M, N, K: 2 * cdiv(M, 64),
+    3: lambda M, N, K: cdiv(M, 64),
+}
+
+
+def check_plan(M, N, K, r, backward, sms):
+    p = binding.plan(M, N, K, r, backward=backward, num_sms=sms)
+    generic = K % 64 != 0 or N % 8 != 0 or r % 8 != 0
+    if generic:
+        assert p["path"] == binding.PATH_GENERIC
+        assert p["lowrank_splits"] == [0, 0, 0, 0]
+        return p
+    if not backward and M == 1 and K <= 32768:     # x fits the GEMV's shared memory
+        assert p["path"] == binding.PATH_GEMV
+    if p["path"] == binding.PATH_GEMV:
+        assert not backward and M == 1
+    else:
+        assert p["path"] == binding.PATH_FUSED
+        bt = p["token_tile"]
+        assert bt == (32 if M <= 32 else 64 if M <= 64 else 128 if M <= 128 else 256)
+        assert p["tiles_t"] == cdiv(M, bt) and (p["tiles_t"] - 1) * bt < M <= p["tiles_t"] * bt
+        assert p["tiles_t"] <= 65535
+        assert p["tiles_w"] == cdiv(K if backward else N, 128)
+        steps = cdiv(N, 64) if backward else K // 64
+        assert p["main_steps"] == steps
+        assert p["lora_steps"] == 2 * cdiv(r, 64)
+        s = p["splits"]
+        assert s in (1, 2, 4, 8)
+        if s > 1:
+            tiles = p["tiles_w"] * p["tiles_t"]
+            assert tiles < sms and tiles * s <= sms
+            assert steps // s >= 4 and nonempty(steps, s)
+    kinds = (0, 1, 2, 3) if (backward and p["path"] == binding.PATH_FUSED) else (0,)
+    for kind in range(4):
+        s = p["lowrank_splits"][kind]
+        if kind not in kinds:
+            assert s == 0
+            continue
+        assert s in (1, 2, 4, 8)
+        if s > 1:
+            assert nonempty(LOWRANK_STEPS[kind](M, N, K), s), (kind, s)
+    return p
+
+
+MS = [1, 2, 16, 31, 32, 33, 64, 65, 127, 128, 129, 256, 257, 512, 2047, 2048, 4096, 16384]
+NS = [8, 64, 128, 136, 640, 1024, 4096, 11008, 28672]
+KS = [64, 128, 192, 256, 1024, 4096, 8192, 28672]
+RS = [8, 16, 64, 72, 128, 256]
+
+
+@pytest.mark.parametrize("sms", [148, 132, 16, 1])
+@pytest.mark.parametrize("backward", [0, 1])
+def test_fused_plans_sweep(sms, backward):
+    for M, N, K, r in itertools.product(MS, NS, KS, RS):
+        check_plan(M, N, K, r, backward, sms)
+
+
+def test_every_split_count_is_exercised():
+    """The sweep reaches splits of 2, 4 and 8 for both products and the
+    low-rank kernels, so the invariants above are not vacuous."""
+    seen_main, seen_low = set(), set()
+    for M, N, K, r in itertools.product(MS, NS, KS, RS[:3]):
+        for backward in (0, 1):
+            p = check_plan(M, N, K, r, backward, 148)
+            if p["path"] == binding.PATH_FUSED:
+                seen_main.add(p["splits"])
+            seen_low.update(p["lowrank_splits"])
+    assert {1, 2, 4, 8} <= seen_main
+    assert {1, 2, 4, 8} <= seen_low
+
+
+@pytest.mark.parametrize("M,N,K,r", [(5, 24, 100, 8), (33, 40, 1000, 12), (17, 13, 64, 8), (1, 96, 130, 4),
+                                     (4096, 4095, 11007, 8), (1, 4096, 4096, 12)])
+def test_ragged_shapes_take_the_generic_path(M, N, K, r):
+    for backward in (0, 1):
+        assert check_plan(M, N, K, r, backward, 148)["path"] == binding.PATH_GENERIC
+
+
+def test_plans_match_the_calls_limits():
+    L = binding.lib()
+    out = binding.QloraPlan()
+    max_fused = 65535 * 256
+    cases = [
+        ((max_fused, 4096, 64, 8), 0),
+        ((max_fused + 1, 4096, 64, 8), 3),       # token tiles beyond grid.y
+        ((max_fused + 1, 4096, 100, 8), 0),      # the generic path walks its tiles
+        ((1 << 31, 8, 64, 8), 3),
+        ((1 << 31, 8, 100, 8), 0),
+        (((1 << 31) + 1, 8, 100, 8), 3),
+        ((16, 1 << 31, 1 << 31, 12), 3),         # Wd copy beyond 2^40 elements
+        ((0, 64, 64, 8), 1),
+        ((16, 64, 64, 0), 1),
+        ((16, 64, 64, 257), 1),
+    ]
+    for (M, N, K, r), code in cases:
+        for backward in (0, 1):
+            assert L.qlora_linear_plan(M, N, K, r, backward, 148, ctypes_ref(out)) == code, (M, N, K, r)
+        assert (L.qlora_workspace_bytes(M, N, K, r) == 0) == (code != 0)
+    assert L.qlora_linear_plan(16, 64, 64, 8, 0, 148, None) == 1
+
+
+def test_fused_call_rejects_too_many_tokens_before_launch():
+    """The forward and backward return NF4_ERR_UNSUPPORTED on the host for a
+    token count the fused grid cannot hold (fake pointers: nothing is read)."""
+    L = binding.lib()
+    fake = binding.ctypes.c_void_p(0x10000)
+    w = binding.NF4Weight(0x10000, 0x10000, 0x10000, 4096, 64)
+    M = 65535 * 256 + 1
+    assert L.qlora_linear_fwd(fake, M, w, fake, fake, 8, 1.0, fake, None, fake, 1 << 62, None) == 3
+    assert L.qlora_linear_bwd(fake, fake, M, w, fake, fake, 8, 1.0, None, fake, fake, fake, fake, 1 << 62,
+                              None) == 3
+
+
+def ctypes_ref(obj):
+    return binding.ctypes.byref(obj)
