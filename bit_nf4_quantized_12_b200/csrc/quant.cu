@@ -333,7 +333,15 @@ cudaError_t launch_dequant(const uint8_t* packed, const uint8_t* c1q, const floa
   for (int i = 0; i < 16; ++i) a.code[i] = cb.code[i];
   const int64_t nunits = numel / 8;
   int64_t grid = (nunits / (32 * kDqUnits) + 7) / 8;   // 8 warps per CTA
-  const int64_t cap = int64_t(num_sms) * 8;
+  // one wave: no more CTAs than fit on the SMs at once (the loop is
+  // grid-stride, so any grid covers the weight), or a partial second wave
+  // of short-lived CTAs would add a tail to every call
+  static const int per_sm = [] {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, nf4_dequant_kernel, 256, 0) != cudaSuccess || n < 1) n = 1;
+    return n;
+  }();
+  const int64_t cap = int64_t(num_sms) * per_sm;
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
   nf4_dequant_kernel<<<dim3(unsigned(grid)), 256, 0, stream>>>(a);
