@@ -169,6 +169,19 @@ def test_70b_kv_shape_uses_split_reduction():
     _run(wl.tokens, N, K, wl.r, wl.s, seed=seed, rows=rows, W=W, io=io)
 
 
+@pytest.mark.parametrize("idx", [4, 6])
+def test_70b_large_shapes_sampled_rows(idx):
+    """The 70B gate (28672 x 8192) and down (8192 x 28672) matrices at 512
+    tokens, r = 64: 48 sampled token rows for Y and dX, full dA and dB."""
+    wl = workloads.WORKLOADS["llama70b"]
+    name, N, K = wl.mats[idx]
+    seed = workloads.matrix_seed("llama70b", 0, idx)
+    W = workloads.weight(N, K, wl.w_std, seed=seed, device=DEV)
+    io = workloads.layer_inputs(wl.tokens, N, K, wl.r, seed=seed, device=DEV)
+    rows = np.sort(np.random.default_rng(idx).choice(wl.tokens, 48, replace=False))
+    _run(wl.tokens, N, K, wl.r, wl.s, seed=seed, rows=rows, W=W, io=io)
+
+
 def test_deterministic_outputs():
     M, N, K, r = 512, 1024, 8192, 64
     W, io = _problem(M, N, K, r, seed=9)

@@ -67,6 +67,18 @@ def test_llama7b_q_full_and_other_matrices_sampled():
         _compare_groups(W, sorted(set(rng.integers(0, ng, 48).tolist()) | {0, ng - 1}), name)
 
 
+def test_llama70b_matrices_sampled_groups():
+    """Every 70B layer shape at full size (one layer's seeds), sampled groups
+    bit for bit, first and last group included."""
+    rng = np.random.default_rng(3)
+    wl = workloads.WORKLOADS["llama70b"]
+    for idx, (name, N, K) in enumerate(wl.mats):
+        W = workloads.weight(N, K, wl.w_std, seed=workloads.matrix_seed("llama70b", 0, idx), device=DEV)
+        ng = (N * K + 16383) // 16384
+        _compare_groups(W, sorted(set(rng.integers(0, ng, 24).tolist()) | {0, ng - 1}), name)
+        del W
+
+
 def test_robustness_weight_full():
     W = workloads.weight(4095, 11007, 0.02, seed=0, device=DEV, kind="student_t_outliers")
     _compare_full(W, "robust")
