@@ -12,6 +12,7 @@ kernels rely on:
     split would add an unwritten accumulator);
   - sizes the calls reject are rejected by the plan query with the same code.
 """
+import ctypes
 import itertools
 
 import pytest
@@ -126,7 +127,7 @@ def test_plans_match_the_calls_limits():
     ]
     for (M, N, K, r), code in cases:
         for backward in (0, 1):
-            assert L.qlora_linear_plan(M, N, K, r, backward, 148, ctypes_ref(out)) == code, (M, N, K, r)
+            assert L.qlora_linear_plan(M, N, K, r, backward, 148, ctypes.byref(out)) == code, (M, N, K, r)
         assert (L.qlora_workspace_bytes(M, N, K, r) == 0) == (code != 0)
     assert L.qlora_linear_plan(16, 64, 64, 8, 0, 148, None) == 1
 
@@ -135,13 +136,10 @@ def test_fused_call_rejects_too_many_tokens_before_launch():
     """The forward and backward return NF4_ERR_UNSUPPORTED on the host for a
     token count the fused grid cannot hold (fake pointers: nothing is read)."""
     L = binding.lib()
-    fake = binding.ctypes.c_void_p(0x10000)
+    fake = ctypes.c_void_p(0x10000)
     w = binding.NF4Weight(0x10000, 0x10000, 0x10000, 4096, 64)
     M = 65535 * 256 + 1
     assert L.qlora_linear_fwd(fake, M, w, fake, fake, 8, 1.0, fake, None, fake, 1 << 62, None) == 3
     assert L.qlora_linear_bwd(fake, fake, M, w, fake, fake, 8, 1.0, None, fake, fake, fake, fake, 1 << 62,
                               None) == 3
 
-
-def ctypes_ref(obj):
-    return binding.ctypes.byref(obj)
