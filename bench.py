@@ -425,11 +425,12 @@ def main():
                 "bound": "tensor", "achieved": gemm_tflops, "peak": peaks["bf16_tflops_sustained"],
                 "unit": "TFLOP/s", "frac": gemm_tflops / peaks["bf16_tflops_sustained"],
                 "peak_kind": f"{peak_kind} bf16_tflops_sustained",
-                # DRAM read+write of one forward fused-GEMM launch on the 4096x4096
-                # weight at 2048 tokens, from an ncu capture of this kernel as built
-                # here (it has not changed since)
-                "traffic": GEMM_FWD_Q_DRAM_BYTES,
-                "traffic_case": "nf4_gemm_kernel<0>, 4096x4096 weight, 2048 tokens, r=64 (ncu, bytes per launch)"}
+                # DRAM read+write per launch is reported only from a capture of the
+                # kernel as built; the fused GEMM changed after the last one
+                # (GEMM_FWD_Q_DRAM_BYTES), so it is withheld until re-captured
+                "traffic": None,
+                "traffic_case": "nf4_gemm_kernel<0>, 4096x4096 weight, 2048 tokens, r=64: not re-captured since "
+                                "the kernel last changed (earlier capture: %d bytes per launch)" % GEMM_FWD_Q_DRAM_BYTES}
 
     # ---- end to end through the public API with host buffers
     h2d, d2h = step.e2e_bytes()
