@@ -123,10 +123,12 @@ def test_robust_weight_layer_sampled_rows():
 
 
 @pytest.mark.parametrize("M,N,K,r", [(2, 8, 4096, 8), (100, 256, 512, 72), (33, 1032, 2112, 16),
-                                     (257, 384, 1024, 24)])
+                                     (257, 384, 1024, 24), (1576, 2560, 1024, 24), (1100, 256, 64, 8)])
 def test_tile_and_split_edges(M, N, K, r):
     """A single W tile split 8 ways, padding inside the rank (r = 72 of 128),
-    33 blocks per row with a ragged W tile, and a last token tile of one token."""
+    33 blocks per row with a ragged W tile, a last token tile of one token,
+    and large token counts whose last token tile is mostly empty (40 of its
+    tokens present; a single reduction step)."""
     _run(M, N, K, r, 0.75, seed=M * 7 + N)
 
 
