@@ -67,15 +67,16 @@ def test_llama7b_q_full_and_other_matrices_sampled():
         _compare_groups(W, sorted(set(rng.integers(0, ng, 48).tolist()) | {0, ng - 1}), name)
 
 
-def test_llama70b_matrices_sampled_groups():
-    """Every 70B layer shape at full size (one layer's seeds), sampled groups
-    bit for bit, first and last group included."""
-    rng = np.random.default_rng(3)
+@pytest.mark.parametrize("layer", [0, 79])
+def test_llama70b_matrices_sampled_groups(layer):
+    """Every 70B layer shape at full size, with the seeds of the first and the
+    last layer: sampled groups bit for bit, first and last group included."""
+    rng = np.random.default_rng(3 + layer)
     wl = workloads.WORKLOADS["llama70b"]
     for idx, (name, N, K) in enumerate(wl.mats):
-        W = workloads.weight(N, K, wl.w_std, seed=workloads.matrix_seed("llama70b", 0, idx), device=DEV)
+        W = workloads.weight(N, K, wl.w_std, seed=workloads.matrix_seed("llama70b", layer, idx), device=DEV)
         ng = (N * K + 16383) // 16384
-        _compare_groups(W, sorted(set(rng.integers(0, ng, 24).tolist()) | {0, ng - 1}), name)
+        _compare_groups(W, sorted(set(rng.integers(0, ng, 24).tolist()) | {0, ng - 1}), f"{name}@{layer}")
         del W
 
 
