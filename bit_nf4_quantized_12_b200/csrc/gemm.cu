@@ -749,7 +749,7 @@ Nf4GemmPlan plan_nf4_gemm(int backward, int64_t M, int64_t N, int64_t K, int r, 
   return p;
 }
 
-SkinnyPlan plan_skinny(int kind, int64_t M, int64_t N, int64_t K, int r, int num_sms) {
+SkinnyPlan plan_skinny(int kind, int64_t M, int64_t N, int64_t K, int /*r*/, int num_sms) {
   SkinnyPlan p{};
   p.kind = kind;
   switch (kind) {
