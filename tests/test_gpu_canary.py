@@ -1,5 +1,5 @@
-"""Out-of-bounds write checks by canary bytes (the memory checker is not
-available on the GPU pool, so guards stand in for it).
+"""Out-of-bounds write checks by canary bytes: guard regions around every
+buffer a kernel writes stand in for a device memory checker.
 
 Every buffer a kernel writes -- quantized weight, dequantized weight, Y, T,
 dX, dA, dB and the workspace, sized exactly as the C ABI states -- sits
