@@ -50,6 +50,7 @@ SIGNATURES = {
     "qlora_linear_bwd": (ctypes.c_int, [_P, _P, _I64, NF4Weight, _P, _P, _I32, _F, _P, _P, _P, _P, _P,
                                         _SZ, _P]),
     "qlora_linear_fwd_noalloc": (ctypes.c_int, [_P, _I64, NF4Weight, _P, _P, _I32, _F, _P, _P, _P]),
+    "qlora_linear_fwd_noalloc_info": (ctypes.c_int, [_P, _P]),
     "qlora_linear_plan": (ctypes.c_int, [_I64, _I64, _I64, _I32, _I32, _I32, _P]),
     "nf4_status_str": (ctypes.c_char_p, [ctypes.c_int]),
 }
@@ -191,6 +192,29 @@ def linear_fwd_noalloc(X, qw: QuantizedWeight, A, B, s, Y=None, T=None, want_T=T
                                           _dev(B, torch.bfloat16, "B"), r, float(s), _dev(Y, torch.bfloat16, "Y"),
                                           None if T is None else _dev(T, torch.bfloat16, "T"), _stream()))
     return Y, T
+
+
+class _DeviceWord:
+    """A view of one int32 at a raw device address (no allocation), for torch."""
+
+    def __init__(self, ptr):
+        self.__cuda_array_interface__ = {"shape": (1,), "typestr": "<i4", "data": (int(ptr), False),
+                                         "version": 3}
+
+
+def noalloc_info():
+    """(device address of the no-allocation status word on the current
+    device, size of the fixed scratch array in bytes)."""
+    ptr, nbytes = ctypes.c_void_p(), ctypes.c_size_t()
+    _check(lib().qlora_linear_fwd_noalloc_info(ctypes.byref(ptr), ctypes.byref(nbytes)))
+    return ptr.value, nbytes.value
+
+
+def noalloc_status():
+    """Status word of the last qlora_linear_fwd_noalloc call on the current
+    device (read after the stream synchronizes)."""
+    ptr, _ = noalloc_info()
+    return int(torch.as_tensor(_DeviceWord(ptr), device="cuda").item())
 
 
 def linear_bwd(dY, X, qw: QuantizedWeight, A, B, s, T=None, ws=None, dX=None, dA=None, dB=None):

@@ -20,8 +20,16 @@
 //    are rejected with NF4_ERR_WORKSPACE before anything is launched.
 //  * zeroing: the 256-byte status header is cleared on the stream by every
 //    call.  The rest is fully written by the kernels before it is read.
+//  * status: the first 4 bytes of the array are the call's status word (bit 1:
+//    a bounded device wait gave up).  qlora_linear_fwd_noalloc_info returns
+//    its device address; read it after the stream synchronizes and before the
+//    next call, which clears it.
 //  * overlapping calls race: two calls in flight at once on one device
 //    (different streams or host threads) share the array.  Order them.
+//  * device reset: the cached address belongs to the device's current
+//    context.  After cudaDeviceReset (or any teardown of the primary context)
+//    the module is loaded anew and the array may move; do not use this entry
+//    point across such a reset.
 #include <cstdint>
 #include <mutex>
 #include <cuda_runtime.h>
@@ -67,6 +75,16 @@ void* scratch_for_current_device(nf4_status* why) {
 }
 
 }  // namespace
+
+extern "C" nf4_status qlora_linear_fwd_noalloc_info(int32_t** d_status_word, size_t* scratch_bytes) {
+  if (scratch_bytes) *scratch_bytes = size_t(QLORA_NOALLOC_SCRATCH_BYTES);
+  if (!d_status_word) return NF4_OK;
+  nf4_status why = NF4_OK;
+  void* scratch = scratch_for_current_device(&why);
+  if (scratch == nullptr) return why;
+  *d_status_word = static_cast<int32_t*>(scratch);
+  return NF4_OK;
+}
 
 extern "C" nf4_status qlora_linear_fwd_noalloc(const uint16_t* X, int64_t M, nf4_weight w, const uint16_t* A,
                                                const uint16_t* B, int32_t r, float s, uint16_t* Y,

@@ -20,7 +20,10 @@
  *   - bf16 tensors are passed as uint16_t bit patterns, row-major.
  *   - Every pointer argument named d_* or documented "device" is a device
  *     pointer owned by the caller; the library allocates no memory and keeps
- *     no state between calls besides the constant NF4 table.
+ *     no state between calls besides the constant NF4 table.  The one
+ *     exception is qlora_linear_fwd_noalloc (below): a fixed per-device
+ *     scratch array in the library's device image, and the host-side table
+ *     of its device addresses, persist across its calls.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
  *     asynchronous on it; the return value reports argument validation and
  *     launch errors only.  Device pointers must be 16-byte aligned
@@ -142,14 +145,30 @@ nf4_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, nf
  *    stream capture begins;
  *  - when qlora_workspace_bytes(M, N, K, r) exceeds
  *    QLORA_NOALLOC_SCRATCH_BYTES the call returns NF4_ERR_WORKSPACE and
- *    launches nothing (at r = 64 that allows M up to 10922 tokens);
- *  - the status word is cleared on the stream by each call;
+ *    launches nothing.  On the tensor-core path at r = 64 that allows M up to
+ *    10922 tokens; shapes that take the generic path (see qlora_linear_fwd)
+ *    also need N * K * 2 bytes for the dequantized weight, so only small
+ *    ragged weights fit;
+ *  - the status word (first 4 bytes of the array) is cleared on the stream by
+ *    each call; qlora_linear_fwd_noalloc_info gives its device address so the
+ *    caller can read it after the stream synchronizes;
  *  - calls that overlap in time on one device (other streams, other host
- *    threads) share the array and race: the caller orders them.
+ *    threads) share the array and race: the caller orders them;
+ *  - the device address is cached per device for the life of the process:
+ *    do not use this entry point across cudaDeviceReset, which may move the
+ *    array.
  * Same arguments and shape rules as qlora_linear_fwd, without ws/ws_bytes. */
 nf4_status qlora_linear_fwd_noalloc(const uint16_t* X, int64_t M, nf4_weight w, const uint16_t* A,
                                     const uint16_t* B, int32_t r, float s, uint16_t* Y, uint16_t* T_out,
                                     void* stream);
+
+/* Companion of qlora_linear_fwd_noalloc (no counterpart in the pages):
+ * *scratch_bytes (may be NULL) receives QLORA_NOALLOC_SCRATCH_BYTES, and
+ * *d_status_word (may be NULL) the device address, on the current device, of
+ * the int32 status word the no-allocation calls write (bit 1: a bounded wait
+ * gave up; outputs then unspecified).  Performs the same one-time set-up as
+ * the first qlora_linear_fwd_noalloc call on the device; allocates nothing. */
+nf4_status qlora_linear_fwd_noalloc_info(int32_t** d_status_word, size_t* scratch_bytes);
 
 /* Launch plan of a qlora_linear_fwd / qlora_linear_bwd call, as the library
  * would choose it for these sizes on a device with num_sms SMs (num_sms <= 0:

@@ -86,7 +86,10 @@ def test_noalloc_entry_point_validates_on_host():
     L = binding.lib()
     fake = ctypes.c_void_p(0x10000)
     w = binding.NF4Weight(0x10000, 0x10000, 0x10000, 256, 512)
-    limit = 4 << 20                              # QLORA_NOALLOC_SCRATCH_BYTES
+    nbytes = ctypes.c_size_t()
+    assert L.qlora_linear_fwd_noalloc_info(None, ctypes.byref(nbytes)) == 0   # size only: no device needed
+    limit = nbytes.value
+    assert limit == 4 << 20                      # the size the header states
     big_m = 12000                                # needs more than the fixed scratch at r = 64
     assert L.qlora_workspace_bytes(big_m, 256, 512, 64) > limit
     assert L.qlora_linear_fwd_noalloc(fake, big_m, w, fake, fake, 64, 1.0, fake, None, None) == 4   # WORKSPACE
