@@ -9,11 +9,21 @@ dequantize it to bf16, QLoRA forward (Y, T) and backward (dX, dA, dB).
 
 Prints one JSON line (rank 0).  `value` = fwd+bwd algorithmic TFLOP/s of the
 whole step (quantize and dequantize time included in the denominator),
-summed over ranks; components report GB/s of quantize / dequantize / decode
-GEMV and TFLOP/s of forward / backward separately.  The step's working set
-(~1.3 GB) is far larger than the 126 MB L2, so no flush is needed between
-steps; the decode component flushes L2 between calls.  N > 1 runs
-independent replicas (weak scaling, no collective on the data path).
+summed over ranks.  The step's working set (~1.3 GB) is far larger than the
+126 MB L2, so no flush is needed between steps.
+
+`components` (one GPU) time each kernel family on its own, with CUDA events,
+inputs out of L2 (rotation over buffer sets larger than twice the L2, or an L2
+flush before each call), medians:
+  quantize / dequant   the 7 weights of the 7B set, GB/s
+  fwd / bwd            the step's qlora_linear calls, TFLOP/s
+  decode               28672x8192 and 8192x28672 at M in {1,4,16}, GB/s
+  llama70b             whole-model (80 layers) quantize and dequantize GB/s;
+                       fwd+bwd TFLOP/s at 512 tokens on the 7 layer shapes
+  robust               4095x11007 at 4096 tokens, r=8: quantize, dequantize,
+                       fwd, bwd
+N > 1 runs independent replicas (weak scaling, no collective on the data
+path).
 """
 import argparse
 import json
@@ -138,7 +148,8 @@ class Step:
             d["ws"] = binding.workspace(M, N, K, r, device)
             if host_copy:
                 d["host"] = {k: d[k].cpu().pin_memory() for k in ("W", "X", "dY", "A", "B")}
-                d["host_out"] = {k: torch.empty(d[k].shape, dtype=d[k].dtype).pin_memory() for k in ("dA", "dB")}
+                d["host_out"] = {k: torch.empty(d[k].shape, dtype=d[k].dtype).pin_memory()
+                                 for k in ("Y", "dX", "dA", "dB")}
             self.mats.append(d)
         self.launches_per_step = 7 * (1 + 1 + 2 + 4)
 
@@ -166,7 +177,7 @@ class Step:
 
     def run_e2e(self):
         """Same step through the public API with host buffers: H2D inputs,
-        compute, D2H of the LoRA gradients."""
+        compute, D2H of the step's results (Y, dX, dA, dB)."""
         for d in self.mats:
             for k, h in d["host"].items():
                 d[k].copy_(h, non_blocking=True)
@@ -225,6 +236,171 @@ def decode_component(device, peaks):
     return res
 
 
+def _median_ms(fn, reps, flush=None, warm=3):
+    """Median CUDA-event time of fn() over reps calls (after warm calls),
+    with flush() (untimed) before each call when given."""
+    times = []
+    for it in range(warm + reps):
+        if flush is not None:
+            flush()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        fn()
+        e.record()
+        torch.cuda.synchronize()
+        if it >= warm:
+            times.append(s.elapsed_time(e))
+    return statistics.median(times)
+
+
+def bandwidth_component(step, peaks, rounds=50):
+    """Quantize and dequantize of the 7 LLaMA-7B-shaped weights, each call
+    timed alone with CUDA events.  The calls rotate over the 7 weights (404 MB
+    of bf16 W, 101 MB of NF4 storage, 404 MB of bf16 output: well over twice
+    the 126 MB L2), so every call starts with its inputs out of L2.  Median of
+    `rounds` calls per weight; GB/s = algorithmic bytes / sum of medians."""
+    b = step.b
+    out = {}
+    for kind in ("quantize", "dequant"):
+        per = {i: [] for i in range(len(step.mats))}
+        for it in range(3 + rounds):
+            for i, d in enumerate(step.mats):
+                s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                s.record()
+                if kind == "quantize":
+                    b.quantize(d["W"], out=d["qw"])
+                else:
+                    b.dequant(d["qw"], out=d["Wd"])
+                e.record()
+                per[i].append((s, e))
+            torch.cuda.synchronize()
+        med = [statistics.median([s.elapsed_time(e) for s, e in per[i][3:]]) for i in per]
+        nbytes = sum(quant_bytes(d["N"], d["K"]) for d in step.mats)
+        gbs = nbytes / (sum(med) * 1e-3) / 1e9
+        out[kind] = {"GB/s": gbs, "frac": gbs / peaks["hbm_gbs"], "us_per_weight_set": sum(med) * 1e3,
+                     "timing": f"median of {rounds} calls per weight, calls rotating over the 7 weights "
+                               f"(inputs out of L2)"}
+    return out
+
+
+def llama70b_component(device, peaks, layers=80, reps=20):
+    """The LLaMA-70B-shaped configuration: every one of the 80 layers' 7
+    weights is generated from its own seed, quantized (only the NF4 storage is
+    kept: 35.3 GB resident), then dequantized once to bf16; each call is timed
+    alone with L2 flushed before it.  Then qlora_linear fwd+bwd at 512 tokens
+    (batch 1 x seq 512), r=64, alpha=16 on the 7 shapes of layer 0."""
+    from bit_nf4_quantized_12_b200 import binding
+    wl = workloads.WORKLOADS["llama70b"]
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    flush = flush_buf.zero_
+    stored = []
+    q_ms = 0.0
+    nbytes = 0
+    for layer in range(layers):
+        for idx, (name, N, K) in enumerate(wl.mats):
+            W = workloads.weight(N, K, wl.w_std, seed=workloads.matrix_seed("llama70b", layer, idx), device=device)
+            qw = binding.empty_quantized(N, K, device)
+            flush()
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            binding.quantize(W, out=qw)
+            e.record()
+            torch.cuda.synchronize()
+            q_ms += s.elapsed_time(e)
+            nbytes += quant_bytes(N, K)
+            stored.append((layer, idx, qw))
+            del W
+    scratch = torch.empty(max(N * K for _, N, K in wl.mats), dtype=torch.bfloat16, device=device)
+    dq_ms = 0.0
+    for layer, idx, qw in stored:
+        out = scratch[: qw.rows * qw.cols].view(qw.rows, qw.cols)
+        flush()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        binding.dequant(qw, out=out)
+        e.record()
+        torch.cuda.synchronize()
+        dq_ms += s.elapsed_time(e)
+    res = {"weights": int(sum(q.rows * q.cols for _, _, q in stored)),
+           "nf4_storage_GB": sum(q.packed.numel() + q.c1q.numel() + 4 * q.c2.numel() for _, _, q in stored) / 1e9,
+           "quantize": {"GB/s": nbytes / (q_ms * 1e-3) / 1e9, "ms": q_ms},
+           "dequant": {"GB/s": nbytes / (dq_ms * 1e-3) / 1e9, "ms": dq_ms}}
+    for k in ("quantize", "dequant"):
+        res[k]["frac"] = res[k]["GB/s"] / peaks["hbm_gbs"]
+    del scratch
+    # fwd + bwd at 512 tokens on layer 0's weights
+    M, r, s_ = wl.tokens, wl.r, wl.s
+    per = {}
+    tf_f = tf_b = ms_f = ms_b = 0.0
+    for layer, idx, qw in stored[: len(wl.mats)]:
+        name, N, K = wl.mats[idx]
+        io = workloads.layer_inputs(M, N, K, r, seed=workloads.matrix_seed("llama70b", 0, idx), device=device)
+        ws = binding.workspace(M, N, K, r, device)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
+        T = torch.empty(M, r, dtype=torch.bfloat16, device=device)
+        dX = torch.empty(M, K, dtype=torch.bfloat16, device=device)
+        dA = torch.empty(K, r, dtype=torch.float32, device=device)
+        dB = torch.empty(r, N, dtype=torch.float32, device=device)
+        f = _median_ms(lambda: binding.linear_fwd(io["X"], qw, io["A"], io["B"], s_, ws=ws, Y=Y, T=T), reps, flush)
+        bb = _median_ms(lambda: binding.linear_bwd(io["dY"], io["X"], qw, io["A"], io["B"], s_, T=T, ws=ws, dX=dX,
+                                                   dA=dA, dB=dB), reps, flush)
+        per[f"{name} {N}x{K}"] = {"fwd_us": round(f * 1e3, 1), "bwd_us": round(bb * 1e3, 1),
+                                  "fwd_TFLOP/s": round(fwd_flops(M, N, K, r) / (f * 1e-3) / 1e12, 1),
+                                  "bwd_TFLOP/s": round(bwd_flops(M, N, K, r) / (bb * 1e-3) / 1e12, 1)}
+        tf_f += fwd_flops(M, N, K, r)
+        tf_b += bwd_flops(M, N, K, r)
+        ms_f += f
+        ms_b += bb
+    fwd_t = tf_f / (ms_f * 1e-3) / 1e12
+    bwd_t = tf_b / (ms_b * 1e-3) / 1e12
+    both = (tf_f + tf_b) / ((ms_f + ms_b) * 1e-3) / 1e12
+    res["linear_512_tokens"] = {
+        "fwd": {"TFLOP/s": fwd_t, "frac": fwd_t / peaks["bf16_tflops_sustained"],
+                "frac_burst": fwd_t / peaks["bf16_tflops"]},
+        "bwd": {"TFLOP/s": bwd_t, "frac": bwd_t / peaks["bf16_tflops_sustained"],
+                "frac_burst": bwd_t / peaks["bf16_tflops"]},
+        "fwd+bwd": {"TFLOP/s": both, "frac": both / peaks["bf16_tflops_sustained"],
+                    "frac_burst": both / peaks["bf16_tflops"]},
+        "per_matrix": per, "timing": f"median of {reps} calls each, L2 flushed before every call"}
+    del stored
+    return res
+
+
+def robust_component(device, peaks, reps=5):
+    """The robustness configuration: W 4095x11007 (ragged final block and
+    group; Student-t(3) with 0.1% outliers x20), qlora_linear fwd+bwd at 4096
+    tokens, r=8, alpha=32; plus quantize / dequantize of that weight."""
+    from bit_nf4_quantized_12_b200 import binding
+    wl = workloads.WORKLOADS["robust"]
+    _, N, K = wl.mats[0]
+    M, r, s_ = wl.tokens, wl.r, wl.s
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    flush = flush_buf.zero_
+    W = workloads.weight(N, K, wl.w_std, seed=0, device=device, kind=wl.w_kind)
+    io = workloads.layer_inputs(M, N, K, r, seed=0, device=device)
+    qw = binding.quantize(W)
+    Wd = torch.empty_like(W)
+    qm = _median_ms(lambda: binding.quantize(W, out=qw), 20, flush)
+    dm = _median_ms(lambda: binding.dequant(qw, out=Wd), 20, flush)
+    ws = binding.workspace(M, N, K, r, device)
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
+    T = torch.empty(M, r, dtype=torch.bfloat16, device=device)
+    f = _median_ms(lambda: binding.linear_fwd(io["X"], qw, io["A"], io["B"], s_, ws=ws, Y=Y, T=T), reps, flush, 1)
+    bb = _median_ms(lambda: binding.linear_bwd(io["dY"], io["X"], qw, io["A"], io["B"], s_, T=T, ws=ws), reps,
+                    flush, 1)
+    plan = binding.plan(M, N, K, r)
+    path = {binding.PATH_FUSED: "fused tensor-core", binding.PATH_GEMV: "gemv",
+            binding.PATH_GENERIC: "generic CUDA-core"}[plan["path"]]
+    qb = quant_bytes(N, K)
+    ft = fwd_flops(M, N, K, r) / (f * 1e-3) / 1e12
+    bt = bwd_flops(M, N, K, r) / (bb * 1e-3) / 1e12
+    return {"path": path,
+            "quantize": {"GB/s": qb / (qm * 1e-3) / 1e9, "frac": qb / (qm * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+            "dequant": {"GB/s": qb / (dm * 1e-3) / 1e9, "frac": qb / (dm * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+            "fwd": {"TFLOP/s": ft, "frac": ft / peaks["bf16_tflops_sustained"], "us": f * 1e3},
+            "bwd": {"TFLOP/s": bt, "frac": bt / peaks["bf16_tflops_sustained"], "us": bb * 1e3}}
+
+
 # ------------------------------------------------------------------ oracle arm
 def oracle_sample_step(wl, frac_rows, seed=0):
     """The oracle over a row sample of every matrix of the step: quantize and
@@ -252,6 +428,30 @@ def oracle_sample_step(wl, frac_rows, seed=0):
         secs += time.perf_counter() - t0
         flops += fwd_flops(M, n_rows, K, r) + bwd_flops(M, n_rows, K, r)
     return flops, secs
+
+
+def blas_threads():
+    """Threads numpy's BLAS uses (the oracle's matmuls); the C quantize and
+    dequantize loops are single-threaded."""
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_baseline(wl, frac, seed=0):
+    """The oracle's sampled step on one host core and on all of them (BLAS
+    threads; the C loops run on one core either way)."""
+    from threadpoolctl import threadpool_limits
+    out = {}
+    with threadpool_limits(limits=1, user_api="blas"):
+        f1, s1 = oracle_sample_step(wl, frac, seed)
+    fa, sa = oracle_sample_step(wl, frac, seed)
+    out["all"] = {"value": fa / sa / 1e12, "cores": blas_threads(), "secs": sa}
+    out["one"] = {"value": f1 / s1 / 1e12, "cores": 1, "secs": s1}
+    return out
 
 
 def max_over_ranks(ms, pg, device):
@@ -282,7 +482,7 @@ def run_reference(args, wl, rank, world):
     value = flops / secs / 1e12
     sample = (f"oracle (plain C quantize/dequant + float64 numpy GEMM) on 1/256 of the output features of each of "
               f"the 7 matrices per step (group-aligned row slice), all {wl.tokens} tokens")
-    cores = torch.get_num_threads()
+    cores = blas_threads()
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -305,8 +505,9 @@ def config_dict(wl, n):
 
 def kernel_case(case, n):
     """n launches of one call on the 7B q matrix (4096x4096, 2048 tokens, r=64),
-    or on the 28672x8192 decode weight at M=16 ("decode") or M=1 ("gemv"):
-    a small case for ncu."""
+    or on the 28672x8192 decode weight at M=16 ("decode") or M=1 ("gemv");
+    quantize and dequant run on the 28672x8192 weight, whose 470 MB of bf16
+    exceed the L2: a small case for ncu."""
     from bit_nf4_quantized_12_b200 import binding
     dev = torch.device("cuda", 0)
     wl = workloads.WORKLOADS["llama7b"]
@@ -314,6 +515,8 @@ def kernel_case(case, n):
     N, K = 4096, 4096
     if case in ("decode", "gemv"):
         M, r, s, N, K = (16 if case == "decode" else 1), 16, 1.0, 28672, 8192
+    if case in ("quantize", "dequant"):
+        M, r, s, N, K = 16, 16, 1.0, 28672, 8192
     W = workloads.weight(N, K, 0.02, seed=0, device=dev)
     io = workloads.layer_inputs(M, N, K, r, seed=0, device=dev)
     qw = binding.quantize(W)
@@ -418,12 +621,14 @@ def main():
         comp[k]["frac"] = comp[k]["GB/s"] / peaks["hbm_gbs"]
     for k in ("fwd", "bwd"):
         comp[k]["frac"] = comp[k]["TFLOP/s"] / peaks["bf16_tflops_sustained"]
+        comp[k]["frac_burst"] = comp[k]["TFLOP/s"] / peaks["bf16_tflops"]
 
     # dominant work: the qlora_linear calls (forward + backward)
     gemm_tflops = (fl_f + fl_b) / ((f_ms + b_ms) * 1e-3) / 1e12
     roofline = {"kernel": "qlora_linear_fwd+bwd calls (nf4_gemm_kernel + skinny_gemm_kernel)",
                 "bound": "tensor", "achieved": gemm_tflops, "peak": peaks["bf16_tflops_sustained"],
                 "unit": "TFLOP/s", "frac": gemm_tflops / peaks["bf16_tflops_sustained"],
+                "frac_burst": gemm_tflops / peaks["bf16_tflops"],
                 "peak_kind": f"{peak_kind} bf16_tflops_sustained",
                 # DRAM read+write per launch is reported only from a capture of the
                 # kernel as built; the fused GEMM changed after the last one
@@ -447,18 +652,28 @@ def main():
     ems = max_over_ranks(e0.elapsed_time(e1), pg, device)
     e2e_value = whole_job_tflops(world, step_flops, args.steps, ems)
 
-    if not args.no_components and rank == 0:
+    if not args.no_components and rank == 0 and world == 1:
+        bw = bandwidth_component(step, peaks)
+        comp["quantize"].update({"step_GB/s": comp["quantize"].pop("GB/s"), "step_frac": comp["quantize"].pop("frac")})
+        comp["dequant"].update({"step_GB/s": comp["dequant"].pop("GB/s"), "step_frac": comp["dequant"].pop("frac")})
+        comp["quantize"].update(bw["quantize"])
+        comp["dequant"].update(bw["dequant"])
         del step
         torch.cuda.empty_cache()
         comp["decode"] = decode_component(device, peaks)
+        torch.cuda.empty_cache()
+        comp["llama70b"] = llama70b_component(device, peaks)
+        torch.cuda.empty_cache()
+        comp["robust"] = robust_component(device, peaks)
 
     cpu = None
     if rank == 0 and world == 1:
-        flops, secs = oracle_sample_step(wl, 1.0 / 256)
-        cpu = {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": torch.get_num_threads(),
-               "kind": "oracle",
-               "sample": "oracle on 1/256 of the output features of each of the 7 matrices "
-                         "(quantize+dequant of those rows, fwd+bwd restricted to them), all 2048 tokens"}
+        ob = oracle_baseline(wl, 1.0 / 256)
+        sample = ("oracle on 1/256 of the output features of each of the 7 matrices (quantize+dequant of those "
+                  "rows, fwd+bwd restricted to them), all 2048 tokens")
+        cpu = {"value": ob["all"]["value"], "unit": "TFLOP/s", "cores": ob["all"]["cores"], "kind": "oracle",
+               "sample": sample + "; C quantize/dequant loops single-threaded, numpy BLAS on all cores",
+               "single_core": {"value": ob["one"]["value"], "unit": "TFLOP/s", "cores": 1}}
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -469,7 +684,7 @@ def main():
                 "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h},
                 "gpu_launches": step_launches * args.steps,
-                "peaks": {"kind": peak_kind, "hbm_gbs": peaks["hbm_gbs"],
+                "peaks": {"kind": peak_kind, "hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"],
                           "bf16_tflops_sustained": peaks["bf16_tflops_sustained"]}}
         print(json.dumps(line), flush=True)
     if pg:

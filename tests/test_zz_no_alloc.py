@@ -1,6 +1,6 @@
 """qlora_linear_fwd_noalloc (scratch from the library's fixed device array)
-against qlora_linear_fwd (caller workspace), through the C ABI, on calls in a
-row with different shapes, plus the rejection of a request larger than the
+against qlora_linear_fwd (caller workspace), through the C ABI, on two calls
+in a row for each of several shapes, plus the rejection of a request larger than the
 fixed array.
 
 The entry point exists for callers that cannot allocate device memory when
@@ -38,24 +38,28 @@ def test_noalloc_matches_workspace_entry_point_two_calls():
     for M, N, K, r, s, seed in cases:
         assert binding.workspace_bytes(M, N, K, r) <= scratch_bytes
         qw, io = _layer(M, N, K, r, seed)
-        Yn = torch.empty(M, N, dtype=torch.bfloat16, device=DEV)
-        Tn = torch.empty(M, r, dtype=torch.bfloat16, device=DEV)
-        binding.noalloc_info()                     # one-time set-up outside the measured window
-        torch.cuda.synchronize()
-        before = (torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0])
-        binding.linear_fwd_noalloc(io["X"], qw, io["A"], io["B"], s, Y=Yn, T=Tn)
-        torch.cuda.synchronize()
-        after = (torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0])
-        assert after == before, (before, after)
-        assert binding.noalloc_status() == 0
         ws = binding.workspace(M, N, K, r, DEV)
         Yw, Tw = binding.linear_fwd(io["X"], qw, io["A"], io["B"], s, ws=ws)
         torch.cuda.synchronize()
         assert binding.workspace_status(ws) == 0
-        tol_check(f64(Yn), f64(Yw), f"Y {M}x{N}x{K} r{r}")
-        tol_check(f64(Tn), f64(Tw), f"T {M}x{N}x{K} r{r}")
-        # same kernels, same launch plan: the results are the same bits
-        assert torch.equal(Yn, Yw) and torch.equal(Tn, Tw)
+        outs = [(torch.empty(M, N, dtype=torch.bfloat16, device=DEV), torch.empty(M, r, dtype=torch.bfloat16, device=DEV))
+                for _ in range(2)]
+        for call, (Yn, Tn) in enumerate(outs):
+            # The first launch of a kernel in a fresh process can make the
+            # driver load its code into device memory, so the free-memory
+            # check brackets the second of the two calls.
+            torch.cuda.synchronize()
+            before = (torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0])
+            binding.linear_fwd_noalloc(io["X"], qw, io["A"], io["B"], s, Y=Yn, T=Tn)
+            torch.cuda.synchronize()
+            after = (torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0])
+            if call == 1:
+                assert after == before, (before, after)
+            assert binding.noalloc_status() == 0
+            tol_check(f64(Yn), f64(Yw), f"Y {M}x{N}x{K} r{r} call {call}")
+            tol_check(f64(Tn), f64(Tw), f"T {M}x{N}x{K} r{r} call {call}")
+            # same kernels, same launch plan: the results are the same bits
+            assert torch.equal(Yn, Yw) and torch.equal(Tn, Tw)
 
 
 def test_noalloc_rejects_oversize_request():
