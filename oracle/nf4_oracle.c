@@ -281,3 +281,175 @@ void oracle_classify_array(const float* w, const float* absmax, int64_t n, int32
     oracle_codebook(codes);
     for (int64_t i = 0; i < n; i++) q[i] = oracle_nearest_code(codes, w[i], absmax[i]);
 }
+
+/* ================================================================== */
+/* Format variants, the FP16 compute type                              */
+/* ================================================================== */
+
+/* Round a real (given exactly as a double) to the nearest IEEE binary16
+ * value, ties to the even significand, written from the definition like
+ * oracle_bf16_round: 1 sign, 5 exponent (bias 15), 10 stored significand
+ * bits; subnormal spacing 2^-24; largest finite 65504; a value whose rounding
+ * reaches 2^16 becomes inf.  FP16 is the compute type the pages name for
+ * GPUs without BF16 ("QLoRA 原理精讲" §三 误区4). */
+uint16_t oracle_f16_round(double x)
+{
+    if (isnan(x)) return 0x7E00;
+    uint16_t sign = signbit(x) ? 0x8000 : 0;
+    double a = fabs(x);
+    if (isinf(a)) return sign | 0x7C00;
+    if (a == 0.0) return sign;
+    int e;
+    frexp(a, &e);                     /* a = m * 2^e, m in [0.5,1) */
+    double ulp = (e - 1 < -14) ? ldexp(1.0, -24) : ldexp(1.0, (e - 1) - 10);
+    double lo = floor(a / ulp) * ulp, hi = lo + ulp;
+    double dlo = a - lo, dhi = hi - a;
+    double r;
+    if (dlo < dhi) r = lo;
+    else if (dhi < dlo) r = hi;
+    else r = (fmod(lo / ulp, 2.0) == 0.0) ? lo : hi;
+    if (r >= 65536.0) return sign | 0x7C00;
+    /* encode r exactly */
+    if (r < ldexp(1.0, -14)) return sign | (uint16_t)(r / ldexp(1.0, -24));      /* subnormal or 0 */
+    frexp(r, &e);
+    int E = e - 1;                                  /* r = 1.f * 2^E */
+    uint16_t frac = (uint16_t)((r / ldexp(1.0, E) - 1.0) * 1024.0);
+    return sign | (uint16_t)((E + 15) << 10) | frac;
+}
+
+double oracle_f16_to_f64(uint16_t h)
+{
+    int s = h >> 15, e = (h >> 10) & 0x1F, f = h & 0x3FF;
+    double v;
+    if (e == 31) v = f ? NAN : INFINITY;
+    else if (e == 0) v = ldexp((double)f, -24);
+    else v = ldexp(1.0 + f / 1024.0, e - 15);
+    return s ? -v : v;
+}
+
+/* Uniform INT4 table ("QLoRA 原理精讲" §2.1: INT4 maps the values onto the 16
+ * integers [-8, 7], evenly spaced).  Reading: the integers are divided by the
+ * largest magnitude, 8, so that the table lies in [-1, 1] like NF4's and the
+ * same absmax normalization applies: codes[i] = (i - 8) / 8. */
+void oracle_codebook_int4(float codes[16])
+{
+    for (int i = 0; i < 16; i++) codes[i] = (float)(i - 8) / 8.0f;
+}
+
+/* quant_type: 0 = NF4, 1 = INT4 (uniform).  double_quant: 0 = FP8 E4M3
+ * scale1 + FP32 scale2 per 256 blocks (the default of the pages), 1 = none
+ * (FP32 scale1 per block, "QLoRA 原理精讲" §2.2 工程动机: 0.5 bit per weight),
+ * 2 = unsigned 8-bit linear scale1 + FP32 scale2 per 256 blocks (the
+ * "8 bit" of "LoRA、Q-LoRA 与 PortLLM" §3.2 read as an integer code). */
+static void codebook_of(int quant_type, float codes[16])
+{
+    if (quant_type == 1) oracle_codebook_int4(codes);
+    else oracle_codebook(codes);
+}
+
+/* Unsigned 8-bit linear code of a non-negative fp32 ratio: nearest integer,
+ * ties to even, clamped to [0, 255]. */
+static uint8_t u8_encode(float t)
+{
+    if (!(t > 0.0f)) return 0;
+    if (t >= 255.0f) return 255;
+    double fl = floor((double)t), d = (double)t - fl;
+    double q = (d > 0.5) ? fl + 1.0 : (d < 0.5) ? fl : ((fmod(fl, 2.0) == 0.0) ? fl : fl + 1.0);
+    return (uint8_t)q;
+}
+
+/* Quantize with a chosen table and first-level-constant format.  Same block
+ * and group layout, codes and packing as oracle_quantize.  c1 receives
+ * nblocks bytes (double_quant 0 or 2) or nblocks fp32 values (double_quant 1);
+ * c2 receives ngroups fp32 values (unused, may be NULL, for double_quant 1).
+ * Returns 1 when W holds a NaN or an infinity. */
+int oracle_quantize_fmt(const uint16_t* W, int64_t numel, int quant_type, int double_quant,
+                        uint8_t* packed, void* c1, float* c2)
+{
+    float codes[16];
+    codebook_of(quant_type, codes);
+    int64_t nb = oracle_nblocks(numel), ng = oracle_ngroups(numel);
+    int nonfinite = 0;
+    for (int64_t g = 0; g < ng; g++) {
+        int64_t b0 = g * ORC_GROUP, b1 = b0 + ORC_GROUP;
+        if (b1 > nb) b1 = nb;
+        float absmax[ORC_GROUP];
+        float gmax = 0.0f;
+        for (int64_t b = b0; b < b1; b++) {            /* scale1 = block absmax */
+            float m = 0.0f;
+            int64_t e0 = b * ORC_BLOCK, e1 = e0 + ORC_BLOCK;
+            if (e1 > numel) e1 = numel;
+            for (int64_t e = e0; e < e1; e++) {
+                float w = (float)oracle_bf16_to_f64(W[e]);
+                if (!isfinite(w)) nonfinite = 1;
+                float a = fabsf(w);
+                if (a > m) m = a;
+            }
+            absmax[b - b0] = m;
+            if (m > gmax) gmax = m;
+        }
+        if (double_quant == 1) {                       /* FP32 scale1, no second level */
+            for (int64_t b = b0; b < b1; b++) ((float*)c1)[b] = absmax[b - b0];
+        } else if (double_quant == 2) {                /* uint8 scale1 / FP32 scale2 */
+            float s2 = gmax / 255.0f;
+            c2[g] = s2;
+            for (int64_t b = b0; b < b1; b++) {
+                float m = absmax[b - b0];
+                ((uint8_t*)c1)[b] = (m == 0.0f) ? (uint8_t)0 : u8_encode(m / s2);
+            }
+        } else {                                       /* E4M3 scale1 / FP32 scale2 */
+            float s2 = gmax / 448.0f;
+            c2[g] = s2;
+            for (int64_t b = b0; b < b1; b++) {
+                float m = absmax[b - b0];
+                ((uint8_t*)c1)[b] = (m == 0.0f) ? (uint8_t)0 : oracle_e4m3_encode(m / s2);
+            }
+        }
+        for (int64_t b = b0; b < b1; b++) {            /* 4-bit codes, packed */
+            int64_t e0 = b * ORC_BLOCK, e1 = e0 + ORC_BLOCK;
+            if (e1 > numel) e1 = numel;
+            for (int64_t e = e0; e < e1; e++) {
+                float w = (float)oracle_bf16_to_f64(W[e]);
+                int q = oracle_nearest_code(codes, w, absmax[b - b0]);
+                if ((e & 1) == 0) packed[e >> 1] = (uint8_t)q;
+                else              packed[e >> 1] = (uint8_t)(packed[e >> 1] | (q << 4));
+            }
+        }
+    }
+    return nonfinite;
+}
+
+/* Dequantize a weight stored in any of the formats above into the compute
+ * type (dtype 0 = bf16, 1 = fp16): scale1' = the stored FP32 scale1, or
+ * fp32(decoded 8-bit code * scale2); w' = round_dtype(fp32(code * scale1')). */
+void oracle_dequant_fmt(const uint8_t* packed, const void* c1, const float* c2, int64_t numel,
+                        int quant_type, int double_quant, int dtype, uint16_t* out)
+{
+    float codes[16];
+    codebook_of(quant_type, codes);
+    for (int64_t e = 0; e < numel; e++) {
+        int64_t b = e / ORC_BLOCK, g = b / ORC_GROUP;
+        float s1;
+        if (double_quant == 1) s1 = ((const float*)c1)[b];
+        else if (double_quant == 2) s1 = (float)((const uint8_t*)c1)[b] * c2[g];
+        else s1 = (float)oracle_e4m3_decode(((const uint8_t*)c1)[b]) * c2[g];
+        int q = (e & 1) ? (packed[e >> 1] >> 4) : (packed[e >> 1] & 0xF);
+        float v = codes[q] * s1;
+        out[e] = dtype ? oracle_f16_round((double)v) : oracle_bf16_round((double)v);
+    }
+}
+
+void oracle_f16_round_array(const double* x, int64_t n, uint16_t* out)
+{
+    for (int64_t i = 0; i < n; i++) out[i] = oracle_f16_round(x[i]);
+}
+void oracle_f16_decode_array(const uint16_t* h, int64_t n, double* out)
+{
+    for (int64_t i = 0; i < n; i++) out[i] = oracle_f16_to_f64(h[i]);
+}
+void oracle_classify_fmt_array(int quant_type, const float* w, const float* absmax, int64_t n, int32_t* q)
+{
+    float codes[16];
+    codebook_of(quant_type, codes);
+    for (int64_t i = 0; i < n; i++) q[i] = oracle_nearest_code(codes, w[i], absmax[i]);
+}
