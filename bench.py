@@ -22,8 +22,9 @@ flush before each call), medians:
                        fwd+bwd TFLOP/s at 512 tokens on the 7 layer shapes
   robust               4095x11007 at 4096 tokens, r=8: quantize, dequantize,
                        fwd, bwd
-N > 1 runs independent replicas (weak scaling, no collective on the data
-path).
+N > 1 runs data-parallel replicas (weak scaling: 2048 tokens per rank); the
+step's one exchange is an NCCL all-reduce of every matrix's dA and dB, held
+in one flat bucket.
 """
 import argparse
 import json
@@ -126,13 +127,18 @@ class ClockSampler:
 class Step:
     """All buffers of one step over the 7B layer set, resident on the GPU."""
 
-    def __init__(self, device, wl, host_copy=False):
-        from bit_nf4_quantized_12_b200 import binding
+    def __init__(self, device, wl, host_copy=False, world=1):
+        from bit_nf4_quantized_12_b200 import binding, dp
         self.b = binding
+        self.dp = dp
         self.wl = wl
         self.dev = device
+        self.world = world
         self.mats = []
         M, r = wl.tokens, wl.r
+        # dA, dB of all 7 matrices live in one flat bucket: with N ranks the
+        # step ends with one all-reduce of it (data-parallel replicas)
+        self.bucket = dp.GradBucket.for_layers([(K, N, r) for _, N, K in wl.mats], device)
         for idx, (name, N, K) in enumerate(wl.mats):
             seed = workloads.matrix_seed(wl.name, 0, idx)
             d = dict(name=name, N=N, K=K)
@@ -143,8 +149,7 @@ class Step:
             d["Y"] = torch.empty(M, N, dtype=torch.bfloat16, device=device)
             d["T"] = torch.empty(M, r, dtype=torch.bfloat16, device=device)
             d["dX"] = torch.empty(M, K, dtype=torch.bfloat16, device=device)
-            d["dA"] = torch.empty(K, r, dtype=torch.float32, device=device)
-            d["dB"] = torch.empty(r, N, dtype=torch.float32, device=device)
+            d["dA"], d["dB"] = self.bucket.views[idx]
             d["ws"] = binding.workspace(M, N, K, r, device)
             if host_copy:
                 d["host"] = {k: d[k].cpu().pin_memory() for k in ("W", "X", "dY", "A", "B")}
@@ -174,6 +179,8 @@ class Step:
                          dA=d["dA"], dB=d["dB"])
             if events is not None:
                 events["bwd"][1].append(_ev())
+        if self.world > 1:   # the one exchange step: global dA, dB over the replicas' tokens
+            self.dp.allreduce_lora_grads([self.bucket.flat])
 
     def run_e2e(self):
         """Same step through the public API with host buffers: H2D inputs,
@@ -499,7 +506,8 @@ def config_dict(wl, n):
     return {"workload": "llama7b_layer_set: q,k,v,o 4096x4096; gate,up 11008x4096; down 4096x11008; "
                         "quantize+dq, dequant, qlora fwd+bwd at 2048 tokens, r=64, alpha=16",
             "global_batch": wl.tokens * n, "seq_len": 512, "rank": wl.r, "alpha": wl.alpha,
-            "parallelism": f"replicas{n}" if n > 1 else "single",
+            "parallelism": f"dp{n}: tokens split across replicas, one NCCL all-reduce of the dA/dB bucket per step"
+                           if n > 1 else "single",
             "l2": "step working set ~1.3 GB > 126 MB L2; no flush between steps"}
 
 
@@ -571,7 +579,7 @@ def main():
         pg = dist
     peaks, peak_kind = load_peaks()
 
-    step = Step(device, wl, host_copy=True)
+    step = Step(device, wl, host_copy=True, world=world)
     step_launches = step.launches_per_step
     # warm-up: at least W steps and at least ~1.5 s of load, with the clock
     # sampler already running so that its samples cover the loaded GPU

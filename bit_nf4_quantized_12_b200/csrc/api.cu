@@ -58,16 +58,19 @@ WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int r, int /*sms*/) {
   return L;
 }
 
-GenericOperand bf16_operand(const uint16_t* base, int64_t si, int64_t sp) { return GenericOperand{base, si, sp, 0}; }
-GenericOperand f32_operand(const float* base, int64_t si, int64_t sp) { return GenericOperand{base, si, sp, 1}; }
+// 16-bit operand in the compute type (kind kOpBF16 / kOpF16) or an fp32 one
+GenericOperand half_operand(int kind, const uint16_t* base, int64_t si, int64_t sp) {
+  return GenericOperand{base, si, sp, kind};
+}
+GenericOperand f32_operand(const float* base, int64_t si, int64_t sp) { return GenericOperand{base, si, sp, kOpF32}; }
 
 // out[I, J] = scale * sum_p a(i, p) b(j, p)
 GenericGemm generic_product(int64_t I, int64_t J, GenericOperand a, GenericOperand b, int64_t P, float scale,
-                            void* out, bool out_fp32) {
+                            void* out, int out_kind) {
   GenericGemm g{};
   g.I = I; g.J = J; g.nseg = 1;
   g.seg[0] = GenericSegment{a, b, P, scale};
-  g.out = out; g.out_fp32 = out_fp32 ? 1 : 0;
+  g.out = out; g.out_kind = out_kind;
   return g;
 }
 
@@ -85,13 +88,28 @@ nf4_status check_sizes(int64_t M, int64_t N, int64_t K, int32_t r) {
   return NF4_OK;
 }
 
+bool format_ok(int32_t quant_type, int32_t double_quant) {
+  return (quant_type == NF4_QUANT_NF4 || quant_type == NF4_QUANT_INT4) &&
+         (double_quant == NF4_DQ_E4M3 || double_quant == NF4_DQ_NONE || double_quant == NF4_DQ_U8);
+}
+
+// The storage buffers of a weight: present, in a known format, aligned.
+nf4_status check_weight(const nf4_weight& w) {
+  if (!format_ok(w.quant_type, w.double_quant)) return NF4_ERR_INVALID_ARG;
+  if (!w.packed || !w.c1q || (w.double_quant != NF4_DQ_NONE && !w.c2)) return NF4_ERR_INVALID_ARG;
+  if (!aligned16(w.packed)) return NF4_ERR_MISALIGNED;
+  if (w.double_quant == NF4_DQ_NONE && (reinterpret_cast<uintptr_t>(w.c1q) & 3u) != 0) return NF4_ERR_MISALIGNED;
+  return NF4_OK;
+}
+
 nf4_status check_linear_shapes(int64_t M, const nf4_weight& w, int32_t r) {
   const nf4_status st = check_sizes(M, w.rows, w.cols, r);
   if (st != NF4_OK) return st;
-  if (!w.packed || !w.c1q || !w.c2) return NF4_ERR_INVALID_ARG;
-  if (!aligned16(w.packed)) return NF4_ERR_MISALIGNED;
-  return NF4_OK;
+  return check_weight(w);
 }
+
+bool dtype_ok(int32_t dtype) { return dtype == QLORA_BF16 || dtype == QLORA_F16; }
+int operand_kind(int32_t dtype) { return dtype == QLORA_F16 ? kOpF16 : kOpBF16; }
 
 }  // namespace
 
@@ -112,23 +130,54 @@ nf4_status nf4_sizes(int64_t numel, size_t* packed_bytes, int64_t* nblocks, int6
   return NF4_OK;
 }
 
-nf4_status nf4_quantize_dq(const uint16_t* W, int64_t rows, int64_t cols, uint8_t* packed, uint8_t* c1q, float* c2,
-                           int32_t* d_status, void* stream) {
-  if (!W || !packed || !c1q || !c2 || rows < 1 || cols < 1) return NF4_ERR_INVALID_ARG;
+nf4_status nf4_quantize(const uint16_t* W, int64_t rows, int64_t cols, int32_t quant_type, int32_t double_quant,
+                        uint8_t* packed, void* c1, float* c2, int32_t* d_status, void* stream) {
+  if (!format_ok(quant_type, double_quant)) return NF4_ERR_INVALID_ARG;
+  if (!W || !packed || !c1 || (double_quant != NF4_DQ_NONE && !c2) || rows < 1 || cols < 1)
+    return NF4_ERR_INVALID_ARG;
   if (rows > (int64_t(1) << 40) / cols) return NF4_ERR_UNSUPPORTED;
   if (!aligned16(W) || !aligned16(packed)) return NF4_ERR_MISALIGNED;
-  if (!quantize_table_ok()) return NF4_ERR_UNSUPPORTED;
-  cudaError_t e = launch_quantize(W, rows * cols, packed, c1q, c2, reinterpret_cast<uint32_t*>(d_status),
-                                  device_sms(), static_cast<cudaStream_t>(stream));
+  if (double_quant == NF4_DQ_NONE && (reinterpret_cast<uintptr_t>(c1) & 3u) != 0) return NF4_ERR_MISALIGNED;
+  if (!quantize_table_ok(quant_type)) return NF4_ERR_UNSUPPORTED;
+  cudaError_t e = launch_quantize(W, rows * cols, quant_type, double_quant, packed, c1, c2,
+                                  reinterpret_cast<uint32_t*>(d_status), device_sms(),
+                                  static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NF4_OK : NF4_ERR_CUDA;
+}
+
+nf4_status nf4_quantize_dq(const uint16_t* W, int64_t rows, int64_t cols, uint8_t* packed, uint8_t* c1q, float* c2,
+                           int32_t* d_status, void* stream) {
+  return nf4_quantize(W, rows, cols, NF4_QUANT_NF4, NF4_DQ_E4M3, packed, c1q, c2, d_status, stream);
+}
+
+nf4_status nf4_dequant(nf4_weight w, int32_t dtype, uint16_t* out, void* stream) {
+  if (!dtype_ok(dtype) || !out || w.rows < 1 || w.cols < 1) return NF4_ERR_INVALID_ARG;
+  const nf4_status st = check_weight(w);
+  if (st != NF4_OK) return st;
+  if (w.rows > (int64_t(1) << 40) / w.cols) return NF4_ERR_UNSUPPORTED;
+  if (!aligned16(out)) return NF4_ERR_MISALIGNED;
+  cudaError_t e = launch_dequant(w.packed, w.c1q, w.c2, w.rows * w.cols, w.quant_type, w.double_quant,
+                                 dtype == QLORA_F16, out, device_sms(), static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? NF4_OK : NF4_ERR_CUDA;
 }
 
 nf4_status nf4_dequant_bf16(nf4_weight w, uint16_t* out, void* stream) {
-  if (!w.packed || !w.c1q || !w.c2 || !out || w.rows < 1 || w.cols < 1) return NF4_ERR_INVALID_ARG;
-  if (w.rows > (int64_t(1) << 40) / w.cols) return NF4_ERR_UNSUPPORTED;
-  if (!aligned16(w.packed) || !aligned16(out)) return NF4_ERR_MISALIGNED;
-  cudaError_t e = launch_dequant(w.packed, w.c1q, w.c2, w.rows * w.cols, out, device_sms(),
-                                 static_cast<cudaStream_t>(stream));
+  return nf4_dequant(w, QLORA_BF16, out, stream);
+}
+
+nf4_status nf4_lora_merge(nf4_weight w, const uint16_t* A, const uint16_t* B, int32_t r, float s, int32_t dtype,
+                          uint16_t* out, void* stream) {
+  if (!dtype_ok(dtype) || !A || !B || !out || w.rows < 1 || w.cols < 1 || r < 1 || r > 256)
+    return NF4_ERR_INVALID_ARG;
+  const nf4_status st = check_weight(w);
+  if (st != NF4_OK) return st;
+  if (w.rows > (int64_t(1) << 40) / w.cols || w.rows > int64_t(65535) * 128) return NF4_ERR_UNSUPPORTED;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(out)) return NF4_ERR_MISALIGNED;
+  MergeArgs a{};
+  a.packed = w.packed; a.c1 = w.c1q; a.c2 = w.c2;
+  a.N = w.rows; a.K = w.cols; a.double_quant = w.double_quant;
+  a.A = A; a.B = B; a.r = r; a.s = s; a.f16 = dtype == QLORA_F16 ? 1 : 0; a.out = out;
+  cudaError_t e = launch_merge(a, host_codebook(w.quant_type).code, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? NF4_OK : NF4_ERR_CUDA;
 }
 
@@ -137,9 +186,12 @@ size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t r) {
   return ws_layout(M, N, K, r, device_sms()).total;
 }
 
-nf4_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight w, const uint16_t* A, const uint16_t* B,
-                            int32_t r, float s, uint16_t* Y, uint16_t* T_out, void* ws, size_t ws_bytes,
-                            void* stream) {
+nf4_status qlora_linear_fwd_ex(int32_t dtype, const uint16_t* X, int64_t M, nf4_weight w, const uint16_t* A,
+                               const uint16_t* B, int32_t r, float s, uint16_t* Y, uint16_t* T_out, void* ws,
+                               size_t ws_bytes, void* stream) {
+  if (!dtype_ok(dtype)) return NF4_ERR_INVALID_ARG;
+  const int f16 = dtype == QLORA_F16 ? 1 : 0;
+  const int hk = operand_kind(dtype);
   nf4_status st = check_linear_shapes(M, w, r);
   if (st != NF4_OK) return st;
   if (!X || !A || !B || !Y) return NF4_ERR_INVALID_ARG;
@@ -162,12 +214,15 @@ nf4_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight w, const ui
   if (needs_generic(N, K, r)) {
     // Wd = dequant(W) into the workspace, T = bf16(X A), Y = bf16(X Wd^T + s T B)
     uint16_t* wd = reinterpret_cast<uint16_t*>(wsb + L.wd);
-    if (launch_dequant(w.packed, w.c1q, w.c2, N * K, wd, sms, strm) != cudaSuccess) return NF4_ERR_CUDA;
-    const GenericGemm gt = generic_product(M, r, bf16_operand(X, K, 1), bf16_operand(A, 1, r), K, 1.0f, t_dst, false);
+    if (launch_dequant(w.packed, w.c1q, w.c2, N * K, w.quant_type, w.double_quant, f16, wd, sms, strm) !=
+        cudaSuccess)
+      return NF4_ERR_CUDA;
+    const GenericGemm gt = generic_product(M, r, half_operand(hk, X, K, 1), half_operand(hk, A, 1, r), K, 1.0f,
+                                           t_dst, hk);
     if (launch_generic_gemm(gt, sms, strm) != cudaSuccess) return NF4_ERR_CUDA;
-    GenericGemm gy = generic_product(M, N, bf16_operand(X, K, 1), bf16_operand(wd, K, 1), K, 1.0f, Y, false);
+    GenericGemm gy = generic_product(M, N, half_operand(hk, X, K, 1), half_operand(hk, wd, K, 1), K, 1.0f, Y, hk);
     gy.nseg = 2;
-    gy.seg[1] = GenericSegment{bf16_operand(t_dst, r, 1), bf16_operand(B, 1, N), r, s};
+    gy.seg[1] = GenericSegment{half_operand(hk, t_dst, r, 1), half_operand(hk, B, 1, N), r, s};
     if (launch_generic_gemm(gy, sms, strm) != cudaSuccess) return NF4_ERR_CUDA;
     return NF4_OK;
   }
@@ -178,6 +233,7 @@ nf4_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight w, const ui
   sa.T_out = t_dst; sa.hilo_out = hilo;
   sa.status = status;
   sa.pdl_mode = kPdlWaitFirst;
+  sa.f16 = f16;
   if (launch_skinny(plan_skinny(kSkinnyT, M, N, K, r, sms), sa, strm, false) != cudaSuccess) return NF4_ERR_CUDA;
 
   if (gemv_supported(M, K)) {
@@ -188,7 +244,8 @@ nf4_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight w, const ui
     va.M = M; va.N = N; va.K = K; va.r = r; va.s = s;
     va.X = X; va.packed = w.packed; va.c1q = w.c1q; va.c2 = w.c2;
     va.T = t_dst; va.B = B; va.Y = Y; va.status = status;
-    if (launch_nf4_gemv(va, host_codebook().code, sms, strm, true) != cudaSuccess) return NF4_ERR_CUDA;
+    va.dq = w.double_quant; va.f16 = f16;
+    if (launch_nf4_gemv(va, host_codebook(w.quant_type).code, sms, strm, true) != cudaSuccess) return NF4_ERR_CUDA;
     return NF4_OK;
   }
 
@@ -200,13 +257,23 @@ nf4_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight w, const ui
   ga.act = X; ga.lora_w = B; ga.lora_act = hilo; ga.out = Y;
   ga.status = status;
   ga.pdl_mode = kPdlWaitLowRank;
+  ga.quant_type = w.quant_type; ga.dq = w.double_quant; ga.f16 = f16;
   if (launch_nf4_gemm(plan_nf4_gemm(0, M, N, K, r, sms), ga, strm, true) != cudaSuccess) return NF4_ERR_CUDA;
   return NF4_OK;
 }
 
-nf4_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, nf4_weight w, const uint16_t* A,
-                            const uint16_t* B, int32_t r, float s, const uint16_t* T, uint16_t* dX, float* dA,
-                            float* dB, void* ws, size_t ws_bytes, void* stream) {
+nf4_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight w, const uint16_t* A, const uint16_t* B,
+                            int32_t r, float s, uint16_t* Y, uint16_t* T_out, void* ws, size_t ws_bytes,
+                            void* stream) {
+  return qlora_linear_fwd_ex(QLORA_BF16, X, M, w, A, B, r, s, Y, T_out, ws, ws_bytes, stream);
+}
+
+nf4_status qlora_linear_bwd_ex(int32_t dtype, const uint16_t* dY, const uint16_t* X, int64_t M, nf4_weight w,
+                               const uint16_t* A, const uint16_t* B, int32_t r, float s, const uint16_t* T,
+                               uint16_t* dX, float* dA, float* dB, void* ws, size_t ws_bytes, void* stream) {
+  if (!dtype_ok(dtype)) return NF4_ERR_INVALID_ARG;
+  const int f16 = dtype == QLORA_F16 ? 1 : 0;
+  const int hk = operand_kind(dtype);
   nf4_status st = check_linear_shapes(M, w, r);
   if (st != NF4_OK) return st;
   if (!dY || !X || !A || !B || !dX || !dA || !dB) return NF4_ERR_INVALID_ARG;
@@ -231,23 +298,29 @@ nf4_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, nf
     // dX = bf16(dY Wd + G A^T); dA = X^T G; dB = s T^T dY
     uint16_t* wd = reinterpret_cast<uint16_t*>(wsb + L.wd);
     float* g = reinterpret_cast<float*>(wsb + L.g);
-    if (launch_dequant(w.packed, w.c1q, w.c2, N * K, wd, sms, strm) != cudaSuccess) return NF4_ERR_CUDA;
+    if (launch_dequant(w.packed, w.c1q, w.c2, N * K, w.quant_type, w.double_quant, f16, wd, sms, strm) !=
+        cudaSuccess)
+      return NF4_ERR_CUDA;
     const uint16_t* Tin = T;
     if (!Tin) {
       uint16_t* tw = reinterpret_cast<uint16_t*>(wsb + L.t_scratch);
-      const GenericGemm gt = generic_product(M, r, bf16_operand(X, K, 1), bf16_operand(A, 1, r), K, 1.0f, tw, false);
+      const GenericGemm gt = generic_product(M, r, half_operand(hk, X, K, 1), half_operand(hk, A, 1, r), K, 1.0f,
+                                             tw, hk);
       if (launch_generic_gemm(gt, sms, strm) != cudaSuccess) return NF4_ERR_CUDA;
       Tin = tw;
     }
-    const GenericGemm gg = generic_product(M, r, bf16_operand(dY, N, 1), bf16_operand(B, N, 1), N, s, g, true);
+    const GenericGemm gg = generic_product(M, r, half_operand(hk, dY, N, 1), half_operand(hk, B, N, 1), N, s, g,
+                                           kOpF32);
     if (launch_generic_gemm(gg, sms, strm) != cudaSuccess) return NF4_ERR_CUDA;
-    GenericGemm gx = generic_product(M, K, bf16_operand(dY, N, 1), bf16_operand(wd, 1, K), N, 1.0f, dX, false);
+    GenericGemm gx = generic_product(M, K, half_operand(hk, dY, N, 1), half_operand(hk, wd, 1, K), N, 1.0f, dX, hk);
     gx.nseg = 2;
-    gx.seg[1] = GenericSegment{f32_operand(g, r, 1), bf16_operand(A, r, 1), r, 1.0f};
+    gx.seg[1] = GenericSegment{f32_operand(g, r, 1), half_operand(hk, A, r, 1), r, 1.0f};
     if (launch_generic_gemm(gx, sms, strm) != cudaSuccess) return NF4_ERR_CUDA;
-    const GenericGemm ga = generic_product(K, r, bf16_operand(X, 1, K), f32_operand(g, 1, r), M, 1.0f, dA, true);
+    const GenericGemm ga = generic_product(K, r, half_operand(hk, X, 1, K), f32_operand(g, 1, r), M, 1.0f, dA,
+                                           kOpF32);
     if (launch_generic_gemm(ga, sms, strm) != cudaSuccess) return NF4_ERR_CUDA;
-    const GenericGemm gb = generic_product(r, N, bf16_operand(Tin, 1, r), bf16_operand(dY, 1, N), M, s, dB, true);
+    const GenericGemm gb = generic_product(r, N, half_operand(hk, Tin, 1, r), half_operand(hk, dY, 1, N), M, s, dB,
+                                           kOpF32);
     if (launch_generic_gemm(gb, sms, strm) != cudaSuccess) return NF4_ERR_CUDA;
     return NF4_OK;
   }
@@ -256,6 +329,7 @@ nf4_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, nf
   sa.M = M; sa.N = N; sa.K = K; sa.r = r; sa.rp = rp; sa.s = s;
   sa.X = X; sa.dY = dY; sa.A = A; sa.B = B;
   sa.status = status;
+  sa.f16 = f16;
 
   // Launch order and overlap: the first kernel waits for all earlier work of
   // the stream; each later one is a programmatic dependent of the one before.
@@ -287,6 +361,7 @@ nf4_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, nf
   ga.act = dY; ga.lora_w = A; ga.lora_act = hilo; ga.out = dX;
   ga.status = status;
   ga.pdl_mode = kPdlWaitFirst;
+  ga.quant_type = w.quant_type; ga.dq = w.double_quant; ga.f16 = f16;
   if (launch_nf4_gemm(plan_nf4_gemm(1, M, N, K, r, sms), ga, strm, true) != cudaSuccess) return NF4_ERR_CUDA;
 
   // dA = X^T G  (G hi + G lo)
@@ -299,6 +374,12 @@ nf4_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, nf
   sa.f32_out = dB;
   if (launch_skinny(plan_skinny(kSkinnyDB, M, N, K, r, sms), sa, strm, true) != cudaSuccess) return NF4_ERR_CUDA;
   return NF4_OK;
+}
+
+nf4_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, nf4_weight w, const uint16_t* A,
+                            const uint16_t* B, int32_t r, float s, const uint16_t* T, uint16_t* dX, float* dA,
+                            float* dB, void* ws, size_t ws_bytes, void* stream) {
+  return qlora_linear_bwd_ex(QLORA_BF16, dY, X, M, w, A, B, r, s, T, dX, dA, dB, ws, ws_bytes, stream);
 }
 
 nf4_status qlora_linear_plan(int64_t M, int64_t N, int64_t K, int32_t r, int32_t backward, int32_t num_sms,

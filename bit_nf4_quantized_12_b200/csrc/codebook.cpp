@@ -1,5 +1,7 @@
 // codebook.cpp -- builds the NF4 table on the host, once.
 //
+// (The uniform INT4 table of the format variants is built here as well.)
+//
 // NF4 ("从LoRA到QLoRA" §2.3; "QLoRA 原理精讲" §2.1): 16 quantiles of N(0,1)
 // taken at probabilities spaced uniformly, normalized to [-1, 1].  The table
 // has an exact zero so that zero weights and padding survive a round trip:
@@ -37,6 +39,25 @@ long double normal_quantile(long double p) {
   return z;
 }
 
+void set_thresholds(Codebook& cb) {
+  for (int i = 0; i < 15; ++i) {
+    // midpoint of two fp32 values is exact in double; round it down to fp32
+    double mid = (static_cast<double>(cb.code[i]) + static_cast<double>(cb.code[i + 1])) * 0.5;
+    float t = static_cast<float>(mid);
+    if (static_cast<double>(t) > mid) t = std::nextafter(t, -INFINITY);
+    cb.thr[i] = t;
+  }
+}
+
+// Uniform INT4 ("QLoRA 原理精讲" §2.1: the 16 integers -8..7, evenly spaced),
+// divided by 8 so that the table lies in [-1, 1]: code i = (i - 8) / 8.
+Codebook build_int4() {
+  Codebook cb{};
+  for (int i = 0; i < 16; ++i) cb.code[i] = static_cast<float>(i - 8) / 8.0f;
+  set_thresholds(cb);
+  return cb;
+}
+
 Codebook build() {
   Codebook cb{};
   const long double d = 0.5L * ((1.0L - 1.0L / 30.0L) + (1.0L - 1.0L / 32.0L));
@@ -48,13 +69,7 @@ Codebook build() {
   for (int i = 0; i < 7; ++i) cb.code[i] = static_cast<float>(neg[i] / scale);
   cb.code[7] = 0.0f;
   for (int i = 0; i < 8; ++i) cb.code[8 + i] = static_cast<float>(pos[7 - i] / scale);
-  for (int i = 0; i < 15; ++i) {
-    // midpoint of two fp32 values is exact in double; round it down to fp32
-    double mid = (static_cast<double>(cb.code[i]) + static_cast<double>(cb.code[i + 1])) * 0.5;
-    float t = static_cast<float>(mid);
-    if (static_cast<double>(t) > mid) t = std::nextafter(t, -INFINITY);
-    cb.thr[i] = t;
-  }
+  set_thresholds(cb);
   return cb;
 }
 
@@ -64,6 +79,14 @@ const Codebook& host_codebook() {
   static Codebook cb;
   static std::once_flag once;
   std::call_once(once, [] { cb = build(); });
+  return cb;
+}
+
+const Codebook& host_codebook(int quant_type) {
+  if (quant_type != kQuantInt4) return host_codebook();
+  static Codebook cb;
+  static std::once_flag once;
+  std::call_once(once, [] { cb = build_int4(); });
   return cb;
 }
 

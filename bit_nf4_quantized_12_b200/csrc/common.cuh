@@ -175,12 +175,16 @@ NF4_DEV void mma_commit(uint64_t* bar) {
                : "memory");
 }
 
-// Instruction descriptor, kind::f16: bf16 A/B, fp32 D, dense.
-//   bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16), 10-12 B format,
-//   15 A major (0 = K, 1 = MN), 16 B major, 17-22 N>>3, 24-28 M>>4.
+// Instruction descriptor, kind::f16: bf16 (or fp16) A/B, fp32 D, dense.
+//   bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16, 0 = f16), 10-12 B
+//   format, 15 A major (0 = K, 1 = MN), 16 B major, 17-22 N>>3, 24-28 M>>4.
+// A and B always share one type.
+__host__ __device__ constexpr uint32_t make_idesc(int M, int N, int a_mn_major, int b_mn_major, bool f16) {
+  return (1u << 4) | (f16 ? 0u : (1u << 7) | (1u << 10)) | (uint32_t(a_mn_major) << 15) |
+         (uint32_t(b_mn_major) << 16) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
 __host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, int a_mn_major, int b_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(a_mn_major) << 15) | (uint32_t(b_mn_major) << 16) |
-         (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+  return make_idesc(M, N, a_mn_major, b_mn_major, false);
 }
 
 // Shared-memory matrix descriptor (sm_100 layout): start>>4 in bits 0-13,
@@ -260,6 +264,22 @@ NF4_DEV uint32_t pack_bf16x2(float lo, float hi) {
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
+// Same for IEEE fp16 (the FP16 compute type).
+NF4_DEV uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// Compute-type helpers: f16 selects IEEE fp16, else bf16 (16-bit patterns).
+NF4_DEV uint32_t pack2(bool f16, float lo, float hi) { return f16 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi); }
+NF4_DEV float half_lo_to_f32(bool f16, uint32_t two) {
+  return f16 ? __half2float(__ushort_as_half(static_cast<unsigned short>(two & 0xFFFFu))) : __uint_as_float(two << 16);
+}
+NF4_DEV float half_hi_to_f32(bool f16, uint32_t two) {
+  return f16 ? __half2float(__ushort_as_half(static_cast<unsigned short>(two >> 16))) : __uint_as_float(two & 0xFFFF0000u);
+}
+// x rounded to the compute type (nearest even), as fp32.
+NF4_DEV float round_to(bool f16, float x) { return half_lo_to_f32(f16, pack2(f16, x, 0.0f)); }
 NF4_DEV uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t r;
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));

@@ -39,6 +39,14 @@ struct Codebook {
   float thr[15];
 };
 
-// Built once on the host (codebook.cpp).
+// Table selectors (include/qlora_nf4.h NF4_QUANT_*).
+constexpr int kQuantNf4 = 0;
+constexpr int kQuantInt4 = 1;
+
+// Built once on the host (codebook.cpp): the NF4 table, or the table of a
+// quant_type.
 const Codebook& host_codebook();
+const Codebook& host_codebook(int quant_type);
+// Index of the exact 0.0 code of a quant_type's table.
+inline int zero_code(int quant_type) { return quant_type == kQuantInt4 ? 8 : kCodeZero; }
 }  // namespace nf4

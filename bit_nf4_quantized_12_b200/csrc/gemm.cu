@@ -214,8 +214,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
     // A operand layouts: forward main steps K-major (rows of W), backward
     // main steps MN-major (columns of W), forward low-rank steps MN-major
     // (B^T by TMA), backward low-rank steps K-major (A by TMA).
-    const uint32_t idesc_k = make_idesc_bf16(128, bt, 0, 0);
-    const uint32_t idesc_mn = make_idesc_bf16(128, bt, 1, 0);
+    const uint32_t idesc_k = make_idesc(128, bt, 0, 0, a.f16 != 0);
+    const uint32_t idesc_mn = make_idesc(128, bt, 1, 0, a.f16 != 0);
     for (int64_t ks = 0; ks < nsteps; ++ks) {
       const int sx = int(ks % SX), sa = int(ks % SA);
       if (!mbar_wait(&x_full[sx], uint32_t(ks / SX) & 1u, a.status, abort_flag)) break;
@@ -261,21 +261,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
       const int64_t kblk = w0 / 64 + (t >> 6);
       return (n < a.N && kblk < KB) ? n * KB + kblk : -1;
     };
+    const bool f16 = a.f16 != 0;
     uint32_t cq[4], nq[4];
     float cc[4], nc[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int64_t b = block_of(wg + int64_t(j) * kDequantWGs);
-      cq[j] = b >= 0 ? uint32_t(__ldg(a.c1q + b)) : 0u;
-      cc[j] = b >= 0 ? __ldg(a.c2 + (b >> 8)) : 0.0f;
+      cq[j] = 0u;
+      cc[j] = 0.0f;
+      if (b >= 0) load_scale_parts(a.dq, a.c1q, a.c2, b, cq[j], cc[j]);
     }
     bool ok = true;
     for (int64_t base = wg; base < nsteps && ok; base += 4 * kDequantWGs) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int64_t b = block_of(base + int64_t(4 + j) * kDequantWGs);
-        nq[j] = b >= 0 ? uint32_t(__ldg(a.c1q + b)) : 0u;
-        nc[j] = b >= 0 ? __ldg(a.c2 + (b >> 8)) : 0.0f;
+        nq[j] = 0u;
+        nc[j] = 0.0f;
+        if (b >= 0) load_scale_parts(a.dq, a.c1q, a.c2, b, nq[j], nc[j]);
       }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -295,7 +298,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
           __syncwarp();
           if (lane == 0) mbar_arrive(&p_empty[sp]);
           uint32_t o[32];
-          dequant64(make_table(P.code, e4m3_to_f32(cq[j]) * cc[j]), p0, p1, o);
+          dequant64(make_table(P.code, scale_from_parts(a.dq, cq[j], cc[j]), f16), p0, p1, o);
           // the A slot must have been released by the MMA of step ks - SA
           if (ks >= SA && !(ok = mbar_wait(&a_empty[sa], a_ph ^ 1u, a.status, abort_flag))) break;
           // forward: row t of Wd (K-major, 128-byte rows); backward: row
@@ -361,7 +364,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
         // ring, then write whole 16-byte pieces of output rows.
         const uint32_t stg = smem_u32(act_s) + uint32_t(c) * (32 * 256);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) sts16(stg + j * 256 + t * 2, pack_bf16x2(__uint_as_float(v[j]), 0.0f));
+        for (int j = 0; j < 32; ++j) sts16(stg + j * 256 + t * 2, pack2(a.f16 != 0, __uint_as_float(v[j]), 0.0f));
         warpgroup_sync(1 + wg);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -407,7 +410,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
           for (int q = 0; q < 8; ++q) acc += part[u][q];
           const int cu = col + u * kDequantWGs;
           const int64_t m = m0 + cu;
-          if (cu < c0 + cps && i < wdim && m < a.M) a.out[m * wdim + i] = uint16_t(pack_bf16x2(acc, 0.0f) & 0xFFFFu);
+          if (cu < c0 + cps && i < wdim && m < a.M)
+            a.out[m * wdim + i] = uint16_t(pack2(a.f16 != 0, acc, 0.0f) & 0xFFFFu);
         }
       }
     }
@@ -438,12 +442,12 @@ struct SkinnyParams {
   int64_t rows;
 };
 
-__device__ __forceinline__ uint32_t bf16_bits(float x) { return pack_bf16x2(x, 0.0f) & 0xFFFFu; }
 
 // Final values of eight consecutive columns j0..j0+7 of row i (j0 % 8 == 0):
 // one 16-byte store per output row segment where the row holds all eight.
 __device__ __forceinline__ void skinny_finish8(const SkinnyParams& P, int64_t i, int j0, const float (&acc)[8]) {
   const SkinnyArgs& a = P.a;
+  const bool f16 = a.f16 != 0;
   switch (P.kind) {
     case kSkinnyT:
     case kSkinnyG: {
@@ -456,16 +460,16 @@ __device__ __forceinline__ void skinny_finish8(const SkinnyParams& P, int64_t i,
         for (int h = 0; h < 2; ++h) {
           const int j = j0 + 2 * u + h;
           if (P.kind == kSkinnyT) {
-            const float tval = __uint_as_float(bf16_bits(acc[2 * u + h]) << 16);   // T in bf16
+            const float tval = round_to(f16, acc[2 * u + h]);   // T in the compute type
             v[h] = (j < a.r) ? a.s * tval : 0.0f;
           } else {
             v[h] = (j < a.r) ? a.s * acc[2 * u + h] : 0.0f;
           }
         }
-        tb[u] = pack_bf16x2(acc[2 * u], acc[2 * u + 1]);
-        hi[u] = pack_bf16x2(v[0], v[1]);
-        const float h0 = __uint_as_float(hi[u] << 16), h1 = __uint_as_float(hi[u] & 0xFFFF0000u);
-        lo[u] = pack_bf16x2(v[0] - h0, v[1] - h1);
+        tb[u] = pack2(f16, acc[2 * u], acc[2 * u + 1]);
+        hi[u] = pack2(f16, v[0], v[1]);
+        const float h0 = half_lo_to_f32(f16, hi[u]), h1 = half_hi_to_f32(f16, hi[u]);
+        lo[u] = pack2(f16, v[0] - h0, v[1] - h1);
       }
       uint16_t* row = a.hilo_out + i * 2 * a.rp;
       *reinterpret_cast<uint4*>(row + j0) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
@@ -585,7 +589,7 @@ __global__ void __launch_bounds__(kSkinnyThreads, 2) skinny_gemm_kernel(const __
     }
     __syncwarp();
   } else if (warp == 1) {
-    const uint32_t idesc = make_idesc_bf16(128, rp, P.a_mn, P.b_mn);
+    const uint32_t idesc = make_idesc(128, rp, P.a_mn, P.b_mn, a.f16 != 0);
     for (int64_t ks = 0; ks < nsteps; ++ks) {
       const int s = int(ks % kSkinnyStages);
       const uint32_t ph = uint32_t(ks / kSkinnyStages) & 1u;
@@ -805,8 +809,9 @@ cudaError_t launch_nf4_gemm(const Nf4GemmPlan& plan, const Nf4GemmArgs& a, cudaS
   P.splits = plan.splits;
   P.main_steps = plan.main_steps;
   P.lora_steps = plan.lora_steps;
-  const Codebook& cb = host_codebook();
+  const Codebook& cb = host_codebook(a.quant_type);
   for (int i = 0; i < 16; ++i) P.code.v[i] = cb.code[i];
+  // 2-byte elements; TMA only moves them, so bf16 and fp16 share the map type
   const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
   const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
@@ -843,7 +848,7 @@ cudaError_t launch_skinny(const SkinnyPlan& plan, const SkinnyArgs& a, cudaStrea
   P.steps = plan.steps;
   P.rows = plan.rows;
   P.pass_steps = plan.steps;
-  const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;   // 2-byte elements (bf16 or fp16)
   const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
   const uint64_t M = a.M, N = a.N, K = a.K, r = uint64_t(a.r), rp = uint64_t(a.rp);
   bool ok = true;

@@ -52,24 +52,37 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
 __device__ __forceinline__ uint32_t x_chunk(int64_t kb, int i) {
   return uint32_t(kb) * 128u + uint32_t((i ^ int(kb & 7)) * 16);
 }
-// acc += x.lo * w.lo, then acc += x.hi * w.hi, for two bf16 pairs: an fp32
-// fma on bf16 operands, equal to widening them first (their product is exact
-// in fp32) but without the integer work of the widening
-__device__ __forceinline__ float fma2_bf16(uint32_t x2, uint32_t w2, float acc) {
-  asm("{\n\t.reg .b16 xl, xh, wl, wh;\n\t"
-      "mov.b32 {xl, xh}, %1;\n\t"
-      "mov.b32 {wl, wh}, %2;\n\t"
-      "fma.rn.f32.bf16 %0, xl, wl, %0;\n\t"
-      "fma.rn.f32.bf16 %0, xh, wh, %0;\n\t}"
-      : "+f"(acc)
-      : "r"(x2), "r"(w2));
+// acc += x.lo * w.lo, then acc += x.hi * w.hi, for two bf16 (or fp16) pairs:
+// an fp32 fma on 16-bit operands, equal to widening them first (their product
+// is exact in fp32) but without the integer work of the widening
+template <bool F16>
+__device__ __forceinline__ float fma2_half(uint32_t x2, uint32_t w2, float acc) {
+  if (F16) {
+    asm("{\n\t.reg .b16 xl, xh, wl, wh;\n\t"
+        "mov.b32 {xl, xh}, %1;\n\t"
+        "mov.b32 {wl, wh}, %2;\n\t"
+        "fma.rn.f32.f16 %0, xl, wl, %0;\n\t"
+        "fma.rn.f32.f16 %0, xh, wh, %0;\n\t}"
+        : "+f"(acc)
+        : "r"(x2), "r"(w2));
+  } else {
+    asm("{\n\t.reg .b16 xl, xh, wl, wh;\n\t"
+        "mov.b32 {xl, xh}, %1;\n\t"
+        "mov.b32 {wl, wh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, xl, wl, %0;\n\t"
+        "fma.rn.f32.bf16 %0, xh, wh, %0;\n\t}"
+        : "+f"(acc)
+        : "r"(x2), "r"(w2));
+  }
   return acc;
 }
 
-// sum over the 64 weights of block kb of x[k] * Wd[n, k]
-__device__ __forceinline__ float block_dot(const CodeTable& code, const uint4& p0, const uint4& p1, uint32_t q,
-                                           float c2, uint32_t xs, int64_t kb, float acc) {
-  const BlockTable t = make_table(code, e4m3_to_f32(q) * c2);
+// sum over the 64 weights of block kb of x[k] * Wd[n, k]; (q, c2) are the
+// block's first-level constant parts in storage format dq
+template <bool F16>
+__device__ __forceinline__ float block_dot(const CodeTable& code, const uint4& p0, const uint4& p1, int dq,
+                                           uint32_t q, float c2, uint32_t xs, int64_t kb, float acc) {
+  const BlockTable t = make_table(code, scale_from_parts(dq, q, c2), F16);
   const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -77,14 +90,15 @@ __device__ __forceinline__ float block_dot(const CodeTable& code, const uint4& p
     lookup4(t, w[i] & 0xFFFFu, o[0], o[1]);   // weights 8i .. 8i+3
     lookup4(t, w[i] >> 16, o[2], o[3]);       // weights 8i+4 .. 8i+7
     const uint4 xv = lds128(xs + x_chunk(kb, i));
-    acc = fma2_bf16(xv.x, o[0], acc);
-    acc = fma2_bf16(xv.y, o[1], acc);
-    acc = fma2_bf16(xv.z, o[2], acc);
-    acc = fma2_bf16(xv.w, o[3], acc);
+    acc = fma2_half<F16>(xv.x, o[0], acc);
+    acc = fma2_half<F16>(xv.y, o[1], acc);
+    acc = fma2_half<F16>(xv.z, o[2], acc);
+    acc = fma2_half<F16>(xv.w, o[3], acc);
   }
   return acc;
 }
 
+template <bool F16>
 __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_kernel(const __grid_constant__ GemvParams P) {
   extern __shared__ __align__(128) uint8_t smem[];
   const Nf4GemvArgs& a = P.a;
@@ -126,10 +140,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_kernel(const __grid_
       bulk_load(ring + s * kPiece, a.packed + n * (a.K / 2) + kb0 * 32, uint32_t(nb) * 32u, &full[s]);
     }
     const int64_t b = n * KB + kb0 + lane;
-    if (kb0 + lane < KB) {
-      q = __ldg(a.c1q + b);
-      c2 = __ldg(a.c2 + (b >> 8));
-    }
+    if (kb0 + lane < KB) load_scale_parts(a.dq, a.c1q, a.c2, b, q, c2);
   };
 
   for (int64_t first = warp0; first < a.N && ok; first += stride * kRows) {
@@ -165,7 +176,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_kernel(const __grid_
           const float cc = c2[s];
           // next piece of this slot: the same row, next pass
           issue(first, nrows, p + 1, r, q[s], c2[s]);
-          if (kb < KB) acc[r] = block_dot(P.code, p0, p1, qc, cc, xs, kb, acc[r]);
+          if (kb < KB) acc[r] = block_dot<F16>(P.code, p0, p1, a.dq, qc, cc, xs, kb, acc[r]);
         }
       }
     }
@@ -180,10 +191,11 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_kernel(const __grid_
         const int64_t n = first + int64_t(r) * stride;
         float v = acc[r];
         for (int j = lane; j < a.r; j += 32)
-          v = fmaf(a.s * bf16lo_to_f32(uint32_t(a.T[j])), bf16lo_to_f32(uint32_t(a.B[int64_t(j) * a.N + n])), v);
+          v = fmaf(a.s * half_lo_to_f32(F16, uint32_t(a.T[j])), half_lo_to_f32(F16, uint32_t(a.B[int64_t(j) * a.N + n])),
+                   v);
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) a.Y[n] = uint16_t(pack_bf16x2(v, 0.0f) & 0xFFFFu);
+        if (lane == 0) a.Y[n] = uint16_t(pack2(F16, v, 0.0f) & 0xFFFFu);
       }
     }
   }
@@ -215,7 +227,8 @@ cudaError_t launch_nf4_gemv(const Nf4GemvArgs& a, const float code[16], int num_
   P.a = a;
   for (int i = 0; i < 16; ++i) P.code.v[i] = code[i];
   const size_t smem = gemv_smem(a.K);
-  cudaError_t e = cudaFuncSetAttribute(nf4_gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  void (*kern)(const GemvParams) = a.f16 ? nf4_gemv_kernel<true> : nf4_gemv_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   // one CTA per SM, fewer when there are not enough rows for every warp
   int64_t blocks = int64_t(num_sms);
@@ -231,7 +244,7 @@ cudaError_t launch_nf4_gemv(const Nf4GemvArgs& a, const float code[16], int num_
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, nf4_gemv_kernel, P);
+  return cudaLaunchKernelEx(&cfg, kern, P);
 }
 
 }  // namespace nf4

@@ -2,14 +2,15 @@
 // does not take (K % 64 != 0, N % 8 != 0 or r % 8 != 0), for example a
 // weight whose rows do not start on an NF4 block ("从LoRA到QLoRA" §3.1;
 // "LoRA、Q-LoRA 与 PortLLM" §3.4 for the layer):
-//   forward : T = bf16(X A),  Y = bf16(X Wd^T + s T B)
-//   backward: G = s dY B^T,  dX = bf16(dY Wd + G A^T),  dA = X^T G,  dB = s T^T dY
+//   forward : T = rnd(X A),  Y = rnd(X Wd^T + s T B)
+//   backward: G = s dY B^T,  dX = rnd(dY Wd + G A^T),  dA = X^T G,  dB = s T^T dY
+// (rnd: round to the compute type, bf16 or fp16)
 // The weight is first dequantized exactly into the workspace by the
 // standalone dequant kernel (any shape), so unlike the fused path Wd reaches
 // memory here.  Every product then runs through one tiled CUDA-core kernel:
 // a 16 x 16 output tile per CTA, up to two reduction segments, operands read
-// through strided accessors (bf16 or fp32), fp32 accumulation in a fixed
-// order, bf16 (round to nearest even) or fp32 output.  Correctness first:
+// through strided accessors (bf16, fp16 or fp32), fp32 accumulation in a
+// fixed order, bf16 / fp16 (round to nearest even) or fp32 output.  Correctness first:
 // this path serves shapes outside the fused kernels, not throughput.
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -23,8 +24,8 @@ constexpr int kTile = 16;
 
 __device__ __forceinline__ float load_operand(const GenericOperand& o, int64_t i, int64_t p) {
   const int64_t idx = i * o.si + p * o.sp;
-  if (o.fp32) return static_cast<const float*>(o.base)[idx];
-  return __uint_as_float(uint32_t(static_cast<const uint16_t*>(o.base)[idx]) << 16);
+  if (o.kind == kOpF32) return static_cast<const float*>(o.base)[idx];
+  return half_lo_to_f32(o.kind == kOpF16, uint32_t(static_cast<const uint16_t*>(o.base)[idx]));
 }
 
 // tile[il][pl] = o(i0 + il, p0 + pl), zero outside [0, I) x [0, P); the
@@ -65,8 +66,8 @@ __global__ void __launch_bounds__(kTile * kTile) generic_gemm_kernel(const __gri
     }
     const int64_t i = i0 + ty, j = j0 + tx;
     if (i < g.I && j < g.J) {
-      if (g.out_fp32) static_cast<float*>(g.out)[i * g.J + j] = total;
-      else static_cast<uint16_t*>(g.out)[i * g.J + j] = uint16_t(pack_bf16x2(total, 0.0f) & 0xFFFFu);
+      if (g.out_kind == kOpF32) static_cast<float*>(g.out)[i * g.J + j] = total;
+      else static_cast<uint16_t*>(g.out)[i * g.J + j] = uint16_t(pack2(g.out_kind == kOpF16, total, 0.0f) & 0xFFFFu);
     }
   }
 }

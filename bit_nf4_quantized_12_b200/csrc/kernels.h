@@ -14,11 +14,32 @@ enum PdlMode : int {
   kPdlWaitLowRank = 2,  // fused GEMM: main product first, wait before the low-rank operand
 };
 
-cudaError_t launch_quantize(const uint16_t* W, int64_t numel, uint8_t* packed, uint8_t* c1q, float* c2,
-                            uint32_t* status, int num_sms, cudaStream_t stream);
-cudaError_t launch_dequant(const uint8_t* packed, const uint8_t* c1q, const float* c2, int64_t numel,
-                           uint16_t* out, int num_sms, cudaStream_t stream);
-bool quantize_table_ok();
+// Quantize W (numel bf16) into the storage format (quant_type: table;
+// dq: DqFormat of the first-level constants, c1 holds bytes or fp32).
+cudaError_t launch_quantize(const uint16_t* W, int64_t numel, int quant_type, int dq, uint8_t* packed, void* c1,
+                            float* c2, uint32_t* status, int num_sms, cudaStream_t stream);
+// Dequantize into the compute type (f16: fp16, else bf16).
+cudaError_t launch_dequant(const uint8_t* packed, const uint8_t* c1, const float* c2, int64_t numel,
+                           int quant_type, int dq, int f16, uint16_t* out, int num_sms, cudaStream_t stream);
+bool quantize_table_ok(int quant_type);
+
+// ---------------------------------------------------------------- LoRA merge
+// out[n, k] = round(Wd[n, k] + s sum_j A[k, j] B[j, n]) in the compute type.
+struct MergeArgs {
+  const uint8_t* packed;
+  const uint8_t* c1;      // first-level constants (bytes, or fp32 for dq == kDqNone)
+  const float* c2;
+  int64_t N, K;
+  int double_quant;       // DqFormat
+  const uint16_t* A;      // [K, r]
+  const uint16_t* B;      // [r, N]
+  int r;
+  float s;
+  int f16;                // compute type fp16 (else bf16)
+  uint16_t* out;          // [N, K]
+};
+cudaError_t launch_merge(const MergeArgs& a, const float code[16], cudaStream_t stream);
+size_t merge_smem_bytes(int r);
 
 // ---------------------------------------------------------------- fused NF4 GEMM
 // Computes, for a tile grid over (W-dim x tokens):
@@ -52,6 +73,9 @@ struct Nf4GemmArgs {
   uint16_t* out;             // Y [M, N] or dX [M, K], bf16
   uint32_t* status;          // kStatusTimeout on a failed wait
   int pdl_mode;              // PdlMode
+  int quant_type;            // table (kQuantNf4 / kQuantInt4)
+  int dq;                    // DqFormat of the first-level constants (c1q holds fp32 for kDqNone)
+  int f16;                   // compute type fp16 (else bf16)
 };
 // pdl: launch as a programmatic dependent of the previous kernel of the stream
 cudaError_t launch_nf4_gemm(const Nf4GemmPlan& plan, const Nf4GemmArgs& a, cudaStream_t stream, bool pdl);
@@ -89,6 +113,7 @@ struct SkinnyArgs {
   float* f32_out;           // kSkinnyDA / kSkinnyDB
   uint32_t* status;
   int pdl_mode;             // PdlMode (kPdlWaitFirst or kPdlWaitLast)
+  int f16;                  // compute type fp16 (else bf16)
 };
 cudaError_t launch_skinny(const SkinnyPlan& plan, const SkinnyArgs& a, cudaStream_t stream, bool pdl);
 
@@ -109,6 +134,8 @@ struct Nf4GemvArgs {
   const uint16_t* B;         // [r, N] bf16
   uint16_t* Y;               // [M, N] bf16
   uint32_t* status;          // kStatusTimeout on a failed wait
+  int dq;                    // DqFormat of the first-level constants
+  int f16;                   // compute type fp16 (else bf16) for X, T, B, Y
 };
 // Whether the GEMV takes this problem (one token, K within its shared memory).
 bool gemv_supported(int64_t M, int64_t K);
@@ -117,12 +144,13 @@ cudaError_t launch_nf4_gemv(const Nf4GemvArgs& a, const float code[16], int num_
 // ---------------------------------------------------------------- generic GEMM
 // C[i, j] = sum over segments of scale * sum_p a(i, p) b(j, p), on CUDA cores,
 // for the linear layer's shapes outside the fused kernels.  An operand
-// element (i, p) sits at base[i * si + p * sp] (bf16 or fp32); C is [I, J]
-// row-major, bf16 (round to nearest even) or fp32.
+// element (i, p) sits at base[i * si + p * sp] (bf16, fp16 or fp32); C is
+// [I, J] row-major, bf16 / fp16 (round to nearest even) or fp32.
+enum OperandKind : int { kOpBF16 = 0, kOpF32 = 1, kOpF16 = 2 };
 struct GenericOperand {
   const void* base;
   int64_t si, sp;
-  int fp32;
+  int kind;        // OperandKind
 };
 struct GenericSegment {
   GenericOperand a, b;
@@ -134,7 +162,7 @@ struct GenericGemm {
   int nseg;        // 1 or 2
   GenericSegment seg[2];
   void* out;
-  int out_fp32;
+  int out_kind;    // OperandKind
 };
 cudaError_t launch_generic_gemm(const GenericGemm& g, int num_sms, cudaStream_t stream);
 

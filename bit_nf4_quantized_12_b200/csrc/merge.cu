@@ -1,0 +1,222 @@
+// merge.cu -- merging the LoRA adapter into the frozen weight for serving:
+//
+//     W' = round(Wd + s (A B)^T),   Wd = dequant(packed, scale1, scale2),
+//
+// "QLoRA 原理精讲" §2.5 (after merging, the weights are BF16 again and
+// inference runs at the original speed) and §三 误区3 (deployment path ②:
+// merge the adapter back, then re-quantize for inference).
+//
+// Per element: wd = round(fp32(code[q] * scale1')) exactly as the standalone
+// dequantization; p = sum_j A[k,j] B[j,n] in fp32 on the tensor cores
+// (mma.sync m16n8k16, exact products, fp32 accumulation); v = fma(s, p, wd)
+// in fp32; W' = round(v) to the compute type.  The kernel is bound by HBM:
+// it reads 0.5 byte of packed code per weight and writes the 2-byte result;
+// the rank-r product adds 2 r flops per weight, which the tensor cores absorb.
+//
+// Tiling: one CTA per 128 (rows of W) x 128 (columns) output tile, 8 warps.
+// The tile's slices of B^T [128 x r] and A [128 x r] are staged in shared
+// memory (zero padded to r rounded up to 16), each warp forms a 32 x 64 part
+// of p with ldmatrix + mma.sync, the whole tile of p is parked in shared
+// memory (over the operand slices), and the epilogue walks each row in
+// 8-column pieces: one 4-byte load of packed codes, one block scale, one
+// 16-byte store, all coalesced along the row.
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include "common.cuh"
+#include "kernels.h"
+#include "nf4_lut.cuh"
+
+namespace nf4 {
+namespace {
+
+constexpr int kMergeThreads = 256;
+constexpr int kTile = 128;             // rows and columns of W per CTA
+constexpr int kPStride = kTile + 4;    // floats per row of the parked product
+
+struct MergeParams {
+  MergeArgs a;
+  float code[16];
+  int rp;                              // r rounded up to 16
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+template <bool F16>
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  if (F16) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  } else {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+}
+
+template <bool F16>
+__global__ void __launch_bounds__(kMergeThreads) nf4_merge_kernel(const __grid_constant__ MergeParams P) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const MergeArgs& a = P.a;
+  const int rp = P.rp;
+  const int srow = (rp + 8) * 2;                 // bytes per staged operand row (ldmatrix conflict-free)
+  uint8_t* bt_s = smem;                          // B^T slice [128 rows of W][rp]
+  uint8_t* a_s = smem + kTile * srow;            // A slice   [128 columns of W][rp]
+  float* p_s = reinterpret_cast<float*>(smem);   // parked product [128][kPStride], after the MMAs
+  __shared__ float code_s[16];
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t k0 = int64_t(blockIdx.x) * kTile;
+  const int64_t n0 = int64_t(blockIdx.y) * kTile;
+  if (tid < 16) code_s[tid] = P.code[tid];
+
+  // ---- stage the operand slices (zero padded past r, N and K)
+  const int jc = rp / 8;                         // 8-wide chunks per operand row
+  for (int i = tid; i < kTile * jc; i += kMergeThreads) {   // A[k0 + row][8c .. 8c+7]
+    const int row = i / jc, c = i % jc;
+    const int64_t k = k0 + row;
+    uint32_t v[4] = {0u, 0u, 0u, 0u};
+    if (k < a.K) {
+      const uint16_t* src = a.A + k * a.r + c * 8;
+      if (c * 8 + 8 <= a.r && (a.r % 8) == 0) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(src));
+        v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
+      } else {
+        for (int j = 0; j < 8; ++j)
+          if (c * 8 + j < a.r) v[j >> 1] |= uint32_t(src[j]) << (16 * (j & 1));
+      }
+    }
+    *reinterpret_cast<uint4*>(a_s + row * srow + c * 16) = make_uint4(v[0], v[1], v[2], v[3]);
+  }
+  constexpr int nc = kTile / 8;                  // 8-wide chunks of a row of B's slice
+  for (int i = tid; i < rp * nc; i += kMergeThreads) {     // B[j][n0 + 8c .. n0 + 8c + 7] -> B^T rows
+    const int j = i / nc, c = i % nc;
+    uint16_t v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (j < a.r) {
+      const int64_t nb = n0 + c * 8;
+      const uint16_t* src = a.B + int64_t(j) * a.N + nb;
+      if (nb + 8 <= a.N && (a.N % 8) == 0) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(src));
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        for (int q = 0; q < 8; ++q) v[q] = uint16_t(w[q >> 1] >> (16 * (q & 1)));
+      } else {
+        for (int q = 0; q < 8; ++q)
+          if (nb + q < a.N) v[q] = src[q];
+      }
+    }
+    for (int q = 0; q < 8; ++q) *reinterpret_cast<uint16_t*>(bt_s + (c * 8 + q) * srow + j * 2) = v[q];
+  }
+  __syncthreads();
+
+  // ---- p = B^T A^T over the rank: warp (wn, wk) owns rows wn*32.. and columns wk*64..
+  const int wn = warp & 3, wk = warp >> 2;
+  float acc[2][8][4];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[mt][nt][q] = 0.0f;
+  const uint32_t bt_base = smem_u32(bt_s), a_base = smem_u32(a_s);
+  for (int kk = 0; kk < rp / 16; ++kk) {
+    uint32_t af[2][4];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+      const int row = wn * 32 + mt * 16 + (lane & 15);
+      const int col = kk * 16 + (lane >> 4) * 8;
+      ldsm_x4(bt_base + row * srow + col * 2, af[mt][0], af[mt][1], af[mt][2], af[mt][3]);
+    }
+#pragma unroll
+    for (int np = 0; np < 4; ++np) {               // pairs of 8-column MMA tiles
+      const int row = wk * 64 + np * 16 + (lane & 7) + ((lane >> 4) << 3);
+      const int col = kk * 16 + ((lane >> 3) & 1) * 8;
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4(a_base + row * srow + col * 2, b0, b1, b2, b3);
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        mma16816<F16>(acc[mt][2 * np], af[mt], b0, b1);
+        mma16816<F16>(acc[mt][2 * np + 1], af[mt], b2, b3);
+      }
+    }
+  }
+  __syncthreads();                                  // operand slices are dead: park p over them
+  {
+    const int g = lane >> 2, c = lane & 3;
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        const int row = wn * 32 + mt * 16 + g;
+        const int col = wk * 64 + nt * 8 + 2 * c;
+        *reinterpret_cast<float2*>(p_s + row * kPStride + col) = make_float2(acc[mt][nt][0], acc[mt][nt][1]);
+        *reinterpret_cast<float2*>(p_s + (row + 8) * kPStride + col) = make_float2(acc[mt][nt][2], acc[mt][nt][3]);
+      }
+  }
+  __syncthreads();
+
+  // ---- epilogue: W' = round(fma(s, p, wd)), 8 columns of one row per piece
+  const bool vec = (a.K % 8) == 0;
+  for (int i = tid; i < kTile * (kTile / 8); i += kMergeThreads) {
+    const int row = i >> 4, pc = i & 15;
+    const int64_t n = n0 + row;
+    const int64_t k = k0 + pc * 8;
+    if (n >= a.N || k >= a.K) continue;
+    const float* pr = p_s + row * kPStride + pc * 8;
+    if (vec) {
+      // K % 8 == 0: the 8 weights share one packed word and one block
+      const int64_t e0 = n * a.K + k;
+      const uint32_t w = __ldcs(reinterpret_cast<const unsigned int*>(a.packed + (e0 >> 1)));
+      const float s1 = block_scale(a.double_quant, a.c1, a.c2, e0 >> 6);
+      uint32_t o[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float wd0 = round_to(F16, code_s[(w >> (8 * h)) & 0xFu] * s1);
+        const float wd1 = round_to(F16, code_s[(w >> (8 * h + 4)) & 0xFu] * s1);
+        o[h] = pack2(F16, fmaf(a.s, pr[2 * h], wd0), fmaf(a.s, pr[2 * h + 1], wd1));
+      }
+      __stcs(reinterpret_cast<uint4*>(a.out + e0), make_uint4(o[0], o[1], o[2], o[3]));
+    } else {
+      for (int q = 0; q < 8 && k + q < a.K; ++q) {
+        const int64_t e = n * a.K + k + q;
+        const uint32_t byte = a.packed[e >> 1];
+        const uint32_t code = (e & 1) ? (byte >> 4) : (byte & 0xFu);
+        const float wd = round_to(F16, code_s[code] * block_scale(a.double_quant, a.c1, a.c2, e >> 6));
+        a.out[e] = uint16_t(pack2(F16, fmaf(a.s, pr[q], wd), 0.0f) & 0xFFFFu);
+      }
+    }
+  }
+}
+
+}  // namespace
+
+size_t merge_smem_bytes(int r) {
+  const int rp = (r + 15) / 16 * 16;
+  const size_t operands = size_t(2) * kTile * (rp + 8) * 2;
+  const size_t parked = size_t(kTile) * kPStride * 4;
+  return operands > parked ? operands : parked;
+}
+
+cudaError_t launch_merge(const MergeArgs& a, const float code[16], cudaStream_t stream) {
+  MergeParams P;
+  P.a = a;
+  for (int i = 0; i < 16; ++i) P.code[i] = code[i];
+  P.rp = (a.r + 15) / 16 * 16;
+  const size_t smem = merge_smem_bytes(a.r);
+  void (*kern)(const MergeParams) = a.f16 ? nf4_merge_kernel<true> : nf4_merge_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  const dim3 grid(unsigned((a.K + kTile - 1) / kTile), unsigned((a.N + kTile - 1) / kTile));
+  kern<<<grid, kMergeThreads, smem, stream>>>(P);
+  return cudaGetLastError();
+}
+
+}  // namespace nf4

@@ -15,17 +15,17 @@ struct CodeTable {
   float v[16];
 };
 
-// 16-entry bf16 table of one block (code[q] * scale1, each an fp32 multiply
-// rounded to bf16) split into low-byte and high-byte planes so that four
-// lookups are a handful of byte permutes.
+// 16-entry table of one block in the compute type (code[q] * scale1, each an
+// fp32 multiply rounded to bf16, or to fp16) split into low-byte and
+// high-byte planes so that four lookups are a handful of byte permutes.
 struct BlockTable {
   uint32_t lo[4], hi[4];
 };
 
-__device__ __forceinline__ BlockTable make_table(const CodeTable& code, float s1) {
+__device__ __forceinline__ BlockTable make_table(const CodeTable& code, float s1, bool f16 = false) {
   uint32_t pr[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) pr[i] = pack_bf16x2(code.v[2 * i] * s1, code.v[2 * i + 1] * s1);
+  for (int i = 0; i < 8; ++i) pr[i] = pack2(f16, code.v[2 * i] * s1, code.v[2 * i + 1] * s1);
   BlockTable t;
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
@@ -55,6 +55,40 @@ __device__ __forceinline__ void dequant64(const BlockTable& t, const uint4& p0, 
     lookup4(t, w[i] & 0xFFFFu, o[4 * i + 0], o[4 * i + 1]);
     lookup4(t, w[i] >> 16, o[4 * i + 2], o[4 * i + 3]);
   }
+}
+
+}  // namespace nf4
+
+namespace nf4 {
+
+// First-level constant of block b in each storage format (include/qlora_nf4.h
+// NF4_DQ_*): FP8 E4M3 code times the group's FP32 scale2 (the method,
+// "QLoRA 原理精讲" §2.2), the FP32 scale1 itself, or an unsigned 8-bit code
+// times scale2.  One fp32 multiply where there are two levels.
+enum DqFormat : int { kDqE4M3 = 0, kDqNone = 1, kDqU8 = 2 };
+
+__device__ __forceinline__ float block_scale(int dq, const uint8_t* c1, const float* c2, int64_t b) {
+  if (dq == kDqNone) return __ldg(reinterpret_cast<const float*>(c1) + b);
+  const uint32_t q = __ldg(c1 + b);
+  const float s2 = __ldg(c2 + (b >> 8));
+  return (dq == kDqU8 ? float(q) : e4m3_to_f32(q)) * s2;
+}
+
+// Raw first-level value of block b as loaded ahead of use: the 8-bit code or
+// the FP32 bits, and the group's scale2 (0 for kDqNone).
+__device__ __forceinline__ void load_scale_parts(int dq, const uint8_t* c1, const float* c2, int64_t b,
+                                                 uint32_t& q, float& s2) {
+  if (dq == kDqNone) {
+    q = __float_as_uint(__ldg(reinterpret_cast<const float*>(c1) + b));
+    s2 = 0.0f;
+  } else {
+    q = __ldg(c1 + b);
+    s2 = __ldg(c2 + (b >> 8));
+  }
+}
+__device__ __forceinline__ float scale_from_parts(int dq, uint32_t q, float s2) {
+  if (dq == kDqNone) return __uint_as_float(q);
+  return (dq == kDqU8 ? float(q) : e4m3_to_f32(q)) * s2;
 }
 
 }  // namespace nf4

@@ -17,6 +17,11 @@
 // Dequantize ("QLoRA 原理精讲" §2.2, reverse order): scale1' = fp32(E4M3 value
 // of c1q * scale2), w' = bf16(fp32(code * scale1')).
 //
+// Both kernels also take the storage variants (a uniform INT4 table; FP32 or
+// unsigned 8-bit first-level constants) and dequantize into fp16 as well as
+// bf16: the table, the per-block constant and the final rounding change,
+// nothing else.
+//
 // Both kernels are HBM-bandwidth bound: 16-byte coalesced loads and stores,
 // the per-block absmax by warp shuffles across the 8 lanes that own a block,
 // and the code decision as one lookup in a 33-cell shared-memory table plus
@@ -26,6 +31,7 @@
 #include <cuda_bf16.h>
 #include "common.cuh"
 #include "kernels.h"
+#include "nf4_lut.cuh"
 
 namespace nf4 {
 namespace {
@@ -102,10 +108,12 @@ struct QuantArgs {
   const uint16_t* W;
   int64_t numel;
   uint8_t* packed;
-  uint8_t* c1q;
-  float* c2;
+  uint8_t* c1q;        // first-level constants: bytes, or fp32 values for kDqNone
+  float* c2;           // unused for kDqNone
   uint32_t* status;
   int64_t ngroups;
+  int dq;              // DqFormat
+  uint32_t zero8;      // eight nibbles of the table's 0.0 code (all-zero blocks)
   float thr[15];
 };
 
@@ -183,8 +191,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2) nf4_quantize_kernel(const __
     // computes that block's code and reciprocal once; the others receive the
     // reciprocal by shuffle.
     const float gmax = __uint_as_float(gm << 16);
-    const float s2 = __fdiv_rn(gmax, 448.0f);
-    if (tid == 0) p.c2[g] = s2;
+    const float s2 = __fdiv_rn(gmax, p.dq == kDqU8 ? 255.0f : 448.0f);
+    if (tid == 0 && p.dq != kDqNone) p.c2[g] = s2;
     const int j = lane & 7;
     uint32_t my_bm = bm[0];
 #pragma unroll
@@ -192,8 +200,16 @@ __global__ void __launch_bounds__(kQuantThreads, 2) nf4_quantize_kernel(const __
     const float my_c1 = __uint_as_float(my_bm << 16);
     if (j < kQuantIters) {
       const int64_t b = g * kGroup + int64_t(j) * (kQuantThreads / 8) + (tid >> 3);
-      if (b < nblk_total)
-        p.c1q[b] = (my_c1 == 0.0f) ? uint8_t(0) : uint8_t(f32_to_e4m3_satfinite(__fdiv_rn(my_c1, s2)));
+      if (b < nblk_total) {
+        if (p.dq == kDqNone) {
+          reinterpret_cast<float*>(p.c1q)[b] = my_c1;
+        } else if (my_c1 == 0.0f) {
+          p.c1q[b] = 0;
+        } else {
+          const float t = __fdiv_rn(my_c1, s2);
+          p.c1q[b] = uint8_t(p.dq == kDqU8 ? min(__float2uint_rn(t), 255u) : f32_to_e4m3_satfinite(t));
+        }
+      }
     }
     // 16 / scale1 must stay a finite normal number: scale1 in [2^-122, 2^125]
     const bool normal = (my_c1 >= 0x1p-122f && my_c1 <= 0x1p125f) || my_c1 == 0.0f;
@@ -208,9 +224,9 @@ __global__ void __launch_bounds__(kQuantThreads, 2) nf4_quantize_kernel(const __
       const float c1 = __uint_as_float(bm[i] << 16);
       uint32_t q8;
       if (fast || (c1 >= 0x1p-122f && c1 <= 0x1p125f)) {
-        q8 = (c1 == 0.0f) ? 0x77777777u : quantize8(cells, v[i], (fast ? inv : __frcp_rn(c1)) * 16.0f);
+        q8 = (c1 == 0.0f) ? p.zero8 : quantize8(cells, v[i], (fast ? inv : __frcp_rn(c1)) * 16.0f);
       } else if (c1 == 0.0f) {
-        q8 = 0x77777777u;                        // all-zero block: the 0.0 code
+        q8 = p.zero8;                            // all-zero block: the 0.0 code
       } else {                                   // keep 16/c1 a normal number
         const float pre = (c1 < 1.0f) ? 0x1p64f : 0x1p-64f;
         q8 = quantize8_scaled(cells, v[i], __frcp_rn(c1 * pre) * 16.0f, pre);
@@ -239,10 +255,12 @@ __global__ void __launch_bounds__(kQuantThreads, 2) nf4_quantize_kernel(const __
 // ---------------------------------------------------------------- dequantize
 struct DequantArgs {
   const uint8_t* packed;
-  const uint8_t* c1q;
+  const uint8_t* c1q;   // first-level constants (bytes, or fp32 for kDqNone)
   const float* c2;
   uint16_t* out;
   int64_t numel;
+  int dq;               // DqFormat
+  int f16;              // output fp16 (else bf16)
   float code[16];
 };
 
@@ -268,8 +286,7 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(const __grid_constant_
       const int64_t u = base + i * 32 + lane;
       if (u < nunits) {
         w[i] = __ldcs(reinterpret_cast<const unsigned int*>(p.packed) + u);
-        const int64_t b = u >> 3;
-        s1[i] = e4m3_to_f32(__ldg(p.c1q + b)) * __ldg(p.c2 + (b >> 8));
+        s1[i] = block_scale(p.dq, p.c1q, p.c2, u >> 3);
       } else {
         w[i] = 0u;
         s1[i] = 0.0f;
@@ -279,39 +296,41 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(const __grid_constant_
     for (int i = 0; i < kDqUnits; ++i) {
       const int64_t u = base + i * 32 + lane;
       if (u >= nunits) break;
+      const bool h = p.f16 != 0;
       uint4 o;
-      o.x = pack_bf16x2(code_s[w[i] & 0xFu] * s1[i], code_s[(w[i] >> 4) & 0xFu] * s1[i]);
-      o.y = pack_bf16x2(code_s[(w[i] >> 8) & 0xFu] * s1[i], code_s[(w[i] >> 12) & 0xFu] * s1[i]);
-      o.z = pack_bf16x2(code_s[(w[i] >> 16) & 0xFu] * s1[i], code_s[(w[i] >> 20) & 0xFu] * s1[i]);
-      o.w = pack_bf16x2(code_s[(w[i] >> 24) & 0xFu] * s1[i], code_s[w[i] >> 28] * s1[i]);
+      o.x = pack2(h, code_s[w[i] & 0xFu] * s1[i], code_s[(w[i] >> 4) & 0xFu] * s1[i]);
+      o.y = pack2(h, code_s[(w[i] >> 8) & 0xFu] * s1[i], code_s[(w[i] >> 12) & 0xFu] * s1[i]);
+      o.z = pack2(h, code_s[(w[i] >> 16) & 0xFu] * s1[i], code_s[(w[i] >> 20) & 0xFu] * s1[i]);
+      o.w = pack2(h, code_s[(w[i] >> 24) & 0xFu] * s1[i], code_s[w[i] >> 28] * s1[i]);
       __stcs(reinterpret_cast<uint4*>(p.out) + u, o);
     }
   }
   // ragged tail: the last numel % 8 weights, one thread
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     for (int64_t e = nunits * 8; e < p.numel; ++e) {
-      const int64_t b = e / kBlock;
-      const float s = e4m3_to_f32(p.c1q[b]) * p.c2[b >> 8];
+      const float s = block_scale(p.dq, p.c1q, p.c2, e / kBlock);
       const uint32_t byte = p.packed[e >> 1];
       const uint32_t q = (e & 1) ? (byte >> 4) : (byte & 0xFu);
-      p.out[e] = uint16_t(pack_bf16x2(code_s[q] * s, 0.0f) & 0xFFFFu);
+      p.out[e] = uint16_t(pack2(p.f16 != 0, code_s[q] * s, 0.0f) & 0xFFFFu);
     }
   }
 }
 
 }  // namespace
 
-cudaError_t launch_quantize(const uint16_t* W, int64_t numel, uint8_t* packed, uint8_t* c1q, float* c2,
-                            uint32_t* status, int num_sms, cudaStream_t stream) {
+cudaError_t launch_quantize(const uint16_t* W, int64_t numel, int quant_type, int dq, uint8_t* packed, void* c1,
+                            float* c2, uint32_t* status, int num_sms, cudaStream_t stream) {
   QuantArgs a{};
   a.W = W;
   a.numel = numel;
   a.packed = packed;
-  a.c1q = c1q;
+  a.c1q = static_cast<uint8_t*>(c1);
   a.c2 = c2;
   a.status = status;
   a.ngroups = ngroups_of(numel);
-  const Codebook& cb = host_codebook();
+  a.dq = dq;
+  a.zero8 = 0x11111111u * uint32_t(zero_code(quant_type));
+  const Codebook& cb = host_codebook(quant_type);
   for (int i = 0; i < 15; ++i) a.thr[i] = cb.thr[i];
   int64_t grid = a.ngroups;
   const int64_t cap = int64_t(num_sms) * 2;
@@ -321,15 +340,17 @@ cudaError_t launch_quantize(const uint16_t* W, int64_t numel, uint8_t* packed, u
   return cudaGetLastError();
 }
 
-cudaError_t launch_dequant(const uint8_t* packed, const uint8_t* c1q, const float* c2, int64_t numel,
-                           uint16_t* out, int num_sms, cudaStream_t stream) {
+cudaError_t launch_dequant(const uint8_t* packed, const uint8_t* c1, const float* c2, int64_t numel,
+                           int quant_type, int dq, int f16, uint16_t* out, int num_sms, cudaStream_t stream) {
   DequantArgs a{};
   a.packed = packed;
-  a.c1q = c1q;
+  a.c1q = c1;
   a.c2 = c2;
   a.out = out;
   a.numel = numel;
-  const Codebook& cb = host_codebook();
+  a.dq = dq;
+  a.f16 = f16;
+  const Codebook& cb = host_codebook(quant_type);
   for (int i = 0; i < 16; ++i) a.code[i] = cb.code[i];
   const int64_t nunits = numel / 8;
   int64_t grid = (nunits / (32 * kDqUnits) + 7) / 8;   // 8 warps per CTA
@@ -350,8 +371,8 @@ cudaError_t launch_dequant(const uint8_t* packed, const uint8_t* c1q, const floa
 
 // Host check that the quantize cell table is well formed: no cell of width
 // 1/16 in x holds two thresholds.
-bool quantize_table_ok() {
-  const Codebook& cb = host_codebook();
+bool quantize_table_ok(int quant_type) {
+  const Codebook& cb = host_codebook(quant_type);
   for (int c = 0; c < kCells; ++c) {
     const float lo = float(c - 16) * 0.0625f, hi = float(c - 15) * 0.0625f;
     int n = 0;

@@ -55,13 +55,45 @@ typedef enum {
   NF4_ERR_CUDA = 6         /* a CUDA runtime call or kernel launch failed */
 } nf4_status;
 
-/* A quantized weight W [rows, cols] (device buffers, see nf4_quantize_dq). */
+/* Storage formats.  The method is NF4 codes with double quantization
+ * (quant_type NF4_QUANT_NF4, double_quant NF4_DQ_E4M3; both 0, so a
+ * zero-initialised format field selects it).  The variants are the ones the
+ * pages set it against, selected like the pages' bnb_4bit_quant_type /
+ * bnb_4bit_use_double_quant flags ([P2] §三 误区5):
+ *   NF4_QUANT_INT4  the 16 evenly spaced integers -8..7 ([P2] §2.1), divided
+ *                   by 8 so the table lies in [-1, 1] like NF4's: code i is
+ *                   (i - 8) / 8; all-zero blocks take code 8 (0.0);
+ *   NF4_DQ_NONE     no double quantization: one FP32 scale1 per block
+ *                   (32/64 = 0.5 bit per weight, [P2] §2.2);
+ *   NF4_DQ_U8       scale1 as an unsigned 8-bit linear code, scale2 =
+ *                   max scale1 of the group / 255 (FP32), code = scale1 /
+ *                   scale2 rounded to the nearest integer (ties to even),
+ *                   at most 255 (an integer reading of the 8-bit scale1 of
+ *                   [P4] §3.2). */
+#define NF4_QUANT_NF4 0
+#define NF4_QUANT_INT4 1
+#define NF4_DQ_E4M3 0
+#define NF4_DQ_NONE 1
+#define NF4_DQ_U8 2
+
+/* Compute types of the dequantized weight, the activations, the LoRA factors
+ * and the layer's outputs: BF16 (the method, [P1] §3.1) or IEEE FP16 (the
+ * pages' choice for GPUs without BF16, [P2] §三 误区4; the
+ * bnb_4bit_compute_dtype flag).  Both are passed as uint16_t bit patterns. */
+#define QLORA_BF16 0
+#define QLORA_F16 1
+
+/* A quantized weight W [rows, cols] (device buffers, see nf4_quantize). */
 typedef struct {
   const uint8_t* packed; /* ceil(rows*cols/2) bytes */
-  const uint8_t* c1q;    /* nblocks bytes */
-  const float* c2;       /* ngroups floats */
+  const uint8_t* c1q;    /* first-level constants: nblocks bytes (NF4_DQ_E4M3,
+                            NF4_DQ_U8) or nblocks fp32 values, 4*nblocks bytes,
+                            4-byte aligned (NF4_DQ_NONE) */
+  const float* c2;       /* ngroups floats (unused, may be NULL, for NF4_DQ_NONE) */
   int64_t rows;          /* N: output features */
   int64_t cols;          /* K: input features */
+  int32_t quant_type;    /* NF4_QUANT_* (0: NF4) */
+  int32_t double_quant;  /* NF4_DQ_* (0: E4M3 scale1 + FP32 scale2) */
 } nf4_weight;
 
 /* The 16 NF4 values, ascending (codes) and the 15 decision thresholds
@@ -89,11 +121,35 @@ nf4_status nf4_sizes(int64_t numel, size_t* packed_bytes, int64_t* nblocks, int6
 nf4_status nf4_quantize_dq(const uint16_t* W, int64_t rows, int64_t cols, uint8_t* packed, uint8_t* c1q,
                            float* c2, int32_t* d_status, void* stream);
 
+/* nf4_quantize_dq with a chosen storage format (NF4_QUANT_*, NF4_DQ_*):
+ * same blocks, groups, nearest-code rule (on the chosen table) and packing;
+ * c1 receives nblocks bytes, or nblocks fp32 values for NF4_DQ_NONE (then
+ * 4-byte aligned); c2 receives ngroups floats and may be NULL for
+ * NF4_DQ_NONE.  NF4_ERR_INVALID_ARG for an unknown format. */
+nf4_status nf4_quantize(const uint16_t* W, int64_t rows, int64_t cols, int32_t quant_type, int32_t double_quant,
+                        uint8_t* packed, void* c1, float* c2, int32_t* d_status, void* stream);
+
 /* Double dequantization to bf16, reverse order ([P2] §2.2):
  * scale1' = fp32(E4M3 value of c1q * c2), out = bf16(fp32(code * scale1'))
  * (one fp32 multiply each, one round-to-nearest-even to bf16).
  * out: device bf16 [rows, cols]. */
 nf4_status nf4_dequant_bf16(nf4_weight w, uint16_t* out, void* stream);
+
+/* Dequantization of any storage format into a compute type (QLORA_BF16 or
+ * QLORA_F16): scale1' = the FP32 scale1, or fp32(decoded 8-bit code *
+ * scale2); out = round(fp32(code * scale1')) to the compute type.
+ * nf4_dequant_bf16(w, out) is nf4_dequant(w, QLORA_BF16, out). */
+nf4_status nf4_dequant(nf4_weight w, int32_t dtype, uint16_t* out, void* stream);
+
+/* Merge the adapter into the frozen weight for serving ([P2] §2.5: merged
+ * weights are BF16 again and inference runs at the original speed; §三 误区3,
+ * deployment path ②):
+ *   out = round(Wd + s (A B)^T),  Wd = nf4_dequant(w, dtype),
+ * A [K, r], B [r, N], out [N, K] (device, compute type dtype).  Arithmetic:
+ * Wd as in nf4_dequant; p = sum_j A[k,j] B[j,n] accumulated in fp32 (exact
+ * products, order unspecified); out = round(fma(s, p, Wd)).  1 <= r <= 256. */
+nf4_status nf4_lora_merge(nf4_weight w, const uint16_t* A, const uint16_t* B, int32_t r, float s, int32_t dtype,
+                          uint16_t* out, void* stream);
 
 /* Device workspace bytes needed by qlora_linear_fwd / qlora_linear_bwd for
  * M tokens, W [N, K] and rank r on the current device (0 on bad sizes). */
@@ -126,6 +182,18 @@ nf4_status qlora_linear_fwd(const uint16_t* X, int64_t M, nf4_weight w, const ui
 nf4_status qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, nf4_weight w, const uint16_t* A,
                             const uint16_t* B, int32_t r, float s, const uint16_t* T, uint16_t* dX, float* dA,
                             float* dB, void* ws, size_t ws_bytes, void* stream);
+
+/* qlora_linear_fwd / qlora_linear_bwd in a chosen compute type: dtype
+ * QLORA_BF16 is exactly those calls; QLORA_F16 takes and returns fp16 in
+ * every place they take bf16 (X, A, B, Y, T, dY, dX; Wd is formed in fp16;
+ * s T and G are carried as fp16 hi/lo pairs), dA and dB stay fp32.  Any
+ * storage format of w.  Same workspace, shapes and errors. */
+nf4_status qlora_linear_fwd_ex(int32_t dtype, const uint16_t* X, int64_t M, nf4_weight w, const uint16_t* A,
+                               const uint16_t* B, int32_t r, float s, uint16_t* Y, uint16_t* T_out, void* ws,
+                               size_t ws_bytes, void* stream);
+nf4_status qlora_linear_bwd_ex(int32_t dtype, const uint16_t* dY, const uint16_t* X, int64_t M, nf4_weight w,
+                               const uint16_t* A, const uint16_t* B, int32_t r, float s, const uint16_t* T,
+                               uint16_t* dX, float* dA, float* dB, void* ws, size_t ws_bytes, void* stream);
 
 /* Size of the fixed scratch array behind qlora_linear_fwd_noalloc (4 MiB per
  * device, part of the library's device image). */
