@@ -210,8 +210,9 @@ def _pair_ms(starts, ends):
 
 
 def decode_component(device, peaks):
-    """Decode GEMV (fused dequant, r=16) on 28672x8192 and 8192x28672 at
-    M in {1,4,16}: each call timed alone, L2 flushed before it."""
+    """Decode (the forward with 1-16 tokens: the dequant-fused decode kernel,
+    r=16) on 28672x8192 and 8192x28672 at M in {1,4,16}: each call timed
+    alone with CUDA events, L2 flushed before it, median of 10."""
     from bit_nf4_quantized_12_b200 import binding
     wl = workloads.WORKLOADS["decode"]
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
@@ -261,14 +262,14 @@ def _median_ms(fn, reps, flush=None, warm=3):
 
 
 def bandwidth_component(step, peaks, rounds=50):
-    """Quantize and dequantize of the 7 LLaMA-7B-shaped weights, each call
-    timed alone with CUDA events.  The calls rotate over the 7 weights (404 MB
+    """Quantize, dequantize and LoRA merge (r=64) of the 7 LLaMA-7B-shaped
+    weights, each call timed alone with CUDA events.  The calls rotate over the 7 weights (404 MB
     of bf16 W, 101 MB of NF4 storage, 404 MB of bf16 output: well over twice
     the 126 MB L2), so every call starts with its inputs out of L2.  Median of
     `rounds` calls per weight; GB/s = algorithmic bytes / sum of medians."""
     b = step.b
     out = {}
-    for kind in ("quantize", "dequant"):
+    for kind in ("quantize", "dequant", "merge"):
         per = {i: [] for i in range(len(step.mats))}
         for it in range(3 + rounds):
             for i, d in enumerate(step.mats):
@@ -276,13 +277,17 @@ def bandwidth_component(step, peaks, rounds=50):
                 s.record()
                 if kind == "quantize":
                     b.quantize(d["W"], out=d["qw"])
-                else:
+                elif kind == "dequant":
                     b.dequant(d["qw"], out=d["Wd"])
+                else:
+                    b.lora_merge(d["qw"], d["A"], d["B"], step.wl.s, out=d["Wd"])
                 e.record()
                 per[i].append((s, e))
             torch.cuda.synchronize()
         med = [statistics.median([s.elapsed_time(e) for s, e in per[i][3:]]) for i in per]
         nbytes = sum(quant_bytes(d["N"], d["K"]) for d in step.mats)
+        if kind == "merge":   # plus the LoRA factors, read once
+            nbytes += sum(2 * step.wl.r * (d["N"] + d["K"]) for d in step.mats)
         gbs = nbytes / (sum(med) * 1e-3) / 1e9
         out[kind] = {"GB/s": gbs, "frac": gbs / peaks["hbm_gbs"], "us_per_weight_set": sum(med) * 1e3,
                      "timing": f"median of {rounds} calls per weight, calls rotating over the 7 weights "
@@ -396,7 +401,7 @@ def robust_component(device, peaks, reps=5):
     bb = _median_ms(lambda: binding.linear_bwd(io["dY"], io["X"], qw, io["A"], io["B"], s_, T=T, ws=ws), reps,
                     flush, 1)
     plan = binding.plan(M, N, K, r)
-    path = {binding.PATH_FUSED: "fused tensor-core", binding.PATH_GEMV: "gemv",
+    path = {binding.PATH_FUSED: "fused tensor-core", binding.PATH_DECODE: "decode",
             binding.PATH_GENERIC: "generic CUDA-core"}[plan["path"]]
     qb = quant_bytes(N, K)
     ft = fwd_flops(M, N, K, r) / (f * 1e-3) / 1e12
@@ -513,7 +518,9 @@ def config_dict(wl, n):
 
 def kernel_case(case, n):
     """n launches of one call on the 7B q matrix (4096x4096, 2048 tokens, r=64),
-    or on the 28672x8192 decode weight at M=16 ("decode") or M=1 ("gemv");
+    or on the 28672x8192 decode weight at M=16 ("decode") or M=1 ("gemv": the
+    same decode kernel with one token); "merge" merges the r=64 adapter into
+    the 4096x4096 weight;
     quantize and dequant run on the 28672x8192 weight, whose 470 MB of bf16
     exceed the L2: a small case for ncu."""
     from bit_nf4_quantized_12_b200 import binding
@@ -536,6 +543,8 @@ def kernel_case(case, n):
             binding.quantize(W, out=qw)
         elif case == "dequant":
             binding.dequant(qw, out=Wd)
+        elif case == "merge":
+            binding.lora_merge(qw, io["A"], io["B"], s, out=Wd)
         elif case in ("fwd", "decode", "gemv"):
             binding.linear_fwd(io["X"], qw, io["A"], io["B"], s, ws=ws, Y=Y, T=T)
         else:
@@ -551,7 +560,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-components", action="store_true")
-    ap.add_argument("--kernel-case", default=None, choices=["quantize", "dequant", "fwd", "bwd", "decode", "gemv"],
+    ap.add_argument("--kernel-case", default=None, choices=["quantize", "dequant", "fwd", "bwd", "decode", "gemv", "merge"],
                     help="run a few launches of one call on one 7B-shaped matrix (for ncu), print nothing")
     args = ap.parse_args()
 
@@ -666,6 +675,7 @@ def main():
         comp["dequant"].update({"step_GB/s": comp["dequant"].pop("GB/s"), "step_frac": comp["dequant"].pop("frac")})
         comp["quantize"].update(bw["quantize"])
         comp["dequant"].update(bw["dequant"])
+        comp["merge"] = bw["merge"]
         del step
         torch.cuda.empty_cache()
         comp["decode"] = decode_component(device, peaks)

@@ -43,7 +43,7 @@ class QloraPlan(ctypes.Structure):
                 ("main_steps", ctypes.c_int64), ("lowrank_splits", ctypes.c_int32 * 4)]
 
 
-PATH_FUSED, PATH_GEMV, PATH_GENERIC = 0, 1, 2
+PATH_FUSED, PATH_DECODE, PATH_GENERIC = 0, 1, 2
 
 # (name, restype, argtypes) for every symbol of include/qlora_nf4.h
 _P, _I64, _I32, _F, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t

@@ -30,13 +30,14 @@ int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 bool needs_generic(int64_t N, int64_t K, int r) { return K % 64 != 0 || N % 8 != 0 || r % 8 != 0; }
 
 // Workspace, fused path:   [status word (256 B) | low-rank hi/lo pair [M, 2rp] bf16 | T scratch [M, r] bf16]
+//   plus, for 1-16 tokens (decode kernel): [fp32 partials of split tiles | tile counters]
 // Workspace, generic path: [status word (256 B) | Wd [N, K] bf16 | T scratch [M, r] bf16 | G [M, r] fp32]
 struct WsLayout {
-  size_t hilo = 0, wd = 0, t_scratch = 0, g = 0, total = 0;
+  size_t hilo = 0, wd = 0, t_scratch = 0, g = 0, partial = 0, counters = 0, counters_bytes = 0, total = 0;
 };
 constexpr size_t kHeaderBytes = 256;
 
-WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int r, int /*sms*/) {
+WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int r, int sms) {
   WsLayout L;
   size_t off = kHeaderBytes;
   if (needs_generic(N, K, r)) {
@@ -54,6 +55,14 @@ WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int r, int /*sms*/) {
   off += size_t(round_up(M * 2 * rp * 2, 256));
   L.t_scratch = off;
   off += size_t(round_up(M * r * 2, 256));
+  if (decode_supported(M, K)) {
+    const DecodePlan d = plan_decode(M, N, K, sms);
+    L.partial = off;
+    off += size_t(round_up(d.partial_floats * 4, 256));
+    L.counters = off;
+    L.counters_bytes = size_t(d.tiles) * 4;
+    off += size_t(round_up(d.tiles * 4, 256));
+  }
   L.total = off;
   return L;
 }
@@ -82,7 +91,7 @@ nf4_status check_sizes(int64_t M, int64_t N, int64_t K, int32_t r) {
   if (N > (int64_t(1) << 31) || K > (int64_t(1) << 31) || M > (int64_t(1) << 31)) return NF4_ERR_UNSUPPORTED;
   if (needs_generic(N, K, r)) {
     if (N > (int64_t(1) << 40) / K) return NF4_ERR_UNSUPPORTED;
-  } else if (M > kMaxFusedTokens && !gemv_supported(M, K)) {
+  } else if (M > kMaxFusedTokens && !decode_supported(M, K)) {
     return NF4_ERR_UNSUPPORTED;
   }
   return NF4_OK;
@@ -234,21 +243,27 @@ nf4_status qlora_linear_fwd_ex(int32_t dtype, const uint16_t* X, int64_t M, nf4_
   sa.status = status;
   sa.pdl_mode = kPdlWaitFirst;
   sa.f16 = f16;
-  if (launch_skinny(plan_skinny(kSkinnyT, M, N, K, r, sms), sa, strm, false) != cudaSuccess) return NF4_ERR_CUDA;
 
-  if (gemv_supported(M, K)) {
-    // one token: a matrix-vector product bound by reading the packed weight,
-    // on CUDA cores; it overlaps T and waits for it only before the low-rank
-    // term
-    Nf4GemvArgs va{};
-    va.M = M; va.N = N; va.K = K; va.r = r; va.s = s;
-    va.X = X; va.packed = w.packed; va.c1q = w.c1q; va.c2 = w.c2;
-    va.T = t_dst; va.B = B; va.Y = Y; va.status = status;
-    va.dq = w.double_quant; va.f16 = f16;
-    if (launch_nf4_gemv(va, host_codebook(w.quant_type).code, sms, strm, true) != cudaSuccess) return NF4_ERR_CUDA;
+  if (decode_supported(M, K)) {
+    // 1-16 tokens: bound by reading the packed weight; each weight is
+    // decoded once and multiplied with every token on mma.sync.  It overlaps
+    // T and waits for it only before the low-rank term.
+    const DecodePlan dp = plan_decode(M, N, K, sms);
+    int* counters = reinterpret_cast<int*>(wsb + L.counters);
+    if (cudaMemsetAsync(counters, 0, L.counters_bytes, strm) != cudaSuccess) return NF4_ERR_CUDA;
+    Nf4DecodeArgs da{};
+    da.M = M; da.N = N; da.K = K; da.r = r; da.s = s;
+    da.X = X; da.packed = w.packed; da.c1q = w.c1q; da.c2 = w.c2;
+    da.T = t_dst; da.B = B; da.Y = Y; da.status = status;
+    da.dq = w.double_quant; da.f16 = f16;
+    da.partial = reinterpret_cast<float*>(wsb + L.partial);
+    da.counters = counters;
+    if (launch_skinny(plan_skinny(kSkinnyT, M, N, K, r, sms), sa, strm, false) != cudaSuccess) return NF4_ERR_CUDA;
+    if (launch_nf4_decode(dp, da, host_codebook(w.quant_type).code, strm, true) != cudaSuccess) return NF4_ERR_CUDA;
     return NF4_OK;
   }
 
+  if (launch_skinny(plan_skinny(kSkinnyT, M, N, K, r, sms), sa, strm, false) != cudaSuccess) return NF4_ERR_CUDA;
   // The fused GEMM may start while T is still being computed: its main
   // product does not need T, and it waits for T before the low-rank steps.
   Nf4GemmArgs ga{};
@@ -392,8 +407,14 @@ nf4_status qlora_linear_plan(int64_t M, int64_t N, int64_t K, int32_t r, int32_t
   memset(&p, 0, sizeof(p));
   if (needs_generic(N, K, r)) {
     p.path = QLORA_PATH_GENERIC;
-  } else if (!backward && gemv_supported(M, K)) {
-    p.path = QLORA_PATH_GEMV;
+  } else if (!backward && decode_supported(M, K)) {
+    const DecodePlan d = plan_decode(M, N, K, sms);
+    p.path = QLORA_PATH_DECODE;
+    p.token_tile = 16;
+    p.splits = int32_t(d.ctas);
+    p.tiles_w = d.tiles;
+    p.tiles_t = 1;
+    p.main_steps = d.nk;
     p.lowrank_splits[kSkinnyT] = plan_skinny(kSkinnyT, M, N, K, r, sms).splits;
   } else {
     const Nf4GemmPlan g = plan_nf4_gemm(backward ? 1 : 0, M, N, K, r, sms);

@@ -117,29 +117,36 @@ struct SkinnyArgs {
 };
 cudaError_t launch_skinny(const SkinnyPlan& plan, const SkinnyArgs& a, cudaStream_t stream, bool pdl);
 
-// ---------------------------------------------------------------- decode GEMV
-// Forward of the linear layer for one token on CUDA cores:
-//   y[n] = bf16(sum_k x[k] Wd[n,k] + s sum_j T[j] B[j,n]),
-// with T = bf16(x A) produced by the previous kernel of the stream (the
-// kernel waits for it only before the low-rank term).
-struct Nf4GemvArgs {
+// ---------------------------------------------------------------- decode (1-16 tokens)
+// Forward of the linear layer for M <= 16 tokens: every weight decoded once
+// in registers and multiplied with all tokens on mma.sync; persistent CTAs
+// over (256-row tile, 256-column chunk) units, split tiles summed in a fixed
+// order by the CTA that finishes last.
+struct Nf4DecodeArgs {
   int64_t M, N, K;
   int r;
   float s;
-  const uint16_t* X;         // [M, K] bf16
+  const uint16_t* X;         // [M, K]
   const uint8_t* packed;
-  const uint8_t* c1q;
+  const uint8_t* c1q;        // first-level constants (bytes, or fp32 for kDqNone)
   const float* c2;
-  const uint16_t* T;         // [M, r] bf16
-  const uint16_t* B;         // [r, N] bf16
-  uint16_t* Y;               // [M, N] bf16
+  const uint16_t* T;         // [M, r] from the previous kernel of the stream
+  const uint16_t* B;         // [r, N]
+  uint16_t* Y;               // [M, N]
   uint32_t* status;          // kStatusTimeout on a failed wait
-  int dq;                    // DqFormat of the first-level constants
-  int f16;                   // compute type fp16 (else bf16) for X, T, B, Y
+  int dq;                    // DqFormat
+  int f16;                   // compute type fp16 (else bf16)
+  float* partial;            // workspace: plan.partial_floats fp32
+  int* counters;             // workspace: plan.tiles int32, zero before the launch
 };
-// Whether the GEMV takes this problem (one token, K within its shared memory).
-bool gemv_supported(int64_t M, int64_t K);
-cudaError_t launch_nf4_gemv(const Nf4GemvArgs& a, const float code[16], int num_sms, cudaStream_t stream, bool pdl);
+struct DecodePlan {
+  int64_t tiles, nk, units, ctas;
+  int64_t partial_floats;
+};
+bool decode_supported(int64_t M, int64_t K);
+DecodePlan plan_decode(int64_t M, int64_t N, int64_t K, int num_sms);
+cudaError_t launch_nf4_decode(const DecodePlan& plan, const Nf4DecodeArgs& a, const float code[16],
+                              cudaStream_t stream, bool pdl);
 
 // ---------------------------------------------------------------- generic GEMM
 // C[i, j] = sum over segments of scale * sum_p a(i, p) b(j, p), on CUDA cores,

@@ -25,7 +25,7 @@
 // Both kernels are HBM-bandwidth bound: 16-byte coalesced loads and stores,
 // the per-block absmax by warp shuffles across the 8 lanes that own a block,
 // and the code decision as one lookup in a 33-cell shared-memory table plus
-// one compare.
+// one compare (about 8 instructions per weight, most on the FMA pipe).
 #include <cstdint>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -61,33 +61,49 @@ __device__ __forceinline__ void build_cells(uint2* cells, const float* thr_smem)
   }
 }
 
+// Code decision for any x16, non-finite included: NaN or |x| > 1 (only with
+// non-finite input) clamps into an end cell.
 __device__ __forceinline__ uint32_t classify16(const uint2* cells, float x16) {
-  // NaN or |x| > 1 (only with non-finite input) clamps into an end cell
   const uint32_t idx = min(uint32_t(__float2int_rd(x16) + 16), uint32_t(kCells - 1));
   const uint2 e = cells[idx];
   return e.y + (x16 > __uint_as_float(e.x) ? 1u : 0u);
 }
 
-// 8 consecutive bf16 (one uint4) -> 8 nibbles (element 0 in bits 0-3);
-// inv16 = 16 / scale1.
-__device__ __forceinline__ uint32_t quantize8(const uint2* cells, const uint4& v, float inv16) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  uint32_t out = 0;
-#pragma unroll
-  for (int j = 3; j >= 0; --j) {
-    out = (out << 4) | classify16(cells, bf16hi_to_f32(w[j]) * inv16);
-    out = (out << 4) | classify16(cells, bf16lo_to_f32(w[j]) * inv16);
-  }
-  return out;
+// Code decision for finite x16 in [-16, 16] (a block with a normal absmax:
+// |w * fp32(1/absmax)| <= 1 holds after rounding).  r = RD(x16 + 2^23 + 16)
+// is the integer 2^23 + 16 + floor(x16), so the low bits of its pattern are
+// the cell index 0..32: one round-down add on the FMA pipe instead of a
+// float-to-int conversion.  cells_biased is the cell table's shared address
+// minus 8 * 0x4B000000 (mod 2^32), so the pattern times 8 addresses the cell
+// directly.  The comparison x16 > 16 T is the sign bit of 16 T - x16, which is
+// +0 for x16 == 16 T (ties go to the lower code) and +inf where the cell holds
+// no threshold.
+__device__ __forceinline__ uint32_t classify_fast(uint32_t cells_biased, float x16) {
+  const float r = __fadd_rd(x16, 8388624.0f);
+  const uint32_t addr = cells_biased + (__float_as_uint(r) << 3);
+  uint32_t t, base;
+  asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(t), "=r"(base) : "r"(addr));
+  return base + (__float_as_uint(__uint_as_float(t) - x16) >> 31);
 }
-// Same with the weights first scaled by a power of two (extreme blocks).
-__device__ __forceinline__ uint32_t quantize8_scaled(const uint2* cells, const uint4& v, float inv16, float pre) {
+
+// 8 consecutive bf16 (one uint4) -> 8 nibbles (element 0 in bits 0-3);
+// inv16 = 16 / scale1 (of the weights first scaled by pre, a power of two,
+// on the careful path for extreme or non-finite blocks).
+template <bool FAST>
+__device__ __forceinline__ uint32_t quantize8(const uint2* cells, uint32_t cells_biased, const uint4& v,
+                                              float inv16, float pre) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   uint32_t out = 0;
 #pragma unroll
   for (int j = 3; j >= 0; --j) {
-    out = (out << 4) | classify16(cells, (bf16hi_to_f32(w[j]) * pre) * inv16);
-    out = (out << 4) | classify16(cells, (bf16lo_to_f32(w[j]) * pre) * inv16);
+    float hi = bf16hi_to_f32(w[j]), lo = bf16lo_to_f32(w[j]);
+    if (!FAST) {
+      hi *= pre;
+      lo *= pre;
+    }
+    const float xh = hi * inv16, xl = lo * inv16;
+    out = out * 16u + (FAST ? classify_fast(cells_biased, xh) : classify16(cells, xh));
+    out = out * 16u + (FAST ? classify_fast(cells_biased, xl) : classify16(cells, xl));
   }
   return out;
 }
@@ -148,6 +164,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) nf4_quantize_kernel(const __
   __syncthreads();
   build_cells(cells, thr_s);
   __syncthreads();
+  const uint32_t cells_biased = smem_u32(cells) - (0x4B000000u << 3);
 
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
@@ -180,42 +197,19 @@ __global__ void __launch_bounds__(kQuantThreads, 2) nf4_quantize_kernel(const __
     uint4 vn[kQuantIters];
     if (gn < p.ngroups) load_group(p, gn, vn);
 
-    __syncthreads();
-    gm = warp_max[parity][0];
-#pragma unroll
-    for (int w = 1; w < kQuantThreads / 32; ++w) gm = max(gm, warp_max[parity][w]);
-    if (gm >= 0x7F80u) bad = 1;
-
-    // second level: fp32 scale2 for the group, E4M3 codes of scale1/scale2.
-    // Lane j < kQuantIters of each 8-lane block group owns pass j: it
-    // computes that block's code and reciprocal once; the others receive the
-    // reciprocal by shuffle.
-    const float gmax = __uint_as_float(gm << 16);
-    const float s2 = __fdiv_rn(gmax, p.dq == kDqU8 ? 255.0f : 448.0f);
-    if (tid == 0 && p.dq != kDqNone) p.c2[g] = s2;
+    // 4-bit codes first: a code depends only on its own block's absmax, so
+    // this work needs no other warp and comes before the group barrier.
+    // Lane j < kQuantIters of each 8-lane block group owns pass j: it takes
+    // that block's reciprocal once; the others receive it by shuffle.
     const int j = lane & 7;
     uint32_t my_bm = bm[0];
 #pragma unroll
     for (int i = 1; i < kQuantIters; ++i) my_bm = (j == i) ? bm[i] : my_bm;
     const float my_c1 = __uint_as_float(my_bm << 16);
-    if (j < kQuantIters) {
-      const int64_t b = g * kGroup + int64_t(j) * (kQuantThreads / 8) + (tid >> 3);
-      if (b < nblk_total) {
-        if (p.dq == kDqNone) {
-          reinterpret_cast<float*>(p.c1q)[b] = my_c1;
-        } else if (my_c1 == 0.0f) {
-          p.c1q[b] = 0;
-        } else {
-          const float t = __fdiv_rn(my_c1, s2);
-          p.c1q[b] = uint8_t(p.dq == kDqU8 ? min(__float2uint_rn(t), 255u) : f32_to_e4m3_satfinite(t));
-        }
-      }
-    }
     // 16 / scale1 must stay a finite normal number: scale1 in [2^-122, 2^125]
     const bool normal = (my_c1 >= 0x1p-122f && my_c1 <= 0x1p125f) || my_c1 == 0.0f;
     const float my_inv = (my_c1 == 0.0f) ? 0.0f : (normal ? __frcp_rn(my_c1) : 0.0f);
     const bool fast = __all_sync(0xffffffffu, normal);
-    // 4-bit codes
 #pragma unroll
     for (int i = 0; i < kQuantIters; ++i) {
       const int64_t e0 = gbase + int64_t(i) * (kQuantThreads * 8) + tid * 8;
@@ -223,13 +217,15 @@ __global__ void __launch_bounds__(kQuantThreads, 2) nf4_quantize_kernel(const __
       if (e0 >= p.numel) continue;
       const float c1 = __uint_as_float(bm[i] << 16);
       uint32_t q8;
-      if (fast || (c1 >= 0x1p-122f && c1 <= 0x1p125f)) {
-        q8 = (c1 == 0.0f) ? p.zero8 : quantize8(cells, v[i], (fast ? inv : __frcp_rn(c1)) * 16.0f);
-      } else if (c1 == 0.0f) {
+      if (c1 == 0.0f) {
         q8 = p.zero8;                            // all-zero block: the 0.0 code
+      } else if (fast) {
+        q8 = quantize8<true>(cells, cells_biased, v[i], inv * 16.0f, 1.0f);
+      } else if (c1 >= 0x1p-122f && c1 <= 0x1p125f) {
+        q8 = quantize8<false>(cells, cells_biased, v[i], __frcp_rn(c1) * 16.0f, 1.0f);
       } else {                                   // keep 16/c1 a normal number
         const float pre = (c1 < 1.0f) ? 0x1p64f : 0x1p-64f;
-        q8 = quantize8_scaled(cells, v[i], __frcp_rn(c1 * pre) * 16.0f, pre);
+        q8 = quantize8<false>(cells, cells_biased, v[i], __frcp_rn(c1 * pre) * 16.0f, pre);
       }
       uint8_t* dst = p.packed + (e0 >> 1);
       if (e0 + 8 <= p.numel) {
@@ -243,6 +239,31 @@ __global__ void __launch_bounds__(kQuantThreads, 2) nf4_quantize_kernel(const __
             if (2 * jj + 1 >= valid) byte &= 0x0Fu;   // pad nibble of an odd tail
             dst[jj] = uint8_t(byte);
           }
+        }
+      }
+    }
+
+    // second level: fp32 scale2 for the group (needs every warp's maximum),
+    // then the 8-bit codes of scale1 / scale2 (lane j < kQuantIters of each
+    // block group stores its block's)
+    __syncthreads();
+    gm = warp_max[parity][0];
+#pragma unroll
+    for (int w = 1; w < kQuantThreads / 32; ++w) gm = max(gm, warp_max[parity][w]);
+    if (gm >= 0x7F80u) bad = 1;
+    const float gmax = __uint_as_float(gm << 16);
+    const float s2 = __fdiv_rn(gmax, p.dq == kDqU8 ? 255.0f : 448.0f);
+    if (tid == 0 && p.dq != kDqNone) p.c2[g] = s2;
+    if (j < kQuantIters) {
+      const int64_t b = g * kGroup + int64_t(j) * (kQuantThreads / 8) + (tid >> 3);
+      if (b < nblk_total) {
+        if (p.dq == kDqNone) {
+          reinterpret_cast<float*>(p.c1q)[b] = my_c1;
+        } else if (my_c1 == 0.0f) {
+          p.c1q[b] = 0;
+        } else {
+          const float t = __fdiv_rn(my_c1, s2);
+          p.c1q[b] = uint8_t(p.dq == kDqU8 ? min(__float2uint_rn(t), 255u) : f32_to_e4m3_satfinite(t));
         }
       }
     }

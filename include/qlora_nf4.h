@@ -164,7 +164,8 @@ size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t r);
  * M, N, K <= 2^31, and M <= 65535 * 256 on the fused path below
  * (NF4_ERR_UNSUPPORTED otherwise, before anything is launched).
  * When K % 64 == 0, N % 8 == 0 and r % 8 == 0, Wd is formed on chip inside
- * the tensor-core product and never written to memory.  Other shapes (rows of
+ * the tensor-core product and never written to memory (1-16 tokens: the
+ * decode kernel; more: the fused tensor-core GEMM).  Other shapes (rows of
  * W that do not start on an NF4 block, a row count or rank off the 8-element
  * granule) take a CUDA-core path that first dequantizes W into the workspace
  * (which then holds N * K bf16 more; N * K <= 2^40) and accumulates in fp32:
@@ -244,23 +245,29 @@ nf4_status qlora_linear_fwd_noalloc_info(int32_t** d_status_word, size_t* scratc
  * nothing and touches no device memory.  The pages have no counterpart; it
  * exists so that callers and tests can see which kernels a shape runs.
  *   path        QLORA_PATH_FUSED: tensor-core GEMM with W dequantized on chip;
- *               QLORA_PATH_GEMV: one-token forward on CUDA cores;
+ *               QLORA_PATH_DECODE: forward with 1-16 tokens, each weight
+ *               decoded once in registers and multiplied with every token
+ *               (mma.sync), persistent CTAs over (tile, column chunk) units;
  *               QLORA_PATH_GENERIC: W dequantized into the workspace, then
  *               CUDA-core products (shapes off the fused kernels' granules).
- *   token_tile  fused: tokens per output tile (32, 64, 128 or 256).
+ *   token_tile  fused: tokens per output tile (32, 64, 128 or 256); decode: 16.
  *   splits      fused: CTAs that share one output tile's reduction (1, 2, 4
  *               or 8, one thread-block cluster); every split gets >= 1 step.
- *   tiles_w     fused: 128-row tiles of the W dimension (N forward, K backward).
- *   tiles_t     fused: token tiles.
- *   main_steps  fused: 64-wide steps of the main reduction (K forward, N backward).
+ *               decode: persistent CTAs (min(units, SMs)).
+ *   tiles_w     fused: 128-row tiles of the W dimension (N forward, K backward);
+ *               decode: 256-row tiles of W.
+ *   tiles_t     fused: token tiles; decode: 1.
+ *   main_steps  fused: 64-wide steps of the main reduction (K forward, N
+ *               backward); decode: 256-column chunks of K (units = tiles_w
+ *               * main_steps).
  *   lora_steps  fused: 64-wide steps of the low-rank term (hi and lo halves).
  *   lowrank_splits[4]  splits of the low-rank products T = X A, G = s dY B^T,
- *               dA = X^T G, dB = s T^T dY (fused and GEMV paths; 0 where the
+ *               dA = X^T G, dB = s T^T dY (fused and decode paths; 0 where the
  *               call does not run that product).
  * Returns NF4_ERR_INVALID_ARG / NF4_ERR_UNSUPPORTED for the sizes that
  * qlora_linear_fwd / qlora_linear_bwd reject with those codes. */
 #define QLORA_PATH_FUSED 0
-#define QLORA_PATH_GEMV 1
+#define QLORA_PATH_DECODE 1
 #define QLORA_PATH_GENERIC 2
 typedef struct {
   int32_t path;

@@ -67,7 +67,7 @@ def test_host_validation_before_launch():
     assert L.qlora_linear_fwd(fake, 16, w_rag, fake, fake, 16, 1.0, fake, None, fake, need - 1, None) == 4
     assert L.qlora_workspace_bytes(16, 64, 128, 12) >= 256 + 64 * 128 * 2          # r % 8 != 0
     assert L.qlora_workspace_bytes(16, 60, 128, 16) >= 256 + 60 * 128 * 2          # N % 8 != 0
-    assert L.qlora_workspace_bytes(16, 64, 128, 16) < 64 * 128 * 2                 # fused: no Wd copy
+    assert L.qlora_workspace_bytes(32, 64, 128, 16) < 64 * 128 * 2                 # fused: no Wd copy
     assert L.qlora_linear_fwd(fake, 16, w, fake, fake, 12, 1.0, fake, None, fake, 16, None) == 4
     assert L.qlora_workspace_bytes(16, 1 << 31, 1 << 31, 12) == 0                  # Wd copy too large
     assert L.qlora_linear_fwd(fake, 16, w, fake, fake, 16, 1.0, fake, None, fake, 16, None) == 4

@@ -6,7 +6,8 @@ dX, dA, dB and the workspace, sized exactly as the C ABI states -- sits
 between two 4 KB guard regions filled with a pattern.  After the calls the
 guards must be intact.  The shapes reach every kernel: quantize/dequant with
 ragged tails, the fused GEMM with and without a split reduction and with
-ragged tiles, the one-token GEMV, and the generic path for ragged shapes.
+ragged tiles, the decode kernel (1-16 tokens, whole and split tiles), and
+the generic path for ragged shapes.
 """
 import pytest
 import torch
@@ -58,7 +59,9 @@ def test_quantize_and_dequant_stay_in_bounds(shape):
 @pytest.mark.parametrize("M,N,K,r", [(32, 1024, 1024, 16),     # fused, no split
                                      (2, 8, 4096, 8),          # one W tile, 8-way split
                                      (257, 384, 1024, 24),     # ragged token and W tiles
-                                     (1, 1024, 1024, 16),      # one-token GEMV (forward)
+                                     (1, 1024, 1024, 16),      # decode kernel (forward), split tiles
+                                     (16, 4104, 4096, 64),     # decode: ragged last 256-row tile
+                                     (9, 512, 1088, 8),        # decode: ragged last column chunk
                                      (5, 24, 100, 8),          # generic path: K % 64 != 0
                                      (17, 13, 64, 12)])        # generic path: N % 8, r % 8
 def test_linear_layer_stays_in_bounds(M, N, K, r):

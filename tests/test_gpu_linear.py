@@ -132,18 +132,39 @@ def test_tile_and_split_edges(M, N, K, r):
     _run(M, N, K, r, 0.75, seed=M * 7 + N)
 
 
-@pytest.mark.parametrize("N,K,r", [(104, 2112, 8), (4104, 64, 16), (8, 64, 8), (520, 4096, 64), (2056, 640, 256)])
-def test_one_token_gemv_edges(N, K, r):
-    """One token takes the CUDA-core GEMV: a last pass with fewer than 32
-    blocks (K = 2112 is 33 blocks), a single block per row, a row count that
-    leaves warps with fewer rows than the ring holds, and the largest rank."""
-    _run(1, N, K, r, 0.5, seed=N + K)
+@pytest.mark.parametrize("M,N,K,r", [(1, 104, 2112, 8), (1, 4104, 64, 16), (1, 8, 64, 8), (1, 520, 4096, 64),
+                                     (1, 2056, 640, 256), (2, 256, 512, 16), (3, 1024, 1024, 72), (7, 264, 320, 8),
+                                     (8, 1024, 1024, 16), (9, 1032, 2112, 24), (12, 776, 768, 32),
+                                     (16, 4096, 4096, 64), (16, 8, 256, 8), (5, 20480, 192, 16)])
+def test_decode_kernel_edges(M, N, K, r):
+    """1-16 tokens take the decode kernel: a last 256-row tile of 8 rows
+    (N = 4104), a last column chunk of one NF4 block (K = 2112, 33 blocks),
+    a single block per row, tiles split between CTAs (stream-K) and whole,
+    one and two 8-token MMA tiles, the largest rank."""
+    _run(M, N, K, r, 0.5, seed=N + K + M)
+
+
+def test_decode_is_deterministic():
+    """Split tiles are summed in a fixed order: two calls give the same bits."""
+    M, N, K, r = 16, 28672, 8192, 16
+    W, io = _problem(M, N, K, r, seed=13)
+    qw, _ = gpu_quantize(W)
+    ws = binding.workspace(M, N, K, r, DEV)
+    assert binding.plan(M, N, K, r)["path"] == binding.PATH_DECODE
+    outs = []
+    for _ in range(3):
+        Y, T = binding.linear_fwd(io["X"], qw, io["A"], io["B"], 1.0, ws=ws)
+        outs.append(Y.clone())
+    torch.cuda.synchronize()
+    assert binding.workspace_status(ws) == 0
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
 
 
 @pytest.mark.parametrize("M", [1, 4, 16])
 @pytest.mark.parametrize("shape", [(28672, 8192), (8192, 28672)])
 def test_decode_shapes_sampled_columns(M, shape):
-    """Decode: full-size weight, every token, 64 sampled output features."""
+    """Decode: full-size weight, every token, 64 sampled output features
+    (the decode kernel: stream-K over 3584 units on all SMs)."""
     wl = workloads.WORKLOADS["decode"]
     N, K = shape
     W = workloads.weight(N, K, wl.w_std, seed=0, device=DEV)

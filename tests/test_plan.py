@@ -4,7 +4,8 @@ qlora_linear_plan reports the path, tiles and reduction splits the library
 picks for a call.  These tests sweep shapes and SM counts and check what the
 kernels rely on:
   - the path: generic exactly when K % 64, N % 8 or r % 8 is nonzero; the
-    one-token GEMV only for a forward with M = 1;
+    decode kernel exactly for a forward with 1 to 16 tokens; its persistent
+    CTAs take every (tile, column chunk) unit once;
   - the tile grid covers the output exactly once and fits the launch limits;
   - a split reduction is used only when the tiles leave SMs idle, fits one
     cluster (<= 8 CTAs) and gives every CTA at least one step of the
@@ -43,10 +44,17 @@ def check_plan(M, N, K, r, backward, sms):
         assert p["path"] == binding.PATH_GENERIC
         assert p["lowrank_splits"] == [0, 0, 0, 0]
         return p
-    if not backward and M == 1 and K <= 32768:     # x fits the GEMV's shared memory
-        assert p["path"] == binding.PATH_GEMV
-    if p["path"] == binding.PATH_GEMV:
-        assert not backward and M == 1
+    if not backward and M <= 16:
+        assert p["path"] == binding.PATH_DECODE
+    if p["path"] == binding.PATH_DECODE:
+        assert not backward and M <= 16
+        assert p["tiles_w"] == cdiv(N, 256) and p["main_steps"] == cdiv(K, 256) and p["tiles_t"] == 1
+        units = p["tiles_w"] * p["main_steps"]
+        ctas = p["splits"]
+        assert 1 <= ctas <= min(units, sms)
+        # the stream-K ranges [p U / P, (p+1) U / P) tile the units, none empty
+        begins = [q * units // ctas for q in range(ctas + 1)]
+        assert begins[0] == 0 and begins[-1] == units and all(b1 > b0 for b0, b1 in zip(begins, begins[1:]))
     else:
         assert p["path"] == binding.PATH_FUSED
         bt = p["token_tile"]
@@ -103,7 +111,7 @@ def test_every_split_count_is_exercised():
 
 
 @pytest.mark.parametrize("M,N,K,r", [(5, 24, 100, 8), (33, 40, 1000, 12), (17, 13, 64, 8), (1, 96, 130, 4),
-                                     (4096, 4095, 11007, 8), (1, 4096, 4096, 12)])
+                                     (4096, 4095, 11007, 8), (1, 4096, 4096, 12), (4, 4095, 4096, 8)])
 def test_ragged_shapes_take_the_generic_path(M, N, K, r):
     for backward in (0, 1):
         assert check_plan(M, N, K, r, backward, 148)["path"] == binding.PATH_GENERIC

@@ -32,7 +32,7 @@ def test_noalloc_matches_workspace_entry_point_two_calls():
     _, scratch_bytes = binding.noalloc_info()
     # the second call has a different shape and rank, so a stale status word
     # or stale scratch from the first would show
-    # (the last two take the one-token GEMV and the generic path for a ragged K)
+    # (the last two take the decode kernel and the generic path for a ragged K)
     cases = [(300, 384, 1024, 64, 0.25, 3), (37, 520, 640, 8, 4.0, 5), (1, 1024, 1024, 16, 1.0, 11),
              (5, 24, 100, 8, 2.0, 9)]
     for M, N, K, r, s, seed in cases:
