@@ -24,16 +24,22 @@ int device_sms() {
 
 int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 
-// Shapes outside the fused tensor-core kernels (W rows not starting on an
-// NF4 block, a W row count or rank off the 8-element store granule) take the
-// generic CUDA-core path of generic.cu.
-bool needs_generic(int64_t N, int64_t K, int r) { return K % 64 != 0 || N % 8 != 0 || r % 8 != 0; }
+// A rank off the 8-element granule (the low-rank operands' 16-byte rows)
+// takes the generic CUDA-core path of generic.cu.  Every other shape runs on
+// the tensor cores: K % 64 != 0 (W rows not starting on an NF4 block) in the
+// fused GEMM's ragged mode, and K or N off the 8-element granule with X, dY
+// and B re-pitched into the workspace (16-byte row pitches for TMA).
+bool needs_generic(int64_t /*N*/, int64_t /*K*/, int r) { return r % 8 != 0; }
+int64_t pitch8(int64_t n) { return (n + 7) / 8 * 8; }
 
 // Workspace, fused path:   [status word (256 B) | low-rank hi/lo pair [M, 2rp] bf16 | T scratch [M, r] bf16]
 //   plus, for 1-16 tokens (decode kernel): [fp32 partials of split tiles | tile counters]
 // Workspace, generic path: [status word (256 B) | Wd [N, K] bf16 | T scratch [M, r] bf16 | G [M, r] fp32]
+//   plus, when K % 8 != 0: X re-pitched [M, pitch8(K)]; when N % 8 != 0: dY
+//   re-pitched [M, pitch8(N)] and B re-pitched [r, pitch8(N)]
 struct WsLayout {
-  size_t hilo = 0, wd = 0, t_scratch = 0, g = 0, partial = 0, counters = 0, counters_bytes = 0, total = 0;
+  size_t hilo = 0, wd = 0, t_scratch = 0, g = 0, partial = 0, counters = 0, counters_bytes = 0;
+  size_t xp = 0, dyp = 0, bp = 0, total = 0;
 };
 constexpr size_t kHeaderBytes = 256;
 
@@ -62,6 +68,16 @@ WsLayout ws_layout(int64_t M, int64_t N, int64_t K, int r, int sms) {
     L.counters = off;
     L.counters_bytes = size_t(d.tiles) * 4;
     off += size_t(round_up(d.tiles * 4, 256));
+  }
+  if (K % 8 != 0) {
+    L.xp = off;
+    off += size_t(round_up(M * pitch8(K) * 2, 256));
+  }
+  if (N % 8 != 0) {
+    L.dyp = off;
+    off += size_t(round_up(M * pitch8(N) * 2, 256));
+    L.bp = off;
+    off += size_t(round_up(int64_t(r) * pitch8(N) * 2, 256));
   }
   L.total = off;
   return L;
@@ -236,9 +252,27 @@ nf4_status qlora_linear_fwd_ex(int32_t dtype, const uint16_t* X, int64_t M, nf4_
     return NF4_OK;
   }
 
+  // X and B with 16-byte row pitches for TMA (re-pitched copies for ragged K, N)
+  const uint16_t* Xa = X;
+  const uint16_t* Ba = B;
+  int64_t ldk = K, ldb = N;
+  if (K % 8 != 0) {
+    ldk = pitch8(K);
+    uint16_t* xp = reinterpret_cast<uint16_t*>(wsb + L.xp);
+    if (launch_repitch(X, M, K, xp, ldk, sms, strm) != cudaSuccess) return NF4_ERR_CUDA;
+    Xa = xp;
+  }
+  if (N % 8 != 0 && !decode_supported(M, K)) {   // the decode kernel reads B by elements
+    ldb = pitch8(N);
+    uint16_t* bp = reinterpret_cast<uint16_t*>(wsb + L.bp);
+    if (launch_repitch(B, r, N, bp, ldb, sms, strm) != cudaSuccess) return NF4_ERR_CUDA;
+    Ba = bp;
+  }
+
   SkinnyArgs sa{};
   sa.M = M; sa.N = N; sa.K = K; sa.r = r; sa.rp = rp; sa.s = s;
-  sa.X = X; sa.A = A; sa.B = B;
+  sa.X = Xa; sa.A = A; sa.B = Ba;
+  sa.ld_x = ldk;
   sa.T_out = t_dst; sa.hilo_out = hilo;
   sa.status = status;
   sa.pdl_mode = kPdlWaitFirst;
@@ -269,7 +303,8 @@ nf4_status qlora_linear_fwd_ex(int32_t dtype, const uint16_t* X, int64_t M, nf4_
   Nf4GemmArgs ga{};
   ga.M = M; ga.N = N; ga.K = K; ga.r = r; ga.rp = rp;
   ga.packed = w.packed; ga.c1q = w.c1q; ga.c2 = w.c2;
-  ga.act = X; ga.lora_w = B; ga.lora_act = hilo; ga.out = Y;
+  ga.act = Xa; ga.lora_w = Ba; ga.lora_act = hilo; ga.out = Y;
+  ga.ld_act = ldk; ga.ld_lw = ldb; ga.packed_bytes = packed_bytes_of(N * K);
   ga.status = status;
   ga.pdl_mode = kPdlWaitLowRank;
   ga.quant_type = w.quant_type; ga.dq = w.double_quant; ga.f16 = f16;
@@ -340,9 +375,31 @@ nf4_status qlora_linear_bwd_ex(int32_t dtype, const uint16_t* dY, const uint16_t
     return NF4_OK;
   }
 
+  // X, dY and B with 16-byte row pitches for TMA (re-pitched copies for ragged K, N)
+  const uint16_t* Xa = X;
+  const uint16_t* dYa = dY;
+  const uint16_t* Ba = B;
+  int64_t ldk = K, ldn = N;
+  if (K % 8 != 0) {
+    ldk = pitch8(K);
+    uint16_t* xp = reinterpret_cast<uint16_t*>(wsb + L.xp);
+    if (launch_repitch(X, M, K, xp, ldk, sms, strm) != cudaSuccess) return NF4_ERR_CUDA;
+    Xa = xp;
+  }
+  if (N % 8 != 0) {
+    ldn = pitch8(N);
+    uint16_t* dyp = reinterpret_cast<uint16_t*>(wsb + L.dyp);
+    uint16_t* bp = reinterpret_cast<uint16_t*>(wsb + L.bp);
+    if (launch_repitch(dY, M, N, dyp, ldn, sms, strm) != cudaSuccess) return NF4_ERR_CUDA;
+    if (launch_repitch(B, r, N, bp, ldn, sms, strm) != cudaSuccess) return NF4_ERR_CUDA;
+    dYa = dyp;
+    Ba = bp;
+  }
+
   SkinnyArgs sa{};
   sa.M = M; sa.N = N; sa.K = K; sa.r = r; sa.rp = rp; sa.s = s;
-  sa.X = X; sa.dY = dY; sa.A = A; sa.B = B;
+  sa.X = Xa; sa.dY = dYa; sa.A = A; sa.B = Ba;
+  sa.ld_x = ldk; sa.ld_dy = ldn; sa.ld_b = ldn;
   sa.status = status;
   sa.f16 = f16;
 
@@ -373,7 +430,8 @@ nf4_status qlora_linear_bwd_ex(int32_t dtype, const uint16_t* dY, const uint16_t
   Nf4GemmArgs ga{};
   ga.M = M; ga.N = N; ga.K = K; ga.r = r; ga.rp = rp;
   ga.packed = w.packed; ga.c1q = w.c1q; ga.c2 = w.c2;
-  ga.act = dY; ga.lora_w = A; ga.lora_act = hilo; ga.out = dX;
+  ga.act = dYa; ga.lora_w = A; ga.lora_act = hilo; ga.out = dX;
+  ga.ld_act = ldn; ga.ld_lw = r; ga.packed_bytes = packed_bytes_of(N * K);
   ga.status = status;
   ga.pdl_mode = kPdlWaitFirst;
   ga.quant_type = w.quant_type; ga.dq = w.double_quant; ga.f16 = f16;

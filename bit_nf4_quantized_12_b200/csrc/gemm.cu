@@ -102,7 +102,70 @@ constexpr int SX = 4, SP = 8, SA = 4;
 // wait would pass on the wrong phase.
 static_assert(SP % kDequantWGs == 0 && SA % kDequantWGs == 0, "ring slots must map to one dequant warpgroup");
 
-template <bool BWD>
+// Ragged mode reuses the idle packed ring: 48 bytes of load slot per dequant
+// thread, then the 64 x 16 lane-mask table of the two-table dequantization.
+constexpr uint32_t kRaggedMaskOffset = 128 * kDequantWGs * 48;
+static_assert(kRaggedMaskOffset + 64 * 16 * 8 <= SP * 4096, "ragged scratch must fit the packed ring");
+
+// The 64 codes of flat elements e0 .. e0 + 63 (element e in nibble e - e0),
+// from global memory at any nibble phase: the three 16-byte chunks that
+// cover them are copied into this thread's 48-byte slot (cp.async, zero fill
+// past the end of the packed array), then shifted into place.
+__device__ __forceinline__ void load_codes64(const uint8_t* packed, int64_t packed_bytes, int64_t e0, uint32_t slot,
+                                             uint32_t (&w)[8]) {
+  const int64_t byte0 = e0 >> 1;
+  const int64_t base = byte0 & ~int64_t(15);
+#pragma unroll
+  for (int j = 0; j < 3; ++j) {
+    const int64_t off = base + 16 * j;
+    const int64_t left = packed_bytes - off;
+    const uint32_t valid = left <= 0 ? 0u : (left >= 16 ? 16u : uint32_t(left));
+    const uint8_t* src = valid ? packed + off : packed;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(slot + 16 * j), "l"(src), "r"(valid)
+                 : "memory");
+  }
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  const uint32_t ob = uint32_t(byte0 - base);          // 0 .. 15
+  const uint32_t wb = slot + (ob & ~3u);
+  uint32_t v[9];
+#pragma unroll
+  for (int i = 0; i < 9; ++i) asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v[i]) : "r"(wb + 4 * i));
+  const uint32_t sel = 0x3210u + 0x1111u * (ob & 3u);   // bytes ob .. ob + 3 of a word pair
+  uint32_t y[9];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) y[i] = prmt(v[i], v[i + 1], sel);
+  y[8] = prmt(v[8], 0u, sel);
+  const uint32_t ns = (e0 & 1) ? 4u : 0u;              // odd e0: its code is the high nibble
+#pragma unroll
+  for (int i = 0; i < 8; ++i) w[i] = __funnelshift_r(y[i], y[i + 1], ns);
+}
+
+// 64 codes -> 32 bf16x2 (or f16x2) words in element order, each element taking
+// its value from t0 or, where its lane of masks[group] is set, from t1.
+__device__ __forceinline__ void dequant64_two(const BlockTable& t0, const BlockTable& t1, const uint32_t (&w)[8],
+                                              const uint2* masks, uint32_t (&o)[32]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t s = h ? (w[i] >> 16) : w[i];
+      uint32_t a01, a23, b01, b23;
+      lookup4(t0, s, a01, a23);
+      lookup4(t1, s, b01, b23);
+      const uint2 m = masks[2 * i + h];
+      o[4 * i + 2 * h] = (a01 & ~m.x) | (b01 & m.x);
+      o[4 * i + 2 * h + 1] = (a23 & ~m.y) | (b23 & m.y);
+    }
+  }
+}
+
+// RAGGED: W rows do not start on an NF4 block (K % 64 != 0).  The packed
+// codes then cannot be cut into TMA boxes; each dequant thread loads its row
+// segment of 64 codes straight from global memory (cp.async into a private
+// slot of the idle packed ring, at any nibble phase), and a segment that
+// straddles two NF4 blocks is dequantized with both blocks' tables, each
+// element taking its own block's value.
+template <bool BWD, bool RAGGED>
 __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_constant__ Nf4GemmParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -134,7 +197,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
   const int64_t my_main = g_end > g_begin ? g_end - g_begin : 0;
   const int my_lora = (split == 0) ? P.lora_steps : 0;
   const int64_t nsteps = my_main + my_lora;
-  const int64_t KB = a.K / kBlock;          // NF4 blocks per W row
   const uint32_t tmem_cols = uint32_t(bt < 32 ? 32 : bt);
 
   if (threadIdx.x == 32) {   // descriptor fetches overlap the setup below
@@ -154,6 +216,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
   if (warp == 2) {
     tmem_alloc(tmem_slot, tmem_cols);
     tmem_relinquish();
+  }
+  if (RAGGED && warp >= 4) {
+    // lane masks of the two-table dequantization: for a segment whose first
+    // element sits at offset o of its NF4 block, elements 64 - o .. 63 belong
+    // to the next block; entry (o, group of 4) selects those 16-bit lanes
+    uint2* masks = reinterpret_cast<uint2*>(pk_s + kRaggedMaskOffset);
+    for (int i = threadIdx.x - 128; i < 64 * 16; i += 128 * kDequantWGs) {
+      const int o = i >> 4, grp = i & 15;
+      uint32_t m[2] = {0u, 0u};
+      for (int e = 0; e < 4; ++e)
+        if (o != 0 && 4 * grp + e >= 64 - o) m[e >> 1] |= 0xFFFFu << (16 * (e & 1));
+      masks[i] = make_uint2(m[0], m[1]);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -191,7 +266,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
     __syncwarp();
   } else if (warp == 3) {
     // ------------------------------------------------------------ packed-W producer
-    if (elect_one()) {
+    if (!RAGGED && elect_one()) {
       int64_t issued = 0;
       for (int64_t ks = 0; ks < my_main; ++ks) {
         const int s = int(ks % SP);
@@ -250,36 +325,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
     // their global-memory latency is off the critical path.
     const int wg = (warp - 4) >> 2;
     const int t = threadIdx.x - 128 - 128 * wg;               // 0..127
-    auto block_of = [&](int64_t ks) -> int64_t {              // NF4 block index used at step ks, or -1
+    // first flat element of this thread's 64-weight row segment at step ks
+    // (row n, columns k0 .. k0 + 63), or -1 when the row or the columns lie
+    // outside W; with K % 64 == 0 it is the start of NF4 block e0 / 64
+    auto seg_of = [&](int64_t ks) -> int64_t {
       if (ks >= my_main) return -1;
       const int64_t g = g_begin + ks;
-      if (!BWD) {
-        const int64_t n = w0 + t;
-        return n < a.N ? n * KB + g : -1;
-      }
-      const int64_t n = g * 64 + (t & 63);
-      const int64_t kblk = w0 / 64 + (t >> 6);
-      return (n < a.N && kblk < KB) ? n * KB + kblk : -1;
+      const int64_t n = BWD ? g * 64 + (t & 63) : w0 + t;
+      const int64_t k0 = BWD ? w0 + (t >> 6) * 64 : g * 64;
+      return (n < a.N && k0 < a.K) ? n * a.K + k0 : -1;
     };
+    const int64_t nblk = nblocks_of(a.N * a.K);
     const bool f16 = a.f16 != 0;
-    uint32_t cq[4], nq[4];
-    float cc[4], nc[4];
+    uint32_t cq[4], nq[4], cq2[4], nq2[4];
+    float cc[4], nc[4], cc2[4], nc2[4];
+    // the constants of the segment's block, and in ragged mode of the next
+    // block when the segment reaches into it
+    auto load_consts = [&](int64_t ks, uint32_t& q, float& c, uint32_t& q2, float& c2) {
+      q = q2 = 0u;
+      c = c2 = 0.0f;
+      const int64_t e0 = seg_of(ks);
+      if (e0 < 0) return;
+      load_scale_parts(a.dq, a.c1q, a.c2, e0 >> 6, q, c);
+      if (RAGGED && (e0 & 63) != 0 && (e0 >> 6) + 1 < nblk) load_scale_parts(a.dq, a.c1q, a.c2, (e0 >> 6) + 1, q2, c2);
+    };
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int64_t b = block_of(wg + int64_t(j) * kDequantWGs);
-      cq[j] = 0u;
-      cc[j] = 0.0f;
-      if (b >= 0) load_scale_parts(a.dq, a.c1q, a.c2, b, cq[j], cc[j]);
-    }
+    for (int j = 0; j < 4; ++j) load_consts(wg + int64_t(j) * kDequantWGs, cq[j], cc[j], cq2[j], cc2[j]);
     bool ok = true;
     for (int64_t base = wg; base < nsteps && ok; base += 4 * kDequantWGs) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int64_t b = block_of(base + int64_t(4 + j) * kDequantWGs);
-        nq[j] = 0u;
-        nc[j] = 0.0f;
-        if (b >= 0) load_scale_parts(a.dq, a.c1q, a.c2, b, nq[j], nc[j]);
-      }
+      for (int j = 0; j < 4; ++j) load_consts(base + int64_t(4 + j) * kDequantWGs, nq[j], nc[j], nq2[j], nc2[j]);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int64_t ks = base + int64_t(j) * kDequantWGs;
@@ -287,18 +362,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
         const int sa = int(ks % SA);
         const uint32_t a_ph = uint32_t(ks / SA) & 1u;
         if (ks < my_main) {
-          const int sp = int(ks % SP);
-          if (!(ok = mbar_wait(&p_full[sp], uint32_t(ks / SP) & 1u, a.status, abort_flag))) break;
-          const uint32_t pa = BWD ? smem_u32(pk_s + sp * 4096 + (t & 63) * 64 + (t >> 6) * 32)
-                                  : smem_u32(pk_s + sp * 4096 + t * 32);
-          const uint4 p0 = lds128(pa), p1 = lds128(pa + 16);
-          // The slot is refilled by TMA, an async-proxy write: order these
-          // generic-proxy reads before it, or the refill can land first.
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&p_empty[sp]);
           uint32_t o[32];
-          dequant64(make_table(P.code, scale_from_parts(a.dq, cq[j], cc[j]), f16), p0, p1, o);
+          if (!RAGGED) {
+            const int sp = int(ks % SP);
+            if (!(ok = mbar_wait(&p_full[sp], uint32_t(ks / SP) & 1u, a.status, abort_flag))) break;
+            const uint32_t pa = BWD ? smem_u32(pk_s + sp * 4096 + (t & 63) * 64 + (t >> 6) * 32)
+                                    : smem_u32(pk_s + sp * 4096 + t * 32);
+            const uint4 p0 = lds128(pa), p1 = lds128(pa + 16);
+            // The slot is refilled by TMA, an async-proxy write: order these
+            // generic-proxy reads before it, or the refill can land first.
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_empty[sp]);
+            dequant64(make_table(P.code, scale_from_parts(a.dq, cq[j], cc[j]), f16), p0, p1, o);
+          } else {
+            const int64_t e0 = seg_of(ks);
+            uint32_t wv[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+            if (e0 >= 0)
+              load_codes64(a.packed, a.packed_bytes, e0, smem_u32(pk_s) + uint32_t(threadIdx.x - 128) * 48u, wv);
+            const uint2* masks = reinterpret_cast<const uint2*>(pk_s + kRaggedMaskOffset) + (e0 >= 0 ? (e0 & 63) : 0) * 16;
+            dequant64_two(make_table(P.code, scale_from_parts(a.dq, cq[j], cc[j]), f16),
+                          make_table(P.code, scale_from_parts(a.dq, cq2[j], cc2[j]), f16), wv, masks, o);
+          }
           // the A slot must have been released by the MMA of step ks - SA
           if (ks >= SA && !(ok = mbar_wait(&a_empty[sa], a_ph ^ 1u, a.status, abort_flag))) break;
           // forward: row t of Wd (K-major, 128-byte rows); backward: row
@@ -339,6 +424,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
       for (int j = 0; j < 4; ++j) {
         cq[j] = nq[j];
         cc[j] = nc[j];
+        cq2[j] = nq2[j];
+        cc2[j] = nc2[j];
       }
     }
 
@@ -370,8 +457,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
         for (int q = 0; q < 4; ++q) {
           const int e = q * 128 + t;                 // 16-byte piece: token row e / 16, columns (e % 16) * 8 ...
           const int64_t m = m0 + c * 32 + (e >> 4);
-          const int64_t col = w0 + (e & 15) * 8;     // wdim % 8 == 0, so the piece is whole or absent
-          if (m < a.M && col < wdim) stg128(a.out + m * wdim + col, lds128(stg + uint32_t(e) * 16));
+          const int64_t col = w0 + (e & 15) * 8;
+          if (m < a.M && col < wdim) {
+            const uint4 piece = lds128(stg + uint32_t(e) * 16);
+            if ((wdim & 7) == 0) {            // whole 16-byte pieces of 16-byte aligned rows
+              stg128(a.out + m * wdim + col, piece);
+            } else {                          // ragged rows: element stores
+              const uint32_t h[4] = {piece.x, piece.y, piece.z, piece.w};
+              for (int u = 0; u < 8 && col + u < wdim; ++u)
+                a.out[m * wdim + col + u] = uint16_t(h[u >> 1] >> (16 * (u & 1)));
+            }
+          }
         }
       } else {
 #pragma unroll
@@ -746,7 +842,7 @@ Nf4GemmPlan plan_nf4_gemm(int backward, int64_t M, int64_t N, int64_t K, int r, 
   const int64_t wdim = backward ? K : N;
   p.tiles_w = cdiv(wdim, 128);
   p.tiles_t = cdiv(M, p.bt);
-  p.main_steps = backward ? cdiv(N, 64) : K / 64;
+  p.main_steps = backward ? cdiv(N, 64) : cdiv(K, 64);
   const int rp = int(cdiv(r, 64) * 64);
   p.lora_steps = 2 * (rp / 64);
   p.splits = choose_splits(p.tiles_w * p.tiles_t, p.main_steps, num_sms, 4, (num_sms * 7) / 8);
@@ -820,20 +916,27 @@ cudaError_t launch_nf4_gemm(const Nf4GemmPlan& plan, const Nf4GemmArgs& a, cudaS
   const uint64_t M = a.M, N = a.N, K = a.K;
   const uint64_t hw = 2 * uint64_t(a.rp);
   const uint32_t act_box = uint32_t(plan.bt);
+  // activations and B may sit in re-pitched copies (row pitch ld_act / ld_lw
+  // elements, a multiple of 8); their extents stay the logical K and N, so TMA
+  // fills everything past them with zeros
+  const bool ragged = K % 64 != 0;
+  const uint64_t lda = uint64_t(a.ld_act), ldl = uint64_t(a.ld_lw);
   if (!plan.backward) {
-    ok &= encode_tmap_2d(&P.tm_act, BF, a.act, K, M, K * 2, 64, act_box, SW);
-    ok &= encode_tmap_2d(&P.tm_pk, U8, a.packed, K / 2, N, K / 2, 32, 128, NOSW);
-    ok &= encode_tmap_2d(&P.tm_lw, BF, a.lora_w, N, uint64_t(a.r), N * 2, 64, 64, SW);
+    ok &= encode_tmap_2d(&P.tm_act, BF, a.act, K, M, lda * 2, 64, act_box, SW);
+    if (!ragged) ok &= encode_tmap_2d(&P.tm_pk, U8, a.packed, K / 2, N, K / 2, 32, 128, NOSW);
+    ok &= encode_tmap_2d(&P.tm_lw, BF, a.lora_w, N, uint64_t(a.r), ldl * 2, 64, 64, SW);
   } else {
-    ok &= encode_tmap_2d(&P.tm_act, BF, a.act, N, M, N * 2, 64, act_box, SW);
-    ok &= encode_tmap_2d(&P.tm_pk, U8, a.packed, K / 2, N, K / 2, 64, 64, NOSW);
+    ok &= encode_tmap_2d(&P.tm_act, BF, a.act, N, M, lda * 2, 64, act_box, SW);
+    if (!ragged) ok &= encode_tmap_2d(&P.tm_pk, U8, a.packed, K / 2, N, K / 2, 64, 64, NOSW);
     ok &= encode_tmap_2d(&P.tm_lw, BF, a.lora_w, uint64_t(a.r), K, uint64_t(a.r) * 2, 64, 128, SW);
   }
   ok &= encode_tmap_2d(&P.tm_lact, BF, a.lora_act, hw, M, hw * 2, 64, act_box, SW);
   if (!ok) return cudaErrorInvalidValue;
   const size_t smem = nf4_gemm_smem(plan.backward, plan.bt);
   dim3 grid(unsigned(plan.tiles_w), unsigned(plan.tiles_t), unsigned(plan.splits));
-  void (*kern)(const Nf4GemmParams) = plan.backward ? nf4_gemm_kernel<true> : nf4_gemm_kernel<false>;
+  void (*kern)(const Nf4GemmParams);
+  if (ragged) kern = plan.backward ? nf4_gemm_kernel<true, true> : nf4_gemm_kernel<false, true>;
+  else kern = plan.backward ? nf4_gemm_kernel<true, false> : nf4_gemm_kernel<false, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   return launch_clustered(kern, grid, dim3(kGemmThreads), smem, stream, dim3(1, 1, unsigned(plan.splits)), pdl, P);
@@ -851,27 +954,31 @@ cudaError_t launch_skinny(const SkinnyPlan& plan, const SkinnyArgs& a, cudaStrea
   const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;   // 2-byte elements (bf16 or fp16)
   const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
   const uint64_t M = a.M, N = a.N, K = a.K, r = uint64_t(a.r), rp = uint64_t(a.rp);
+  // row pitches (elements) of X, dY and B: their re-pitched copies for ragged shapes
+  const uint64_t ldk = a.ld_x ? uint64_t(a.ld_x) : K;
+  const uint64_t ldn = a.ld_dy ? uint64_t(a.ld_dy) : N;
+  const uint64_t ldb = a.ld_b ? uint64_t(a.ld_b) : N;
   bool ok = true;
   switch (plan.kind) {
     case kSkinnyT:   // A-op X [M,K] K-major; B-op A [K,r] MN-major
       P.a_mn = 0; P.b_mn = 1;
-      ok &= encode_tmap_2d(&P.tm_a, BF, a.X, K, M, K * 2, 64, 128, SW);
+      ok &= encode_tmap_2d(&P.tm_a, BF, a.X, K, M, ldk * 2, 64, 128, SW);
       ok &= encode_tmap_2d(&P.tm_b, BF, a.A, r, K, r * 2, 64, 64, SW);
       break;
     case kSkinnyG:   // A-op dY [M,N] K-major; B-op B [r,N] K-major
       P.a_mn = 0; P.b_mn = 0;
-      ok &= encode_tmap_2d(&P.tm_a, BF, a.dY, N, M, N * 2, 64, 128, SW);
-      ok &= encode_tmap_2d(&P.tm_b, BF, a.B, N, r, N * 2, 64, uint32_t(rp), SW);
+      ok &= encode_tmap_2d(&P.tm_a, BF, a.dY, N, M, ldn * 2, 64, 128, SW);
+      ok &= encode_tmap_2d(&P.tm_b, BF, a.B, N, r, ldb * 2, 64, uint32_t(rp), SW);
       break;
     case kSkinnyDA:  // A-op X^T (MN-major view of X); B-op G hi/lo MN-major
       P.a_mn = 1; P.b_mn = 1;
       P.pass_steps = plan.steps / 2;
-      ok &= encode_tmap_2d(&P.tm_a, BF, a.X, K, M, K * 2, 64, 64, SW);
+      ok &= encode_tmap_2d(&P.tm_a, BF, a.X, K, M, ldk * 2, 64, 64, SW);
       ok &= encode_tmap_2d(&P.tm_b, BF, a.hilo_in, 2 * rp, M, 2 * rp * 2, 64, 64, SW);
       break;
     default:         // dB^T: A-op dY^T (MN-major view of dY); B-op T MN-major
       P.a_mn = 1; P.b_mn = 1;
-      ok &= encode_tmap_2d(&P.tm_a, BF, a.dY, N, M, N * 2, 64, 64, SW);
+      ok &= encode_tmap_2d(&P.tm_a, BF, a.dY, N, M, ldn * 2, 64, 64, SW);
       ok &= encode_tmap_2d(&P.tm_b, BF, a.T, r, M, r * 2, 64, 64, SW);
       break;
   }

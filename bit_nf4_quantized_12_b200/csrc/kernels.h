@@ -23,6 +23,11 @@ cudaError_t launch_dequant(const uint8_t* packed, const uint8_t* c1, const float
                            int quant_type, int dq, int f16, uint16_t* out, int num_sms, cudaStream_t stream);
 bool quantize_table_ok(int quant_type);
 
+// Copy src [rows, cols] (2-byte elements, pitch cols) into dst with row pitch
+// ld >= cols (elements); the columns past cols are left as they are.
+cudaError_t launch_repitch(const uint16_t* src, int64_t rows, int64_t cols, uint16_t* dst, int64_t ld, int num_sms,
+                           cudaStream_t stream);
+
 // ---------------------------------------------------------------- LoRA merge
 // out[n, k] = round(Wd[n, k] + s sum_j A[k, j] B[j, n]) in the compute type.
 struct MergeArgs {
@@ -76,6 +81,9 @@ struct Nf4GemmArgs {
   int quant_type;            // table (kQuantNf4 / kQuantInt4)
   int dq;                    // DqFormat of the first-level constants (c1q holds fp32 for kDqNone)
   int f16;                   // compute type fp16 (else bf16)
+  int64_t packed_bytes;      // size of the packed array (loads past it read zeros)
+  int64_t ld_act;            // row pitch (elements) of act: K or N, or a re-pitched copy's
+  int64_t ld_lw;             // row pitch of lora_w (forward: B's, N or its copy's; backward: r)
 };
 // pdl: launch as a programmatic dependent of the previous kernel of the stream
 cudaError_t launch_nf4_gemm(const Nf4GemmPlan& plan, const Nf4GemmArgs& a, cudaStream_t stream, bool pdl);
@@ -114,6 +122,7 @@ struct SkinnyArgs {
   uint32_t* status;
   int pdl_mode;             // PdlMode (kPdlWaitFirst or kPdlWaitLast)
   int f16;                  // compute type fp16 (else bf16)
+  int64_t ld_x, ld_dy, ld_b;  // row pitches of X, dY, B when they are re-pitched copies (0: K, N, N)
 };
 cudaError_t launch_skinny(const SkinnyPlan& plan, const SkinnyArgs& a, cudaStream_t stream, bool pdl);
 

@@ -59,14 +59,18 @@ def test_host_validation_before_launch():
     # linear layer: rank bounds, workspace
     assert L.qlora_linear_fwd(fake, 16, w, fake, fake, 0, 1.0, fake, None, fake, 1 << 30, None) == 1
     assert L.qlora_linear_fwd(fake, 16, w, fake, fake, 300, 1.0, fake, None, fake, 1 << 30, None) == 1
-    # shapes off the fused kernels' granules (K % 64, N % 8, r % 8) take the
-    # generic path, whose workspace also holds the dequantized W
+    # a rank off the 8-element granule takes the generic path, whose workspace
+    # also holds the dequantized W; ragged K and N stay on the tensor cores,
+    # with X (K % 8 != 0), dY and B (N % 8 != 0) re-pitched instead
     w_rag = binding.NF4Weight(0x10000, 0x10000, 0x10000, 64, 100)      # K % 64 != 0
+    need = L.qlora_workspace_bytes(16, 64, 100, 12)
+    assert need >= 256 + 64 * 100 * 2 + 16 * 12 * 2 + 16 * 12 * 4
+    assert L.qlora_linear_fwd(fake, 16, w_rag, fake, fake, 12, 1.0, fake, None, fake, need - 1, None) == 4
     need = L.qlora_workspace_bytes(16, 64, 100, 16)
-    assert need >= 256 + 64 * 100 * 2 + 16 * 16 * 2 + 16 * 16 * 4
+    assert 16 * 104 * 2 <= need < 64 * 100 * 2 + 16 * 104 * 2                     # X re-pitched, no Wd copy
     assert L.qlora_linear_fwd(fake, 16, w_rag, fake, fake, 16, 1.0, fake, None, fake, need - 1, None) == 4
     assert L.qlora_workspace_bytes(16, 64, 128, 12) >= 256 + 64 * 128 * 2          # r % 8 != 0
-    assert L.qlora_workspace_bytes(16, 60, 128, 16) >= 256 + 60 * 128 * 2          # N % 8 != 0
+    assert L.qlora_workspace_bytes(64, 60, 128, 16) >= 256 + 2 * 64 * 64 * 2        # N % 8: dY, B re-pitched
     assert L.qlora_workspace_bytes(32, 64, 128, 16) < 64 * 128 * 2                 # fused: no Wd copy
     assert L.qlora_linear_fwd(fake, 16, w, fake, fake, 12, 1.0, fake, None, fake, 16, None) == 4
     assert L.qlora_workspace_bytes(16, 1 << 31, 1 << 31, 12) == 0                  # Wd copy too large

@@ -109,19 +109,24 @@ def test_llama7b_layer_sampled_rows(idx):
 
 
 @pytest.mark.parametrize("M,N,K,r,s", [(5, 24, 100, 8, 2.0), (33, 40, 1000, 12, 0.5), (17, 13, 64, 8, 1.0),
-                                       (1, 96, 130, 4, 4.0), (70, 100, 257, 3, 1.5), (40, 8, 4095, 16, 0.25)])
-def test_ragged_shapes_generic_path(M, N, K, r, s):
-    """Shapes outside the fused kernels: K % 64 != 0 (rows of W do not start on
-    an NF4 block), N % 8 != 0, r % 8 != 0, and one token with a ragged K."""
+                                       (1, 96, 130, 4, 4.0), (70, 100, 257, 3, 1.5), (40, 8, 4095, 16, 0.25),
+                                       (2, 13, 4100, 8, 1.0), (300, 520, 11007, 16, 0.5), (129, 4095, 1000, 8, 4.0),
+                                       (64, 1001, 129, 64, 0.25), (16, 1024, 3001, 8, 1.0)])
+def test_ragged_shapes(M, N, K, r, s):
+    """K % 64 != 0 (rows of W do not start on an NF4 block, nibble phase odd
+    or even, segments straddling two blocks), N % 8 != 0 (ragged output rows),
+    one or two tokens, split reductions: the fused GEMM's ragged mode.  A rank
+    off the 8-element granule (r = 12, 4, 3): the generic path."""
     _run(M, N, K, r, s, seed=M + N + K)
 
 
 def test_robust_weight_layer_sampled_rows():
     """The 4095 x 11007 Student-t weight with outliers at 4096 tokens, r = 8,
     alpha = 32 (K = 11007 is not a multiple of the block): 128 sampled token
-    rows for Y and dX, full dA and dB."""
+    rows for Y and dX, full dA and dB, on the tensor cores (ragged mode)."""
     wl = workloads.WORKLOADS["robust"]
     _, N, K = wl.mats[0]
+    assert binding.plan(wl.tokens, N, K, wl.r)["path"] == binding.PATH_FUSED
     W = workloads.weight(N, K, wl.w_std, seed=0, device=DEV, kind=wl.w_kind)
     io = workloads.layer_inputs(wl.tokens, N, K, wl.r, seed=0, device=DEV)
     rows = np.sort(np.random.default_rng(5).choice(wl.tokens, 128, replace=False))
@@ -151,13 +156,14 @@ def test_decode_kernel_edges(M, N, K, r):
 
 
 @pytest.mark.parametrize("M,N,K", [(16, 4104, 2112), (1, 1024, 4096), (7, 520, 640), (64, 1032, 2112),
-                                   (300, 384, 1024)])
+                                   (300, 384, 1024), (40, 1001, 1000), (3, 13, 4099), (257, 4095, 1007)])
 def test_one_hot_tokens_give_the_dequantized_weight_bitwise(M, N, K):
     """Token m = the unit vector e_{k_m} and A = 0: Y[m, n] = Wd[n, k_m], a
     single exact product, so Y must equal the oracle's dequantized weight
     bit for bit.  Likewise dY = e_{n_m}, B = 0: dX[m, k] = Wd[n_m, k].  This
     pins the on-chip dequantization of the decode kernel (M <= 16) and of the
-    fused GEMM (forward and backward) to the fp32-multiply-then-round rule."""
+    fused GEMM (forward and backward, aligned and ragged K) to the
+    fp32-multiply-then-round rule."""
     r = 16
     W = workloads.weight(N, K, 0.02, seed=N + K, device=DEV)
     qw, st = gpu_quantize(W)

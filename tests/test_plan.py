@@ -3,9 +3,10 @@
 qlora_linear_plan reports the path, tiles and reduction splits the library
 picks for a call.  These tests sweep shapes and SM counts and check what the
 kernels rely on:
-  - the path: generic exactly when K % 64, N % 8 or r % 8 is nonzero; the
-    decode kernel exactly for a forward with 1 to 16 tokens; its persistent
-    CTAs take every (tile, column chunk) unit once;
+  - the path: generic exactly when r % 8 is nonzero (ragged K and N run on
+    the tensor cores); the decode kernel exactly for a forward with 1 to 16
+    tokens and K % 64 == 0; its persistent CTAs take every (tile, column
+    chunk) unit once;
   - the tile grid covers the output exactly once and fits the launch limits;
   - a split reduction is used only when the tiles leave SMs idle, fits one
     cluster (<= 8 CTAs) and gives every CTA at least one step of the
@@ -39,15 +40,15 @@ LOWRANK_STEPS = {  # 64-wide reduction steps of T, G, dA (hi and lo passes), dB
 
 def check_plan(M, N, K, r, backward, sms):
     p = binding.plan(M, N, K, r, backward=backward, num_sms=sms)
-    generic = K % 64 != 0 or N % 8 != 0 or r % 8 != 0
+    generic = r % 8 != 0
     if generic:
         assert p["path"] == binding.PATH_GENERIC
         assert p["lowrank_splits"] == [0, 0, 0, 0]
         return p
-    if not backward and M <= 16:
+    if not backward and M <= 16 and K % 64 == 0:
         assert p["path"] == binding.PATH_DECODE
     if p["path"] == binding.PATH_DECODE:
-        assert not backward and M <= 16
+        assert not backward and M <= 16 and K % 64 == 0
         assert p["tiles_w"] == cdiv(N, 256) and p["main_steps"] == cdiv(K, 256) and p["tiles_t"] == 1
         units = p["tiles_w"] * p["main_steps"]
         ctas = p["splits"]
@@ -62,7 +63,7 @@ def check_plan(M, N, K, r, backward, sms):
         assert p["tiles_t"] == cdiv(M, bt) and (p["tiles_t"] - 1) * bt < M <= p["tiles_t"] * bt
         assert p["tiles_t"] <= 65535
         assert p["tiles_w"] == cdiv(K if backward else N, 128)
-        steps = cdiv(N, 64) if backward else K // 64
+        steps = cdiv(N, 64) if backward else cdiv(K, 64)
         assert p["main_steps"] == steps
         assert p["lora_steps"] == 2 * cdiv(r, 64)
         s = p["splits"]
@@ -110,11 +111,23 @@ def test_every_split_count_is_exercised():
     assert {1, 2, 4, 8} <= seen_low
 
 
-@pytest.mark.parametrize("M,N,K,r", [(5, 24, 100, 8), (33, 40, 1000, 12), (17, 13, 64, 8), (1, 96, 130, 4),
-                                     (4096, 4095, 11007, 8), (1, 4096, 4096, 12), (4, 4095, 4096, 8)])
-def test_ragged_shapes_take_the_generic_path(M, N, K, r):
+@pytest.mark.parametrize("M,N,K,r", [(33, 40, 1000, 12), (1, 96, 130, 4), (1, 4096, 4096, 12), (5, 24, 100, 3)])
+def test_ranks_off_the_granule_take_the_generic_path(M, N, K, r):
     for backward in (0, 1):
         assert check_plan(M, N, K, r, backward, 148)["path"] == binding.PATH_GENERIC
+
+
+@pytest.mark.parametrize("M,N,K,r", [(5, 24, 100, 8), (17, 13, 64, 8), (4096, 4095, 11007, 8), (4, 4095, 4096, 8),
+                                     (1, 8, 4100, 16), (2048, 11008, 4095, 64)])
+def test_ragged_shapes_take_the_tensor_cores(M, N, K, r):
+    """K % 64 != 0 (rows not starting on an NF4 block) and N % 8 != 0 run on
+    the tensor cores: the fused GEMM, or the decode kernel for a forward with
+    up to 16 tokens whose rows start on blocks."""
+    for backward in (0, 1):
+        p = check_plan(M, N, K, r, backward, 148)
+        want = binding.PATH_DECODE if (not backward and M <= 16 and K % 64 == 0) else binding.PATH_FUSED
+        assert p["path"] == want
+        assert binding.workspace_bytes(M, N, K, r) < N * K * 2 or M * (K + N) * 2 >= N * K  # no copy of Wd
 
 
 def test_plans_match_the_calls_limits():
@@ -124,10 +137,11 @@ def test_plans_match_the_calls_limits():
     cases = [
         ((max_fused, 4096, 64, 8), 0),
         ((max_fused + 1, 4096, 64, 8), 3),       # token tiles beyond grid.y
-        ((max_fused + 1, 4096, 100, 8), 0),      # the generic path walks its tiles
+        ((max_fused + 1, 4096, 100, 8), 3),      # ragged K runs on the fused grid too
+        ((max_fused + 1, 4096, 100, 12), 0),     # the generic path walks its tiles
         ((1 << 31, 8, 64, 8), 3),
-        ((1 << 31, 8, 100, 8), 0),
-        (((1 << 31) + 1, 8, 100, 8), 3),
+        ((1 << 31, 8, 100, 12), 0),
+        (((1 << 31) + 1, 8, 100, 12), 3),
         ((16, 1 << 31, 1 << 31, 12), 3),         # Wd copy beyond 2^40 elements
         ((0, 64, 64, 8), 1),
         ((16, 64, 64, 0), 1),
