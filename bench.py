@@ -532,6 +532,8 @@ def kernel_case(case, n):
         M, r, s, N, K = (16 if case == "decode" else 1), 16, 1.0, 28672, 8192
     if case in ("quantize", "dequant"):
         M, r, s, N, K = 16, 16, 1.0, 28672, 8192
+    if case in ("robust_fwd", "robust_bwd"):   # ragged K and N: the fused GEMM's ragged mode
+        M, r, s, N, K = 4096, 8, 4.0, 4095, 11007
     W = workloads.weight(N, K, 0.02, seed=0, device=dev)
     io = workloads.layer_inputs(M, N, K, r, seed=0, device=dev)
     qw = binding.quantize(W)
@@ -545,7 +547,7 @@ def kernel_case(case, n):
             binding.dequant(qw, out=Wd)
         elif case == "merge":
             binding.lora_merge(qw, io["A"], io["B"], s, out=Wd)
-        elif case in ("fwd", "decode", "gemv"):
+        elif case in ("fwd", "decode", "gemv", "robust_fwd"):
             binding.linear_fwd(io["X"], qw, io["A"], io["B"], s, ws=ws, Y=Y, T=T)
         else:
             binding.linear_bwd(io["dY"], io["X"], qw, io["A"], io["B"], s, T=T, ws=ws)
@@ -560,7 +562,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-components", action="store_true")
-    ap.add_argument("--kernel-case", default=None, choices=["quantize", "dequant", "fwd", "bwd", "decode", "gemv", "merge"],
+    ap.add_argument("--kernel-case", default=None, choices=["quantize", "dequant", "fwd", "bwd", "decode", "gemv", "merge", "robust_fwd",
+                                                         "robust_bwd"],
                     help="run a few launches of one call on one 7B-shaped matrix (for ncu), print nothing")
     args = ap.parse_args()
 

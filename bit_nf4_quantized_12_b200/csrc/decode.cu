@@ -171,14 +171,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) nf4_decode_kernel(const __grid
 #pragma unroll
     for (int q = 0; q < 4; ++q) acc[nt][q] = 0.0f;
 
-  // block constants of (row, block c of unit u), loaded one unit ahead
-  auto load_scales = [&](int64_t u, uint32_t (&q)[2], float (&s2)[2]) {
+  // block constants of (row, block c of unit (tile, kc)), loaded one unit ahead
+  auto load_scales = [&](bool valid, int64_t tile, int64_t kc, uint32_t (&q)[2], float (&s2)[2]) {
     q[0] = q[1] = 0u;
     s2[0] = s2[1] = 0.0f;
-    if (u >= u1) return;
-    const int64_t tile = u / P.nk, kc = u % P.nk;
     const int64_t kb = kc * 4 + c;
-    if (kb >= KB) return;
+    if (!valid || kb >= KB) return;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int64_t n = tile * kDecTileRows + row0 + 8 * h;
@@ -187,7 +185,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) nf4_decode_kernel(const __grid
   };
   uint32_t cq[2], nq[2];
   float cs[2], ns[2];
-  load_scales(u0, cq, cs);
+  int64_t tile = u0 / P.nk, kc = u0 % P.nk;          // unit u = tile * nk + kc, advanced without division
+  load_scales(true, tile, kc, cq, cs);
 
   // Every consumer warp walks the same units and meets the same barriers,
   // whatever happens: after a failed wait (ok == false) a warp skips the work
@@ -198,8 +197,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) nf4_decode_kernel(const __grid
   for (int64_t u = u0; u < u1; ++u) {
     const int64_t i = u - u0;
     const int s = int(i % kDecStages);
-    const int64_t tile = u / P.nk, kc = u % P.nk;
-    load_scales(u + 1, nq, ns);
+    {
+      const bool last_kc = kc + 1 == P.nk;
+      load_scales(u + 1 < u1, last_kc ? tile + 1 : tile, last_kc ? 0 : kc + 1, nq, ns);
+    }
     if (ok) ok = mbar_wait(&full[s], uint32_t(i / kDecStages) & 1u, a.status, abort_flag);
     if (ok) {
       const uint32_t st = smem_u32(smem + s * P.stage_bytes);
@@ -222,8 +223,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) nf4_decode_kernel(const __grid
       const uint32_t xb = st + kPkBytes + uint32_t(c) * P.xbox_bytes + uint32_t(g) * 128u;
 #pragma unroll
       for (int t = 0; t < 16; ++t) {
-        const uint32_t s0 = (t & 1) ? (w0[t >> 1] >> 16) : w0[t >> 1];
-        const uint32_t s1 = (t & 1) ? (w1[t >> 1] >> 16) : w1[t >> 1];
+        // upper halves by a high multiply (FMA pipe): the integer pipe is the
+        // one the lookups keep busy
+        const uint32_t s0 = (t & 1) ? __umulhi(w0[t >> 1], 0x10000u) : w0[t >> 1];
+        const uint32_t s1 = (t & 1) ? __umulhi(w1[t >> 1], 0x10000u) : w1[t >> 1];
         uint32_t a0, a1, a2, a3;
         lookup4(t0, s0, a0, a2);
         lookup4(t1, s1, a1, a3);
@@ -242,7 +245,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) nf4_decode_kernel(const __grid
     cq[0] = nq[0]; cq[1] = nq[1]; cs[0] = ns[0]; cs[1] = ns[1];
 
     // ---------------------------------------------------------- tile segment end
-    if (kc != P.nk - 1 && u != u1 - 1) continue;
+    if (kc != P.nk - 1 && u != u1 - 1) {
+      ++kc;
+      continue;
+    }
     const bool whole = seg_first_kc == 0 && kc == P.nk - 1;
     // park the accumulators as red[token][row]
 #pragma unroll
@@ -283,31 +289,48 @@ __global__ void __launch_bounds__(kDecThreads, 1) nf4_decode_kernel(const __grid
         griddep_wait();
         have_T = true;
       }
-      for (int64_t e = tid; e < per_slot; e += kDecWarps * 32) {
-        const int tk = int(e / kDecTileRows), row = int(e % kDecTileRows);
-        const int64_t n = n0 + row;
-        if (n >= a.N) continue;
-        float v;
-        if (whole) {
-          v = red[e];
-        } else {   // contributors in CTA order: a fixed summation order
-          v = 0.0f;
-          for (int64_t q = pa; q <= pb; ++q) {
-            const int slot = (unit_begin(q, P.units, NP) / P.nk == tile) ? 0 : 1;
-            v += __ldcg(a.partial + (q * 2 + slot) * per_slot + e);
+      // this thread's outputs: e = tid + 512 j (token e / 256, row e % 256)
+      constexpr int kPer = 16 * kDecTileRows / (kDecWarps * 32);   // 8
+      float v[kPer];
+#pragma unroll
+      for (int jj = 0; jj < kPer; ++jj) {
+        const int64_t e = tid + int64_t(jj) * (kDecWarps * 32);
+        v[jj] = (whole && e < per_slot) ? red[e] : 0.0f;
+      }
+      if (!whole) {   // contributors in CTA order: a fixed summation order
+        for (int64_t q = pa; q <= pb; ++q) {
+          const int slot = unit_begin(q, P.units, NP) >= tile * P.nk ? 0 : 1;
+          const float* part = a.partial + (q * 2 + slot) * per_slot;
+#pragma unroll
+          for (int jj = 0; jj < kPer; ++jj) {
+            const int64_t e = tid + int64_t(jj) * (kDecWarps * 32);
+            if (e < per_slot) v[jj] += __ldcg(part + e);
           }
         }
+      }
+#pragma unroll
+      for (int jj = 0; jj < kPer; ++jj) {
+        const int64_t e = tid + int64_t(jj) * (kDecWarps * 32);
+        const int tk = int(e / kDecTileRows), row = int(e % kDecTileRows);
+        const int64_t n = n0 + row;
+        if (e >= per_slot || n >= a.N) continue;
         float lr = 0.0f;
         for (int j = 0; j < a.r; ++j)
           lr = fmaf(half_lo_to_f32(F16, a.T[int64_t(tk) * a.r + j]), half_lo_to_f32(F16, a.B[int64_t(j) * a.N + n]),
                     lr);
-        a.Y[int64_t(tk) * a.N + n] = uint16_t(pack2(F16, fmaf(a.s, lr, v), 0.0f) & 0xFFFFu);
+        a.Y[int64_t(tk) * a.N + n] = uint16_t(pack2(F16, fmaf(a.s, lr, v[jj]), 0.0f) & 0xFFFFu);
       }
       if (!whole && tid == 0) a.counters[tile] = 0;   // ready for the next call
     }
     consumer_sync();   // red is reused by the next segment
     first_segment = false;
     seg_first_kc = 0;
+    if (kc + 1 == P.nk) {
+      ++tile;
+      kc = 0;
+    } else {
+      ++kc;
+    }
   }
   if (!have_T) griddep_wait();   // complete only after the previous kernel
 }

@@ -79,41 +79,87 @@ __global__ void __launch_bounds__(kMergeThreads) nf4_merge_kernel(const __grid_c
   const int64_t n0 = int64_t(blockIdx.y) * kTile;
   if (tid < 16) code_s[tid] = P.code[tid];
 
-  // ---- stage the operand slices (zero padded past r, N and K)
-  const int jc = rp / 8;                         // 8-wide chunks per operand row
-  for (int i = tid; i < kTile * jc; i += kMergeThreads) {   // A[k0 + row][8c .. 8c+7]
-    const int row = i / jc, c = i % jc;
-    const int64_t k = k0 + row;
-    uint32_t v[4] = {0u, 0u, 0u, 0u};
-    if (k < a.K) {
-      const uint16_t* src = a.A + k * a.r + c * 8;
-      if (c * 8 + 8 <= a.r && (a.r % 8) == 0) {
-        const uint4 u = __ldg(reinterpret_cast<const uint4*>(src));
-        v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
-      } else {
-        for (int j = 0; j < 8; ++j)
-          if (c * 8 + j < a.r) v[j >> 1] |= uint32_t(src[j]) << (16 * (j & 1));
+  // ---- the epilogue's packed codes and block constants, loaded first so that
+  // their latency overlaps the staging and the MMAs.  Thread tid handles the
+  // 8-column piece pc = tid % 16 of rows tid / 16 + 16 j, j = 0..7.
+  const bool vec = (a.K % 8) == 0;
+  const int pc = tid & 15;
+  constexpr int kPieces = kTile * (kTile / 8) / kMergeThreads;   // 8
+  uint32_t pw[kPieces];
+  float ps[kPieces];
+  if (vec) {
+#pragma unroll
+    for (int j = 0; j < kPieces; ++j) {
+      const int64_t n = n0 + (tid >> 4) + 16 * j;
+      const int64_t k = k0 + pc * 8;
+      pw[j] = 0u;
+      ps[j] = 0.0f;
+      if (n < a.N && k < a.K) {
+        const int64_t e0 = n * a.K + k;
+        pw[j] = __ldcs(reinterpret_cast<const unsigned int*>(a.packed + (e0 >> 1)));
+        ps[j] = block_scale(a.double_quant, a.c1, a.c2, e0 >> 6);
       }
     }
-    *reinterpret_cast<uint4*>(a_s + row * srow + c * 16) = make_uint4(v[0], v[1], v[2], v[3]);
+  }
+
+  // ---- stage the operand slices (zero padded past r, N and K), four 16-byte
+  // loads in flight per thread
+  const int jc = rp / 8;                         // 8-wide chunks per operand row
+  for (int i0 = tid; i0 < kTile * jc; i0 += 4 * kMergeThreads) {   // A[k0 + row][8c .. 8c+7]
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * kMergeThreads;
+      v[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (i >= kTile * jc) continue;
+      const int row = i / jc, c = i % jc;
+      const int64_t k = k0 + row;
+      if (k >= a.K) continue;
+      const uint16_t* src = a.A + k * a.r + c * 8;
+      if (c * 8 + 8 <= a.r && (a.r % 8) == 0) {
+        v[u] = __ldg(reinterpret_cast<const uint4*>(src));
+      } else {
+        uint32_t t[4] = {0u, 0u, 0u, 0u};
+        for (int j = 0; j < 8; ++j)
+          if (c * 8 + j < a.r) t[j >> 1] |= uint32_t(src[j]) << (16 * (j & 1));
+        v[u] = make_uint4(t[0], t[1], t[2], t[3]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * kMergeThreads;
+      if (i < kTile * jc) *reinterpret_cast<uint4*>(a_s + (i / jc) * srow + (i % jc) * 16) = v[u];
+    }
   }
   constexpr int nc = kTile / 8;                  // 8-wide chunks of a row of B's slice
-  for (int i = tid; i < rp * nc; i += kMergeThreads) {     // B[j][n0 + 8c .. n0 + 8c + 7] -> B^T rows
-    const int j = i / nc, c = i % nc;
-    uint16_t v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    if (j < a.r) {
+  for (int i0 = tid; i0 < rp * nc; i0 += 4 * kMergeThreads) {     // B[j][n0 + 8c ..] -> B^T rows
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * kMergeThreads;
+      v[u] = make_uint4(0u, 0u, 0u, 0u);
+      const int j = i / nc, c = i % nc;
+      if (i >= rp * nc || j >= a.r) continue;
       const int64_t nb = n0 + c * 8;
       const uint16_t* src = a.B + int64_t(j) * a.N + nb;
       if (nb + 8 <= a.N && (a.N % 8) == 0) {
-        const uint4 u = __ldg(reinterpret_cast<const uint4*>(src));
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-        for (int q = 0; q < 8; ++q) v[q] = uint16_t(w[q >> 1] >> (16 * (q & 1)));
+        v[u] = __ldg(reinterpret_cast<const uint4*>(src));
       } else {
+        uint32_t t[4] = {0u, 0u, 0u, 0u};
         for (int q = 0; q < 8; ++q)
-          if (nb + q < a.N) v[q] = src[q];
+          if (nb + q < a.N) t[q >> 1] |= uint32_t(src[q]) << (16 * (q & 1));
+        v[u] = make_uint4(t[0], t[1], t[2], t[3]);
       }
     }
-    for (int q = 0; q < 8; ++q) *reinterpret_cast<uint16_t*>(bt_s + (c * 8 + q) * srow + j * 2) = v[q];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * kMergeThreads;
+      if (i >= rp * nc) continue;
+      const int j = i / nc, c = i % nc;
+      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      for (int q = 0; q < 8; ++q)
+        *reinterpret_cast<uint16_t*>(bt_s + (c * 8 + q) * srow + j * 2) = uint16_t(w[q >> 1] >> (16 * (q & 1)));
+    }
   }
   __syncthreads();
 
@@ -164,27 +210,32 @@ __global__ void __launch_bounds__(kMergeThreads) nf4_merge_kernel(const __grid_c
   __syncthreads();
 
   // ---- epilogue: W' = round(fma(s, p, wd)), 8 columns of one row per piece
-  const bool vec = (a.K % 8) == 0;
-  for (int i = tid; i < kTile * (kTile / 8); i += kMergeThreads) {
-    const int row = i >> 4, pc = i & 15;
-    const int64_t n = n0 + row;
-    const int64_t k = k0 + pc * 8;
-    if (n >= a.N || k >= a.K) continue;
-    const float* pr = p_s + row * kPStride + pc * 8;
-    if (vec) {
-      // K % 8 == 0: the 8 weights share one packed word and one block
-      const int64_t e0 = n * a.K + k;
-      const uint32_t w = __ldcs(reinterpret_cast<const unsigned int*>(a.packed + (e0 >> 1)));
-      const float s1 = block_scale(a.double_quant, a.c1, a.c2, e0 >> 6);
+  if (vec) {
+    // K % 8 == 0: the 8 weights of a piece share one packed word and one block
+#pragma unroll
+    for (int j = 0; j < kPieces; ++j) {
+      const int row = (tid >> 4) + 16 * j;
+      const int64_t n = n0 + row;
+      const int64_t k = k0 + pc * 8;
+      if (n >= a.N || k >= a.K) continue;
+      const float* pr = p_s + row * kPStride + pc * 8;
+      const uint32_t w = pw[j];
       uint32_t o[4];
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
-        const float wd0 = round_to(F16, code_s[(w >> (8 * h)) & 0xFu] * s1);
-        const float wd1 = round_to(F16, code_s[(w >> (8 * h + 4)) & 0xFu] * s1);
+        const float wd0 = round_to(F16, code_s[(w >> (8 * h)) & 0xFu] * ps[j]);
+        const float wd1 = round_to(F16, code_s[(w >> (8 * h + 4)) & 0xFu] * ps[j]);
         o[h] = pack2(F16, fmaf(a.s, pr[2 * h], wd0), fmaf(a.s, pr[2 * h + 1], wd1));
       }
-      __stcs(reinterpret_cast<uint4*>(a.out + e0), make_uint4(o[0], o[1], o[2], o[3]));
-    } else {
+      __stcs(reinterpret_cast<uint4*>(a.out + n * a.K + k), make_uint4(o[0], o[1], o[2], o[3]));
+    }
+  } else {
+    for (int i = tid; i < kTile * (kTile / 8); i += kMergeThreads) {
+      const int row = i >> 4, pcc = i & 15;
+      const int64_t n = n0 + row;
+      const int64_t k = k0 + pcc * 8;
+      if (n >= a.N || k >= a.K) continue;
+      const float* pr = p_s + row * kPStride + pcc * 8;
       for (int q = 0; q < 8 && k + q < a.K; ++q) {
         const int64_t e = n * a.K + k + q;
         const uint32_t byte = a.packed[e >> 1];

@@ -86,24 +86,47 @@ __device__ __forceinline__ uint32_t classify_fast(uint32_t cells_biased, float x
   return base + (__float_as_uint(__uint_as_float(t) - x16) >> 31);
 }
 
+// Code decision with an exact comparison, for tables whose thresholds are
+// dyadic (the uniform INT4 table: odd sixteenths).  There w / scale1 can hit a
+// threshold exactly, and w * fp32(1/scale1) can then land on either side of
+// it; the cell is still taken from the rounded x16 (a neighbouring cell gives
+// the same code there), but the comparison w > T scale1 is made exactly: the
+// fma forms 16 w - 16T scale1 with the exact product and one rounding, which
+// keeps the sign.  c1 is the block absmax (after the same scaling as w).
+__device__ __forceinline__ uint32_t classify_exact(const uint2* cells, float x16, float w, float c1) {
+  const uint32_t idx = min(uint32_t(__float2int_rd(x16) + 16), uint32_t(kCells - 1));
+  const uint2 e = cells[idx];
+  return e.y + (fmaf(-__uint_as_float(e.x), c1, w * 16.0f) > 0.0f ? 1u : 0u);
+}
+
 // 8 consecutive bf16 (one uint4) -> 8 nibbles (element 0 in bits 0-3);
 // inv16 = 16 / scale1 (of the weights first scaled by pre, a power of two,
-// on the careful path for extreme or non-finite blocks).
-template <bool FAST>
+// on the careful path for extreme or non-finite blocks); c1 = scale1 * pre.
+// MODE 0: fast cells (NF4 blocks with a normal scale1); 1: clamped cells (any
+// input); 2: exact comparison (dyadic thresholds).
+template <int MODE>
 __device__ __forceinline__ uint32_t quantize8(const uint2* cells, uint32_t cells_biased, const uint4& v,
-                                              float inv16, float pre) {
+                                              float inv16, float pre, float c1) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   uint32_t out = 0;
 #pragma unroll
   for (int j = 3; j >= 0; --j) {
     float hi = bf16hi_to_f32(w[j]), lo = bf16lo_to_f32(w[j]);
-    if (!FAST) {
+    if (MODE != 0) {
       hi *= pre;
       lo *= pre;
     }
     const float xh = hi * inv16, xl = lo * inv16;
-    out = out * 16u + (FAST ? classify_fast(cells_biased, xh) : classify16(cells, xh));
-    out = out * 16u + (FAST ? classify_fast(cells_biased, xl) : classify16(cells, xl));
+    if (MODE == 0) {
+      out = out * 16u + classify_fast(cells_biased, xh);
+      out = out * 16u + classify_fast(cells_biased, xl);
+    } else if (MODE == 1) {
+      out = out * 16u + classify16(cells, xh);
+      out = out * 16u + classify16(cells, xl);
+    } else {
+      out = out * 16u + classify_exact(cells, xh, hi, c1);
+      out = out * 16u + classify_exact(cells, xl, lo, c1);
+    }
   }
   return out;
 }
@@ -129,6 +152,7 @@ struct QuantArgs {
   uint32_t* status;
   int64_t ngroups;
   int dq;              // DqFormat
+  int exact;           // exact comparisons (tables with dyadic thresholds)
   uint32_t zero8;      // eight nibbles of the table's 0.0 code (all-zero blocks)
   float thr[15];
 };
@@ -219,13 +243,17 @@ __global__ void __launch_bounds__(kQuantThreads, 2) nf4_quantize_kernel(const __
       uint32_t q8;
       if (c1 == 0.0f) {
         q8 = p.zero8;                            // all-zero block: the 0.0 code
+      } else if (p.exact) {                      // dyadic thresholds: exact comparisons
+        const bool nrm = c1 >= 0x1p-122f && c1 <= 0x1p125f;
+        const float pre = nrm ? 1.0f : ((c1 < 1.0f) ? 0x1p64f : 0x1p-64f);
+        q8 = quantize8<2>(cells, cells_biased, v[i], __frcp_rn(c1 * pre) * 16.0f, pre, c1 * pre);
       } else if (fast) {
-        q8 = quantize8<true>(cells, cells_biased, v[i], inv * 16.0f, 1.0f);
+        q8 = quantize8<0>(cells, cells_biased, v[i], inv * 16.0f, 1.0f, c1);
       } else if (c1 >= 0x1p-122f && c1 <= 0x1p125f) {
-        q8 = quantize8<false>(cells, cells_biased, v[i], __frcp_rn(c1) * 16.0f, 1.0f);
+        q8 = quantize8<1>(cells, cells_biased, v[i], __frcp_rn(c1) * 16.0f, 1.0f, c1);
       } else {                                   // keep 16/c1 a normal number
         const float pre = (c1 < 1.0f) ? 0x1p64f : 0x1p-64f;
-        q8 = quantize8<false>(cells, cells_biased, v[i], __frcp_rn(c1 * pre) * 16.0f, pre);
+        q8 = quantize8<1>(cells, cells_biased, v[i], __frcp_rn(c1 * pre) * 16.0f, pre, c1);
       }
       uint8_t* dst = p.packed + (e0 >> 1);
       if (e0 + 8 <= p.numel) {
@@ -351,6 +379,7 @@ cudaError_t launch_quantize(const uint16_t* W, int64_t numel, int quant_type, in
   a.ngroups = ngroups_of(numel);
   a.dq = dq;
   a.zero8 = 0x11111111u * uint32_t(zero_code(quant_type));
+  a.exact = quant_type == kQuantInt4 ? 1 : 0;
   const Codebook& cb = host_codebook(quant_type);
   for (int i = 0; i < 15; ++i) a.thr[i] = cb.thr[i];
   int64_t grid = a.ngroups;

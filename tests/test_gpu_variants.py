@@ -86,10 +86,15 @@ def _merge_check(got, Wd, A, B, s, dtype):
         u = 2.0 ** -23                                   # twice the fp32 unit roundoff
         bound = abs(s) * r * u * absp + u * (np.abs(s) * absp + np.abs(exact))
         mid = (g[bad] + rv[bad]) / 2
-        assert np.all(np.abs(exact[bad] - mid) <= bound[bad]), "mismatch away from a rounding midpoint"
+        far = np.abs(exact[bad] - mid) > bound[bad]
         gb, rb = got[bad].astype(np.int64), ref[bad].astype(np.int64)
         same_sign = (gb >> 15) == (rb >> 15)
-        assert np.all(np.abs(gb - rb)[same_sign] == 1), "not a neighbouring value"
+        apart = same_sign & (np.abs(gb - rb) != 1)
+        idx = np.argwhere(bad)
+        worst = [(tuple(idx[i]), int(gb[i]), int(rb[i]), float(exact[bad][i]), float(bound[bad][i]))
+                 for i in np.nonzero(far | apart)[0][:8]]
+        assert not far.any(), f"mismatch away from a rounding midpoint: {worst}"
+        assert not apart.any(), f"not a neighbouring value: {worst}"
         assert np.all(np.abs(g[bad][~same_sign]) <= 2.0 ** -14), "sign differs away from zero"
     assert bad.mean() < 1e-3, bad.mean()
     return int(bad.sum())
