@@ -65,6 +65,7 @@ SIGNATURES = {
     "qlora_linear_fwd_noalloc": (ctypes.c_int, [_P, _I64, NF4Weight, _P, _P, _I32, _F, _P, _P, _P]),
     "qlora_linear_fwd_noalloc_info": (ctypes.c_int, [_P, _P]),
     "qlora_linear_plan": (ctypes.c_int, [_I64, _I64, _I64, _I32, _I32, _I32, _P]),
+    "nf4_wait_selftest": (ctypes.c_int, [_P, _I64, _P]),
     "nf4_status_str": (ctypes.c_char_p, [ctypes.c_int]),
 }
 
@@ -241,6 +242,12 @@ class _DeviceWord:
     def __init__(self, ptr):
         self.__cuda_array_interface__ = {"shape": (1,), "typestr": "<i4", "data": (int(ptr), False),
                                          "version": 3}
+
+
+def wait_selftest(status: torch.Tensor, limit_cycles: int):
+    """Run the bounded device wait on a barrier nothing arrives at (see
+    nf4_wait_selftest); status: int32 CUDA tensor of one element."""
+    _check(lib().nf4_wait_selftest(_dev(status, torch.int32, "status"), int(limit_cycles), _stream()))
 
 
 def noalloc_info():

@@ -94,7 +94,8 @@ NF4_DEV bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_n
 // (at most ~20 us), and the cycle counter is read every 16 polls, so waiting
 // costs almost no issue slots and the bound stays coarse but finite.
 constexpr long long kWaitLimitCycles = 4000000000ll;
-NF4_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err, volatile int* abort_flag) {
+NF4_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err, volatile int* abort_flag,
+                       long long limit_cycles = kWaitLimitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   long long t0 = -1;
   uint32_t spins = 0;
@@ -105,7 +106,7 @@ NF4_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err, volatile i
       const long long now = clock64();
       if (t0 < 0) {
         t0 = now;
-      } else if (now - t0 > kWaitLimitCycles) {
+      } else if (now - t0 > limit_cycles) {
         if (err) atomicOr(err, kStatusTimeout);
         if (abort_flag) *abort_flag = 1;
         return false;

@@ -131,34 +131,46 @@ __global__ void __launch_bounds__(kMergeThreads) nf4_merge_kernel(const __grid_c
       if (i < kTile * jc) *reinterpret_cast<uint4*>(a_s + (i / jc) * srow + (i % jc) * 16) = v[u];
     }
   }
+  // B's slice goes in transposed: thread (c, jp) loads 8 columns of rows 2jp
+  // and 2jp + 1 and writes them as 32-bit pairs down the rows of B^T, so the
+  // lanes of a warp write neighbouring words of one B^T row (no bank conflicts)
   constexpr int nc = kTile / 8;                  // 8-wide chunks of a row of B's slice
-  for (int i0 = tid; i0 < rp * nc; i0 += 4 * kMergeThreads) {     // B[j][n0 + 8c ..] -> B^T rows
-    uint4 v[4];
+  const int jp_n = rp / 2;
+  for (int i0 = tid; i0 < nc * jp_n; i0 += 2 * kMergeThreads) {
+    uint4 v[2][2];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < 2; ++u) {
       const int i = i0 + u * kMergeThreads;
-      v[u] = make_uint4(0u, 0u, 0u, 0u);
-      const int j = i / nc, c = i % nc;
-      if (i >= rp * nc || j >= a.r) continue;
-      const int64_t nb = n0 + c * 8;
-      const uint16_t* src = a.B + int64_t(j) * a.N + nb;
-      if (nb + 8 <= a.N && (a.N % 8) == 0) {
-        v[u] = __ldg(reinterpret_cast<const uint4*>(src));
-      } else {
-        uint32_t t[4] = {0u, 0u, 0u, 0u};
-        for (int q = 0; q < 8; ++q)
-          if (nb + q < a.N) t[q >> 1] |= uint32_t(src[q]) << (16 * (q & 1));
-        v[u] = make_uint4(t[0], t[1], t[2], t[3]);
+      const int c = i / jp_n, jp = i % jp_n;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int j = 2 * jp + h;
+        v[u][h] = make_uint4(0u, 0u, 0u, 0u);
+        if (i >= nc * jp_n || j >= a.r) continue;
+        const int64_t nb = n0 + c * 8;
+        const uint16_t* src = a.B + int64_t(j) * a.N + nb;
+        if (nb + 8 <= a.N && (a.N % 8) == 0) {
+          v[u][h] = __ldg(reinterpret_cast<const uint4*>(src));
+        } else {
+          uint32_t t[4] = {0u, 0u, 0u, 0u};
+          for (int q = 0; q < 8; ++q)
+            if (nb + q < a.N) t[q >> 1] |= uint32_t(src[q]) << (16 * (q & 1));
+          v[u][h] = make_uint4(t[0], t[1], t[2], t[3]);
+        }
       }
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < 2; ++u) {
       const int i = i0 + u * kMergeThreads;
-      if (i >= rp * nc) continue;
-      const int j = i / nc, c = i % nc;
-      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-      for (int q = 0; q < 8; ++q)
-        *reinterpret_cast<uint16_t*>(bt_s + (c * 8 + q) * srow + j * 2) = uint16_t(w[q >> 1] >> (16 * (q & 1)));
+      if (i >= nc * jp_n) continue;
+      const int c = i / jp_n, jp = i % jp_n;
+      const uint32_t w0[4] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w};
+      const uint32_t w1[4] = {v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const uint32_t lo = (w0[q >> 1] >> (16 * (q & 1))) & 0xFFFFu, hi = (w1[q >> 1] >> (16 * (q & 1))) & 0xFFFFu;
+        *reinterpret_cast<uint32_t*>(bt_s + (c * 8 + q) * srow + jp * 4) = lo | (hi << 16);
+      }
     }
   }
   __syncthreads();

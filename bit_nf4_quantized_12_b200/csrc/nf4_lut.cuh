@@ -39,7 +39,10 @@ __device__ __forceinline__ BlockTable make_table(const CodeTable& code, float s1
 __device__ __forceinline__ void lookup4(const BlockTable& t, uint32_t s, uint32_t& o01, uint32_t& o23) {
   const uint32_t sel_a = s;                   // entries 0-7 (bit 3 clear)
   const uint32_t sel_b = s ^ 0x8888u;         // entries 8-15
-  const uint32_t sel2 = ((s >> 1) & 0x4444u) | 0x3210u;   // pick a or b per byte by bit 3
+  // pick a or b per byte by bit 3: ((s & 0x8888) >> 1) | 0x3210, the shift
+  // and the OR (no bits in common) as one high multiply-add on the FMA pipe,
+  // leaving the integer pipe to the byte permutes
+  const uint32_t sel2 = __umulhi(s & 0x8888u, 0x80000000u) + 0x3210u;
   const uint32_t lo = prmt(prmt(t.lo[0], t.lo[1], sel_a), prmt(t.lo[2], t.lo[3], sel_b), sel2);
   const uint32_t hi = prmt(prmt(t.hi[0], t.hi[1], sel_a), prmt(t.hi[2], t.hi[3], sel_b), sel2);
   o01 = prmt(lo, hi, 0x5140);

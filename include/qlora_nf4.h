@@ -282,6 +282,15 @@ typedef struct {
 nf4_status qlora_linear_plan(int64_t M, int64_t N, int64_t K, int32_t r, int32_t backward, int32_t num_sms,
                              qlora_plan* out);
 
+/* Self-test of the bounded device wait every kernel of this library uses
+ * (no counterpart in the pages).  Launches one thread on `stream` that waits
+ * on a shared-memory barrier nothing arrives at, giving up after about
+ * limit_cycles SM cycles (1 .. 2^40; the kernels use ~4e9, about 2 s): it
+ * then ORs bit 1 (timeout) into *d_status (a device int32 the caller zeroed)
+ * and returns, and the stream continues normally.  A lost arrival in any
+ * kernel ends the same way: a status bit, never a hang. */
+nf4_status nf4_wait_selftest(int32_t* d_status, int64_t limit_cycles, void* stream);
+
 /* Human-readable name of a status code (static string). */
 const char* nf4_status_str(nf4_status status);
 

@@ -5,10 +5,10 @@ LoRA merge against the oracle.
     packed codes, 8-bit codes or FP32 scale1, FP32 scale2;
   - dequantize: bit-exact into bf16 and into fp16 ("QLoRA 原理精讲" §三 误区4);
   - LoRA merge ("QLoRA 原理精讲" §2.5, §三 误区3): bit-exact except where the
-    exact merged value lies so close to a rounding midpoint that the kernel's
-    fp32 accumulation of the rank-r product (and its fp32 sum) may round the
-    other way; there the result may be the neighbouring value, and such
-    elements must be rare;
+    kernel's fp32 arithmetic (accumulation of the rank-r product, the fused
+    add) may round the other way: near rounding ties, or where the merged
+    value cancels to far below its inputs; every such element must lie within
+    that arithmetic's error bound of the exact value, and they must be rare;
   - the QLoRA linear layer in FP16, and in bf16 on the variant formats,
     within the build's GEMM tolerance (relative Frobenius 2e-3, elementwise
     1e-2 with the denominator floored at 1e-2 x rms)."""
@@ -74,28 +74,40 @@ def test_int4_zero_and_extreme_blocks():
 
 
 # ------------------------------------------------------------------ LoRA merge
+def _ulp(v, dtype):
+    """Spacing of the compute type at each value (bf16: 8 significant bits,
+    fp16: 11; subnormal spacing below the smallest normal)."""
+    a = np.abs(v)
+    if dtype == oracle.F16:
+        e = np.floor(np.log2(np.maximum(a, 2.0 ** -14)))
+        return 2.0 ** (e - 10)
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -126)))
+    return 2.0 ** (e - 7)
+
+
 def _merge_check(got, Wd, A, B, s, dtype):
-    """got: uint16 bits [N,K]; Wd, A, B: oracle-side bits."""
+    """got: uint16 bits [N,K]; Wd, A, B: oracle-side bits.  Every element
+    that differs from the oracle's correctly rounded value must lie within
+    the kernel's arithmetic error of the exact value: the fp32 accumulation
+    of the r products (at most r units of 2^-23 relative to sum |a b|, twice
+    the fp32 unit roundoff per step, scaled by |s|), the fp32 rounding of the
+    sum, and half a step of the compute type at the result.  Such elements
+    (near-ties, and values that cancel to far below their inputs) must be
+    rare."""
     ref, exact = oracle.lora_merge(Wd, A, B, s, dtype)
     dec = oracle.f16_to_f64 if dtype == oracle.F16 else oracle.bf16_to_f64
-    g, rv = dec(got), dec(ref)
     bad = got != ref
     if bad.any():
         r = A.shape[1]
-        absp = (np.abs(dec(A)) @ np.abs(dec(B))).T
-        u = 2.0 ** -23                                   # twice the fp32 unit roundoff
-        bound = abs(s) * r * u * absp + u * (np.abs(s) * absp + np.abs(exact))
-        mid = (g[bad] + rv[bad]) / 2
-        far = np.abs(exact[bad] - mid) > bound[bad]
-        gb, rb = got[bad].astype(np.int64), ref[bad].astype(np.int64)
-        same_sign = (gb >> 15) == (rb >> 15)
-        apart = same_sign & (np.abs(gb - rb) != 1)
+        g = dec(got[bad])
+        absp = (np.abs(dec(A)) @ np.abs(dec(B))).T[bad]
+        u = 2.0 ** -23
+        bound = abs(s) * r * u * absp + u * (abs(s) * absp + np.abs(exact[bad])) + 0.5 * _ulp(g, dtype) * (1 + 1e-6)
+        far = np.abs(g - exact[bad]) > bound
         idx = np.argwhere(bad)
-        worst = [(tuple(idx[i]), int(gb[i]), int(rb[i]), float(exact[bad][i]), float(bound[bad][i]))
-                 for i in np.nonzero(far | apart)[0][:8]]
-        assert not far.any(), f"mismatch away from a rounding midpoint: {worst}"
-        assert not apart.any(), f"not a neighbouring value: {worst}"
-        assert np.all(np.abs(g[bad][~same_sign]) <= 2.0 ** -14), "sign differs away from zero"
+        worst = [(tuple(idx[i]), int(got[bad][i]), int(ref[bad][i]), float(exact[bad][i]), float(bound[i]))
+                 for i in np.nonzero(far)[0][:8]]
+        assert not far.any(), f"outside the arithmetic's error bound: {worst}"
     assert bad.mean() < 1e-3, bad.mean()
     return int(bad.sum())
 
