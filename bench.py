@@ -22,6 +22,9 @@ flush before each call), medians:
                        fwd+bwd TFLOP/s at 512 tokens on the 7 layer shapes
   robust               4095x11007 at 4096 tokens, r=8: quantize, dequantize,
                        fwd, bwd
+  merge                LoRA merge (r=64) of the 7 weights, GB/s
+  f16                  the FP16 compute type: fwd+bwd on q, gate, down
+  variants             quantize / dequantize GB/s of the storage variants
 N > 1 runs data-parallel replicas (weak scaling: 2048 tokens per rank); the
 step's one exchange is an NCCL all-reduce of every matrix's dA and dB, held
 in one flat bucket.
@@ -378,6 +381,60 @@ def llama70b_component(device, peaks, layers=80, reps=20):
     return res
 
 
+def f16_component(device, peaks, reps=10):
+    """The FP16 compute type: qlora_linear fwd+bwd on three 7B-shaped weights
+    (q 4096x4096, gate 11008x4096, down 4096x11008) at 2048 tokens, r=64, with
+    X, A, B, dY in fp16; each call timed alone, L2 flushed before it."""
+    from bit_nf4_quantized_12_b200 import binding
+    wl = workloads.WORKLOADS["llama7b"]
+    M, r, s_ = wl.tokens, wl.r, wl.s
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device).zero_
+    fl = ms = 0.0
+    per = {}
+    for idx in (0, 4, 6):
+        name, N, K = wl.mats[idx]
+        seed = workloads.matrix_seed("llama7b", 0, idx)
+        qw = binding.quantize(workloads.weight(N, K, wl.w_std, seed=seed, device=device))
+        io = {k: v.to(torch.float16) for k, v in workloads.layer_inputs(M, N, K, r, seed=seed, device=device).items()}
+        ws = binding.workspace(M, N, K, r, device)
+        Y = torch.empty(M, N, dtype=torch.float16, device=device)
+        T = torch.empty(M, r, dtype=torch.float16, device=device)
+        f = _median_ms(lambda: binding.linear_fwd(io["X"], qw, io["A"], io["B"], s_, ws=ws, Y=Y, T=T), reps, flush)
+        b = _median_ms(lambda: binding.linear_bwd(io["dY"], io["X"], qw, io["A"], io["B"], s_, T=T, ws=ws), reps, flush)
+        w = fwd_flops(M, N, K, r) + bwd_flops(M, N, K, r)
+        per[f"{name} {N}x{K}"] = round(w / ((f + b) * 1e-3) / 1e12, 1)
+        fl += w
+        ms += f + b
+    t = fl / (ms * 1e-3) / 1e12
+    return {"fwd+bwd": {"TFLOP/s": t, "frac": t / peaks["bf16_tflops_sustained"]}, "per_matrix_TFLOP/s": per,
+            "peak_note": "fp16 and bf16 share one dense tensor-core rate; the bf16 measured peak is used"}
+
+
+def variants_component(device, peaks, reps=20):
+    """Quantize and dequantize of the 11008x4096 weight in each storage
+    format variant (uniform INT4 table; FP32 scale1; uint8 scale1), each call
+    timed alone with L2 flushed before it."""
+    from bit_nf4_quantized_12_b200 import binding
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device).zero_
+    N, K = 11008, 4096
+    W = workloads.weight(N, K, 0.02, seed=4, device=device)
+    Wd = torch.empty_like(W)
+    res = {}
+    for qt, dq, name in ((binding.QUANT_NF4, binding.DQ_E4M3, "nf4+fp8/fp32 (the method)"),
+                         (binding.QUANT_INT4, binding.DQ_E4M3, "int4+fp8/fp32"),
+                         (binding.QUANT_NF4, binding.DQ_NONE, "nf4+fp32 scale1"),
+                         (binding.QUANT_NF4, binding.DQ_U8, "nf4+uint8/fp32")):
+        qw = binding.empty_quantized(N, K, device, qt, dq)
+        q = _median_ms(lambda: binding.quantize(W, out=qw), reps, flush)
+        d = _median_ms(lambda: binding.dequant(qw, out=Wd), reps, flush)
+        nbytes = 2 * N * K + qw.packed.numel() + qw.c1q.numel() * qw.c1q.element_size() + 4 * qw.c2.numel()
+        res[name] = {"quantize_GB/s": round(nbytes / (q * 1e-3) / 1e9, 1),
+                     "dequant_GB/s": round(nbytes / (d * 1e-3) / 1e9, 1),
+                     "quantize_frac": round(nbytes / (q * 1e-3) / 1e9 / peaks["hbm_gbs"], 3),
+                     "dequant_frac": round(nbytes / (d * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)}
+    return res
+
+
 def robust_component(device, peaks, reps=5):
     """The robustness configuration: W 4095x11007 (ragged final block and
     group; Student-t(3) with 0.1% outliers x20), qlora_linear fwd+bwd at 4096
@@ -686,6 +743,9 @@ def main():
         comp["llama70b"] = llama70b_component(device, peaks)
         torch.cuda.empty_cache()
         comp["robust"] = robust_component(device, peaks)
+        torch.cuda.empty_cache()
+        comp["f16"] = f16_component(device, peaks)
+        comp["variants"] = variants_component(device, peaks)
 
     cpu = None
     if rank == 0 and world == 1:
