@@ -102,6 +102,28 @@ constexpr int SX = 4, SP = 8, SA = 4;
 // wait would pass on the wrong phase.
 static_assert(SP % kDequantWGs == 0 && SA % kDequantWGs == 0, "ring slots must map to one dequant warpgroup");
 
+// Forward main steps keep the dequantized weight operand in tensor memory:
+// the dequant warps store it with tcgen05.st (thread t = row t = lane t, the
+// 64 weights of its row segment as 32 columns of bf16x2) and the MMA reads A
+// from there.  That takes the operand's 16 KB store and 16 KB read per step
+// off shared memory, whose bandwidth the activation tile, the TMA fills and
+// the operand otherwise share.  The ring of SA slots sits after the
+// accumulator's columns.
+// In tensor memory the ring can also be deeper than the shared-memory one:
+// SAT = 8 slots of 32 columns fit beside a 256-column accumulator, so the
+// dequant warpgroups run up to 8 steps ahead of the tensor core, which hides
+// the latency of one warpgroup's step (each warpgroup owns every fourth step).
+// The forward's low-rank steps (A = a tile of B^T, by TMA) keep the
+// shared-memory ring.
+constexpr bool kTmemA = true;
+constexpr int SAT = 8;
+static_assert(SAT % kDequantWGs == 0, "tensor-memory ring slots must map to one dequant warpgroup");
+__host__ __device__ constexpr uint32_t acc_cols_of(int bt) { return uint32_t(bt < 32 ? 32 : bt); }
+__host__ __device__ constexpr uint32_t tmem_cols_of(bool bwd, int bt) {
+  // accumulator [+ operand ring], rounded up to a power of two (>= 32)
+  return (bwd || !kTmemA) ? acc_cols_of(bt) : (acc_cols_of(bt) + SAT * 32 <= 256 ? 256u : 512u);
+}
+
 // Ragged mode reuses the idle packed ring: 48 bytes of load slot per dequant
 // thread, then the 64 x 16 lane-mask table of the two-table dequantization.
 constexpr uint32_t kRaggedMaskOffset = 128 * kDequantWGs * 48;
@@ -183,7 +205,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
   uint64_t* a_full = p_empty + SP;
   uint64_t* a_empty = a_full + SA;
   uint64_t* accf = a_empty + SA;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  uint64_t* t_full = accf + 1;             // tensor-memory operand ring (forward main steps)
+  uint64_t* t_empty = t_full + SAT;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(t_empty + SAT);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -197,7 +221,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
   const int64_t my_main = g_end > g_begin ? g_end - g_begin : 0;
   const int my_lora = (split == 0) ? P.lora_steps : 0;
   const int64_t nsteps = my_main + my_lora;
-  const uint32_t tmem_cols = uint32_t(bt < 32 ? 32 : bt);
+  const uint32_t tmem_cols = tmem_cols_of(BWD, bt);
+  const uint32_t a_tmem_col = acc_cols_of(bt);   // forward: operand ring column base
 
   if (threadIdx.x == 32) {   // descriptor fetches overlap the setup below
     tma_prefetch_desc(&P.tm_act);
@@ -209,6 +234,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
     for (int s = 0; s < SX; ++s) { mbar_init(&x_full[s], 1); mbar_init(&x_empty[s], 1); }
     for (int s = 0; s < SP; ++s) { mbar_init(&p_full[s], 1); mbar_init(&p_empty[s], 4); }
     for (int s = 0; s < SA; ++s) { mbar_init(&a_full[s], 4); mbar_init(&a_empty[s], 1); }
+    for (int s = 0; s < SAT; ++s) { mbar_init(&t_full[s], 4); mbar_init(&t_empty[s], 1); }
     mbar_init(accf, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -292,9 +318,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
     const uint32_t idesc_k = make_idesc(128, bt, 0, 0, a.f16 != 0);
     const uint32_t idesc_mn = make_idesc(128, bt, 1, 0, a.f16 != 0);
     for (int64_t ks = 0; ks < nsteps; ++ks) {
-      const int sx = int(ks % SX), sa = int(ks % SA);
+      const int sx = int(ks % SX);
+      // operand slot: forward main steps in the tensor-memory ring, every
+      // other step in the shared-memory ring (the forward's low-rank steps
+      // counted from the first of them)
+      const bool a_in_tmem = !BWD && kTmemA && ks < my_main;
+      const int64_t ls = (!BWD && kTmemA) ? ks - my_main : ks;
+      const int sa = a_in_tmem ? int(ks % SAT) : int(ls % SA);
+      const uint32_t aph = a_in_tmem ? uint32_t(ks / SAT) & 1u : uint32_t(ls / SA) & 1u;
       if (!mbar_wait(&x_full[sx], uint32_t(ks / SX) & 1u, a.status, abort_flag)) break;
-      if (!mbar_wait(&a_full[sa], uint32_t(ks / SA) & 1u, a.status, abort_flag)) break;
+      if (!mbar_wait(a_in_tmem ? &t_full[sa] : &a_full[sa], aph, a.status, abort_flag)) break;
       tc_fence_after();
       if (elect_one()) {
         const uint32_t act_addr = smem_u32(act_s + sx * act_bytes);
@@ -304,12 +337,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t bdesc = make_sdesc_sw128(act_addr + kk * 32, 16, 1024);
-          const uint64_t adesc = a_mn ? make_sdesc_sw128(a_addr + kk * 2048, 8192, 1024)
-                                      : make_sdesc_sw128(a_addr + kk * 32, 16, 1024);
-          mma_ss(tmem_base, adesc, bdesc, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+          if (a_in_tmem) {   // 16 K-elements = 8 columns per MMA
+            mma_ts(tmem_base, tmem_base + a_tmem_col + uint32_t(sa) * 32u + uint32_t(kk) * 8u, bdesc, idesc,
+                   (ks > 0 || kk > 0) ? 1u : 0u);
+          } else {
+            const uint64_t adesc = a_mn ? make_sdesc_sw128(a_addr + kk * 2048, 8192, 1024)
+                                        : make_sdesc_sw128(a_addr + kk * 32, 16, 1024);
+            mma_ss(tmem_base, adesc, bdesc, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         mma_commit(&x_empty[sx]);
-        mma_commit(&a_empty[sa]);
+        mma_commit(a_in_tmem ? &t_empty[sa] : &a_empty[sa]);
       }
       __syncwarp();
     }
@@ -359,8 +397,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
       for (int j = 0; j < 4; ++j) {
         const int64_t ks = base + int64_t(j) * kDequantWGs;
         if (!ok || ks >= nsteps) break;
-        const int sa = int(ks % SA);
-        const uint32_t a_ph = uint32_t(ks / SA) & 1u;
+        const int64_t ls = (!BWD && kTmemA) ? ks - my_main : ks;   // shared-ring step index
+        const int sa = int(ls % SA);
+        const uint32_t a_ph = uint32_t(ls / SA) & 1u;
         if (ks < my_main) {
           uint32_t o[32];
           if (!RAGGED) {
@@ -384,6 +423,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
             dequant64_two(make_table(P.code, scale_from_parts(a.dq, cq[j], cc[j]), f16),
                           make_table(P.code, scale_from_parts(a.dq, cq2[j], cc2[j]), f16), wv, masks, o);
           }
+          if (!BWD && kTmemA) {
+            // forward: row t of Wd into tensor memory, lane t (this warp's
+            // quarter), the slot's 32 columns, once the MMA of step ks - SAT
+            // has released the slot (the fence orders its reads first)
+            const int ts = int(ks % SAT);
+            if (ks >= SAT && !(ok = mbar_wait(&t_empty[ts], (uint32_t(ks / SAT) & 1u) ^ 1u, a.status, abort_flag)))
+              break;
+            tc_fence_after();
+            tmem_st_32x32b_x32(tmem_base + (uint32_t((warp & 3) * 32) << 16) + a_tmem_col + uint32_t(ts) * 32u, o);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&t_full[ts]);
+            continue;
+          }
           // the A slot must have been released by the MMA of step ks - SA
           if (ks >= SA && !(ok = mbar_wait(&a_empty[sa], a_ph ^ 1u, a.status, abort_flag))) break;
           // forward: row t of Wd (K-major, 128-byte rows); backward: row
@@ -401,7 +454,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
           // low-rank step: the A operand is a tile of a LoRA factor, by TMA
           // (forward: B^T [128 features x 64 ranks], two MN-major boxes;
           //  backward: A [128 inputs x 64 ranks], one K-major box)
-          if (ks >= SA && !(ok = mbar_wait(&a_empty[sa], a_ph ^ 1u, a.status, abort_flag))) break;
+          if (ls >= SA && !(ok = mbar_wait(&a_empty[sa], a_ph ^ 1u, a.status, abort_flag))) break;
           __syncwarp();
           if (lane == 0) {
             if ((warp & 3) == 0) {

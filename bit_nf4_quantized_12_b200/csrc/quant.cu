@@ -183,7 +183,7 @@ __device__ __forceinline__ void load_group(const QuantArgs& p, int64_t g, uint4 
 __global__ void __launch_bounds__(kQuantThreads, 2) nf4_quantize_kernel(const __grid_constant__ QuantArgs p) {
   __shared__ uint2 cells[kCells];
   __shared__ float thr_s[16];
-  __shared__ uint32_t warp_max[2][kQuantThreads / 32];
+  __shared__ __align__(16) uint32_t warp_max[2][kQuantThreads / 32];
   if (threadIdx.x < 15) thr_s[threadIdx.x] = p.thr[threadIdx.x];
   __syncthreads();
   build_cells(cells, thr_s);
@@ -234,11 +234,13 @@ __global__ void __launch_bounds__(kQuantThreads, 2) nf4_quantize_kernel(const __
     const bool normal = (my_c1 >= 0x1p-122f && my_c1 <= 0x1p125f) || my_c1 == 0.0f;
     const float my_inv = (my_c1 == 0.0f) ? 0.0f : (normal ? __frcp_rn(my_c1) : 0.0f);
     const bool fast = __all_sync(0xffffffffu, normal);
+    const int64_t ebase = gbase + tid * 8;
+    const bool full = gbase + kGroupElems <= p.numel;   // no element of this group is past the end
 #pragma unroll
     for (int i = 0; i < kQuantIters; ++i) {
-      const int64_t e0 = gbase + int64_t(i) * (kQuantThreads * 8) + tid * 8;
+      const int64_t e0 = ebase + i * (kQuantThreads * 8);
       const float inv = __shfl_sync(0xffffffffu, my_inv, (lane & ~7) | i);
-      if (e0 >= p.numel) continue;
+      if (!full && e0 >= p.numel) continue;
       const float c1 = __uint_as_float(bm[i] << 16);
       uint32_t q8;
       if (c1 == 0.0f) {
@@ -256,7 +258,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) nf4_quantize_kernel(const __
         q8 = quantize8<1>(cells, cells_biased, v[i], __frcp_rn(c1 * pre) * 16.0f, pre, c1);
       }
       uint8_t* dst = p.packed + (e0 >> 1);
-      if (e0 + 8 <= p.numel) {
+      if (full || e0 + 8 <= p.numel) {
         __stcs(reinterpret_cast<unsigned int*>(dst), q8);
       } else {
         const int valid = int(p.numel - e0);
@@ -275,9 +277,15 @@ __global__ void __launch_bounds__(kQuantThreads, 2) nf4_quantize_kernel(const __
     // then the 8-bit codes of scale1 / scale2 (lane j < kQuantIters of each
     // block group stores its block's)
     __syncthreads();
-    gm = warp_max[parity][0];
+    {   // the group maximum over the warps' maxima, four per 16-byte load
+      const uint4* wm = reinterpret_cast<const uint4*>(warp_max[parity]);
+      gm = 0;
 #pragma unroll
-    for (int w = 1; w < kQuantThreads / 32; ++w) gm = max(gm, warp_max[parity][w]);
+      for (int w = 0; w < kQuantThreads / 128; ++w) {
+        const uint4 q = wm[w];
+        gm = max(gm, max(max(q.x, q.y), max(q.z, q.w)));
+      }
+    }
     if (gm >= 0x7F80u) bad = 1;
     const float gmax = __uint_as_float(gm << 16);
     const float s2 = __fdiv_rn(gmax, p.dq == kDqU8 ? 255.0f : 448.0f);
