@@ -109,14 +109,13 @@ static_assert(SP % kDequantWGs == 0 && SA % kDequantWGs == 0, "ring slots must m
 // off shared memory, whose bandwidth the activation tile, the TMA fills and
 // the operand otherwise share.  The ring of SA slots sits after the
 // accumulator's columns.
-// In tensor memory the ring can also be deeper than the shared-memory one:
-// SAT = 8 slots of 32 columns fit beside a 256-column accumulator, so the
-// dequant warpgroups run up to 8 steps ahead of the tensor core, which hides
-// the latency of one warpgroup's step (each warpgroup owns every fourth step).
-// The forward's low-rank steps (A = a tile of B^T, by TMA) keep the
-// shared-memory ring.
+// The tensor-memory ring has its own SAT slots and barriers; the forward's
+// low-rank steps (A = a tile of B^T, by TMA) keep the shared-memory ring.  An
+// 8-deep tensor-memory ring (the dequant warpgroups up to 8 steps ahead of the
+// tensor core) measured slower than 4 (809 against 852 TFLOP/s on the
+// forward calls of the 7B step), so the ring stays at the shared ring's depth.
 constexpr bool kTmemA = true;
-constexpr int SAT = 8;
+constexpr int SAT = 4;
 static_assert(SAT % kDequantWGs == 0, "tensor-memory ring slots must map to one dequant warpgroup");
 __host__ __device__ constexpr uint32_t acc_cols_of(int bt) { return uint32_t(bt < 32 ? 32 : bt); }
 __host__ __device__ constexpr uint32_t tmem_cols_of(bool bwd, int bt) {
