@@ -95,12 +95,22 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
 // dequantized weight operand in shared memory (16 KB per step).  The dequant
 // warps compute a step before they wait for its A slot, so they run ahead of
 // the tensor core by up to SA steps.
-constexpr int SX = 4, SP = 8, SA = 4;
+// Backward: SX = 4, SP = 8, SA = 4.  Forward: its weight operand lives in
+// tensor memory (below), so the shared-memory operand ring shrinks to the one
+// slot the low-rank steps use, and the activation ring takes the space: 6
+// slots (5 in ragged mode, whose per-thread scratch needs the 8-slot packed
+// ring), with 4 packed slots.  The activation tile (32 KB at 256 tokens) is
+// the largest refill of a step; a deeper ring covers its TMA latency.
+__host__ __device__ constexpr int ring_x(bool bwd, bool ragged) { return bwd ? 4 : (ragged ? 5 : 6); }
+__host__ __device__ constexpr int ring_p(bool bwd, bool ragged) { return (bwd || ragged) ? 8 : 4; }
+__host__ __device__ constexpr int ring_a(bool bwd) { return bwd ? 4 : 1; }
+constexpr int SP = 8, SA = 4;   // the backward's packed and operand rings (the largest of each)
 // Each packed and operand slot must belong to a single dequant warpgroup
 // (slot = step mod ring size, warpgroup = step mod kDequantWGs).  Otherwise two
 // warpgroups share a slot, one can run two barrier phases ahead, and a parity
 // wait would pass on the wrong phase.
 static_assert(SP % kDequantWGs == 0 && SA % kDequantWGs == 0, "ring slots must map to one dequant warpgroup");
+static_assert(ring_p(false, false) % kDequantWGs == 0, "ring slots must map to one dequant warpgroup");
 
 // Forward main steps keep the dequantized weight operand in tensor memory:
 // the dequant warps store it with tcgen05.st (thread t = row t = lane t, the
@@ -193,6 +203,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
   const Nf4GemmArgs& a = P.a;
   const int bt = P.bt;
   const uint32_t act_bytes = uint32_t(bt) * 128u;
+  constexpr int SX = ring_x(BWD, RAGGED), SP = ring_p(BWD, RAGGED), SA = ring_a(BWD);
   uint8_t* act_s = smem;                                   // SX x act_bytes
   uint8_t* pk_s = act_s + SX * act_bytes;                  // SP x 4096
   uint8_t* a_s = pk_s + SP * 4096;                         // SA x 16384
@@ -232,7 +243,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
   if (threadIdx.x == 0) {
     for (int s = 0; s < SX; ++s) { mbar_init(&x_full[s], 1); mbar_init(&x_empty[s], 1); }
     for (int s = 0; s < SP; ++s) { mbar_init(&p_full[s], 1); mbar_init(&p_empty[s], 4); }
-    for (int s = 0; s < SA; ++s) { mbar_init(&a_full[s], 4); mbar_init(&a_empty[s], 1); }
+    // backward: the 4 warps of a dequant warpgroup arrive; forward: the
+    // activation producer's one arrival with the low-rank tile's bytes
+    for (int s = 0; s < SA; ++s) { mbar_init(&a_full[s], BWD ? 4 : 1); mbar_init(&a_empty[s], 1); }
     for (int s = 0; s < SAT; ++s) { mbar_init(&t_full[s], 4); mbar_init(&t_empty[s], 1); }
     mbar_init(accf, 1);
     *abort_flag = 0;
@@ -266,6 +279,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
     // ------------------------------------------------------------ X producer
     if (elect_one()) {
       int64_t issued = 0;
+      int lr_issued = 0;
       for (int64_t ks = 0; ks < nsteps; ++ks) {
         const int s = int(ks % SX);
         const uint32_t ph = uint32_t(ks / SX) & 1u;
@@ -280,12 +294,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
           const int nchunk = a.rp / 64;
           tma_load_2d(dst, &P.tm_lact, &x_full[s], int32_t((l / nchunk) * a.rp + (l % nchunk) * 64),
                       int32_t(m0));
+          if (!BWD) {
+            // forward: the low-rank A operand, B^T [128 features x 64 ranks]
+            // as two MN-major boxes, into the one shared operand slot once the
+            // previous low-rank step's MMA has released it
+            if (l >= 1 && !mbar_wait(&a_empty[0], (uint32_t(l) & 1u) ^ 1u, a.status, abort_flag)) break;
+            const int c = l % nchunk;
+            mbar_arrive_expect_tx(&a_full[0], 16384u);
+            tma_load_2d(a_s, &P.tm_lw, &a_full[0], int32_t(w0), int32_t(c * 64));
+            tma_load_2d(a_s + 8192, &P.tm_lw, &a_full[0], int32_t(w0 + 64), int32_t(c * 64));
+            lr_issued = l + 1;
+          }
         }
         issued = ks + 1;
       }
       if (*abort_flag) {   // let copies already in flight land before the CTA exits
         for (int64_t ks = (issued > SX ? issued - SX : 0); ks < issued; ++ks)
           mbar_drain(&x_full[ks % SX], uint32_t(ks / SX) & 1u);
+        if (!BWD && lr_issued > 0) mbar_drain(&a_full[0], uint32_t(lr_issued - 1) & 1u);
       }
     }
     __syncwarp();
@@ -451,8 +477,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
           if (lane == 0) mbar_arrive(&a_full[sa]);
         } else {
           // low-rank step: the A operand is a tile of a LoRA factor, by TMA
-          // (forward: B^T [128 features x 64 ranks], two MN-major boxes;
-          //  backward: A [128 inputs x 64 ranks], one K-major box)
+          // (forward: loaded by the activation producer; backward: A [128
+          // inputs x 64 ranks], one K-major box, by this warpgroup)
+          if (!BWD) continue;
           if (ls >= SA && !(ok = mbar_wait(&a_empty[sa], a_ph ^ 1u, a.status, abort_flag))) break;
           __syncwarp();
           if (lane == 0) {
@@ -942,8 +969,9 @@ static cudaError_t launch_clustered(void (*kern)(const Params), dim3 grid, dim3 
   return cudaLaunchKernelEx(&cfg, kern, P);
 }
 
-static size_t nf4_gemm_smem(int /*backward*/, int bt) {
-  return 1024 + size_t(SX) * bt * 128 + size_t(SP) * 4096 + size_t(SA) * 16384 + 512;
+static size_t nf4_gemm_smem(int backward, bool ragged, int bt) {
+  return 1024 + size_t(ring_x(backward != 0, ragged)) * bt * 128 + size_t(ring_p(backward != 0, ragged)) * 4096 +
+         size_t(ring_a(backward != 0)) * 16384 + 512;
 }
 static size_t skinny_smem(int rp, int splits) {
   return 1024 + size_t(kSkinnyStages) * (16384 + size_t(rp) * 128) + (splits > 1 ? size_t(rp) * 512 : 0) + 256;
@@ -984,7 +1012,7 @@ cudaError_t launch_nf4_gemm(const Nf4GemmPlan& plan, const Nf4GemmArgs& a, cudaS
   }
   ok &= encode_tmap_2d(&P.tm_lact, BF, a.lora_act, hw, M, hw * 2, 64, act_box, SW);
   if (!ok) return cudaErrorInvalidValue;
-  const size_t smem = nf4_gemm_smem(plan.backward, plan.bt);
+  const size_t smem = nf4_gemm_smem(plan.backward, ragged, plan.bt);
   dim3 grid(unsigned(plan.tiles_w), unsigned(plan.tiles_t), unsigned(plan.splits));
   void (*kern)(const Nf4GemmParams);
   if (ragged) kern = plan.backward ? nf4_gemm_kernel<true, true> : nf4_gemm_kernel<false, true>;

@@ -13,7 +13,8 @@
 // it reads 0.5 byte of packed code per weight and writes the 2-byte result;
 // the rank-r product adds 2 r flops per weight, which the tensor cores absorb.
 //
-// Tiling: one CTA per 128 (rows of W) x 128 (columns) output tile, 8 warps.
+// Tiling: one CTA per 128 (rows of W) x 128 (columns) output tile, 8 warps,
+// three CTAs per SM.
 // The tile's slices of B^T [128 x r] and A [128 x r] are staged in shared
 // memory (zero padded to r rounded up to 16), each warp forms a 32 x 64 part
 // of p with ldmatrix + mma.sync, the whole tile of p is parked in shared
@@ -64,7 +65,7 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
 }
 
 template <bool F16>
-__global__ void __launch_bounds__(kMergeThreads) nf4_merge_kernel(const __grid_constant__ MergeParams P) {
+__global__ void __launch_bounds__(kMergeThreads, 3) nf4_merge_kernel(const __grid_constant__ MergeParams P) {
   extern __shared__ __align__(16) uint8_t smem[];
   const MergeArgs& a = P.a;
   const int rp = P.rp;
@@ -78,29 +79,6 @@ __global__ void __launch_bounds__(kMergeThreads) nf4_merge_kernel(const __grid_c
   const int64_t k0 = int64_t(blockIdx.x) * kTile;
   const int64_t n0 = int64_t(blockIdx.y) * kTile;
   if (tid < 16) code_s[tid] = P.code[tid];
-
-  // ---- the epilogue's packed codes and block constants, loaded first so that
-  // their latency overlaps the staging and the MMAs.  Thread tid handles the
-  // 8-column piece pc = tid % 16 of rows tid / 16 + 16 j, j = 0..7.
-  const bool vec = (a.K % 8) == 0;
-  const int pc = tid & 15;
-  constexpr int kPieces = kTile * (kTile / 8) / kMergeThreads;   // 8
-  uint32_t pw[kPieces];
-  float ps[kPieces];
-  if (vec) {
-#pragma unroll
-    for (int j = 0; j < kPieces; ++j) {
-      const int64_t n = n0 + (tid >> 4) + 16 * j;
-      const int64_t k = k0 + pc * 8;
-      pw[j] = 0u;
-      ps[j] = 0.0f;
-      if (n < a.N && k < a.K) {
-        const int64_t e0 = n * a.K + k;
-        pw[j] = __ldcs(reinterpret_cast<const unsigned int*>(a.packed + (e0 >> 1)));
-        ps[j] = block_scale(a.double_quant, a.c1, a.c2, e0 >> 6);
-      }
-    }
-  }
 
   // ---- stage the operand slices (zero padded past r, N and K), four 16-byte
   // loads in flight per thread
@@ -220,6 +198,30 @@ __global__ void __launch_bounds__(kMergeThreads) nf4_merge_kernel(const __grid_c
       }
   }
   __syncthreads();
+
+  // ---- the epilogue's packed codes and block constants, all eight pieces'
+  // loads in flight at once (after the MMAs, so that the accumulators and
+  // these registers are never live together: three CTAs fit an SM).  Thread
+  // tid handles the 8-column piece pc = tid % 16 of rows tid / 16 + 16 j.
+  const bool vec = (a.K % 8) == 0;
+  const int pc = tid & 15;
+  constexpr int kPieces = kTile * (kTile / 8) / kMergeThreads;   // 8
+  uint32_t pw[kPieces];
+  float ps[kPieces];
+  if (vec) {
+#pragma unroll
+    for (int j = 0; j < kPieces; ++j) {
+      const int64_t n = n0 + (tid >> 4) + 16 * j;
+      const int64_t k = k0 + pc * 8;
+      pw[j] = 0u;
+      ps[j] = 0.0f;
+      if (n < a.N && k < a.K) {
+        const int64_t e0 = n * a.K + k;
+        pw[j] = __ldcs(reinterpret_cast<const unsigned int*>(a.packed + (e0 >> 1)));
+        ps[j] = block_scale(a.double_quant, a.c1, a.c2, e0 >> 6);
+      }
+    }
+  }
 
   // ---- epilogue: W' = round(fma(s, p, wd)), 8 columns of one row per piece
   if (vec) {
