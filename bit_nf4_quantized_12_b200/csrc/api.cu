@@ -179,7 +179,7 @@ nf4_status nf4_dequant(nf4_weight w, int32_t dtype, uint16_t* out, void* stream)
   if (!dtype_ok(dtype) || !out || w.rows < 1 || w.cols < 1) return NF4_ERR_INVALID_ARG;
   const nf4_status st = check_weight(w);
   if (st != NF4_OK) return st;
-  if (w.rows > (int64_t(1) << 40) / w.cols) return NF4_ERR_UNSUPPORTED;
+  if (w.rows > (int64_t(1) << 37) / w.cols) return NF4_ERR_UNSUPPORTED;   // the output's tile rows are int32
   if (!aligned16(out)) return NF4_ERR_MISALIGNED;
   cudaError_t e = launch_dequant(w.packed, w.c1q, w.c2, w.rows * w.cols, w.quant_type, w.double_quant,
                                  dtype == QLORA_F16, out, device_sms(), static_cast<cudaStream_t>(stream));

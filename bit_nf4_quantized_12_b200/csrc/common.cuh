@@ -129,6 +129,20 @@ NF4_DEV void tma_load_2d(void* dst, const CUtensorMap* m, uint64_t* bar, int32_t
       "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
 }
+// Shared -> global tile store by TMA (2-D tensor map; rows past the tensor's
+// extent are not written), tracked as a bulk async-group of this thread.
+NF4_DEV void tma_store_2d(const CUtensorMap* m, const void* src, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+NF4_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// this thread's committed bulk stores have read their shared source
+NF4_DEV void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// this thread's committed bulk stores are complete
+NF4_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Contiguous global -> shared copy by the bulk-copy engine, completing on an
 // mbarrier; both addresses and the size are multiples of 16 bytes.
 NF4_DEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {

@@ -18,7 +18,8 @@
 // consecutive weights per MMA (MMA t takes weights 4t .. 4t+3 of the block as
 // its slots 2c, 2c+1, 2c+8, 2c+9).  So every lane builds one 16-entry table
 // per block and row (the same byte-permute lookup as the tensor-core GEMM),
-// and the B fragment is four consecutive x values of that block.
+// and the B fragment is four consecutive x values of that block; one 16-byte
+// shared load gives the x values of two consecutive MMAs.
 //
 // Work split.  A tile is 256 rows of W (16 consumer warps x 16 rows); a unit
 // is one tile x 256 columns.  Persistent CTAs (one per SM) take contiguous
@@ -28,9 +29,13 @@
 // workspace, and the last one adds them in CTA order (a fixed order, so the
 // result does not depend on timing).  One producer warp streams the units
 // through a ring of shared-memory stages with TMA: the 256 x 128-byte box of
-// packed codes and the 4 x (64 columns x M tokens) boxes of X, both with the
-// 128-byte swizzle so that the fragment reads spread over the banks.  Every
-// wait is bounded and reports kStatusTimeout instead of hanging.
+// packed codes and the 4 boxes of X (64 columns each), both with the 128-byte
+// swizzle.  The X box of block c is loaded from token row -2c (rows before
+// token 0 and past the last token read as zeros), so token m sits in shared
+// row m + 2c and the eight lanes that share a 128-byte phase of a load (two
+// token rows x four blocks) meet eight different swizzle phases: the loads
+// are free of bank conflicts.  Every wait is bounded and reports
+// kStatusTimeout instead of hanging.
 #include <cstdint>
 #include <cstring>
 #include <cuda.h>
@@ -54,19 +59,16 @@ struct DecodeParams {
   CUtensorMap tm_x;    // X [M, K] 2-byte, box {64, M}, 128-byte swizzle
   Nf4DecodeArgs a;
   CodeTable code;
+  ShiftMuls km;
   int64_t tiles, nk, units;
-  uint32_t xbox_bytes;  // shared bytes per X box (1024 per 8 tokens)
+  uint32_t xrows;       // rows of an X box: 8 per token tile + 6 for the block offsets
+  uint32_t xbox_bytes;  // shared bytes per X box (xrows x 128, a multiple of 1024)
   uint32_t stage_bytes;
 };
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ uint2 lds64(uint32_t addr) {
-  uint2 v;
-  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
   return v;
 }
 __device__ __forceinline__ void consumer_sync() {   // the 16 consumer warps
@@ -141,11 +143,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) nf4_decode_kernel(const __grid
         if (i >= kDecStages && !mbar_wait(&empty[s], uint32_t(i / kDecStages - 1) & 1u, a.status, abort_flag)) break;
         const int64_t tile = u / P.nk, kc = u % P.nk;
         uint8_t* st = smem + s * P.stage_bytes;
-        mbar_arrive_expect_tx(&full[s], kPkBytes + 4u * uint32_t(a.M) * 128u);
+        mbar_arrive_expect_tx(&full[s], kPkBytes + 4u * P.xrows * 128u);
         tma_load_2d(st, &P.tm_pk, &full[s], int32_t(kc * 128), int32_t(tile * kDecTileRows));
 #pragma unroll
         for (int c = 0; c < 4; ++c)
-          tma_load_2d(st + kPkBytes + c * P.xbox_bytes, &P.tm_x, &full[s], int32_t(kc * kDecChunk + c * 64), 0);
+          tma_load_2d(st + kPkBytes + c * P.xbox_bytes, &P.tm_x, &full[s], int32_t(kc * kDecChunk + c * 64),
+                      -2 * c);
         issued = i + 1;
       }
       if (*abort_flag) {   // let copies already in flight land before the CTA exits
@@ -165,11 +168,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) nf4_decode_kernel(const __grid
   const int g = lane >> 2, c = lane & 3;
   const int row0 = warp * 16 + g;           // rows row0 and row0 + 8 of the tile
   bool ok = true, have_T = false;
-  float acc[NT][4];
+  // two accumulators per token tile (even and odd MMAs), so that two chains
+  // of dependent MMAs are in flight; summed when a segment ends
+  float acc[NT][4], acc2[NT][4];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-    for (int q = 0; q < 4; ++q) acc[nt][q] = 0.0f;
+    for (int q = 0; q < 4; ++q) acc[nt][q] = acc2[nt][q] = 0.0f;
 
   // block constants of (row, block c of unit (tile, kc)), loaded one unit ahead
   auto load_scales = [&](bool valid, int64_t tile, int64_t kc, uint32_t (&q)[2], float (&s2)[2]) {
@@ -183,6 +188,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) nf4_decode_kernel(const __grid
       if (n < a.N) load_scale_parts(a.dq, a.c1q, a.c2, n * KB + kb, q[h], s2[h]);
     }
   };
+  const uint32_t xph = uint32_t((g + 2 * c) & 7) << 4;   // swizzle phase of this lane's token rows
   uint32_t cq[2], nq[2];
   float cs[2], ns[2];
   int64_t tile = u0 / P.nk, kc = u0 % P.nk;          // unit u = tile * nk + kc, advanced without division
@@ -219,22 +225,20 @@ __global__ void __launch_bounds__(kDecThreads, 1) nf4_decode_kernel(const __grid
       }
       const BlockTable t0 = make_table(P.code, scale_from_parts(a.dq, cq[0], cs[0]), F16);
       const BlockTable t1 = make_table(P.code, scale_from_parts(a.dq, cq[1], cs[1]), F16);
-      // X box c, token row nt * 8 + g (its index mod 8 is g)
-      const uint32_t xb = st + kPkBytes + uint32_t(c) * P.xbox_bytes + uint32_t(g) * 128u;
+      // X box c: token nt * 8 + g sits in shared row nt * 8 + g + 2c
+      // (the row starts on 128 bytes, so chunk i of it is at row ^ ((i << 4) ^ xph))
+      const uint32_t xb = (st + kPkBytes + uint32_t(c) * P.xbox_bytes + uint32_t(g + 2 * c) * 128u) | xph;
 #pragma unroll
-      for (int t = 0; t < 16; ++t) {
-        // upper halves by a high multiply (FMA pipe): the integer pipe is the
-        // one the lookups keep busy
-        const uint32_t s0 = (t & 1) ? __umulhi(w0[t >> 1], 0x10000u) : w0[t >> 1];
-        const uint32_t s1 = (t & 1) ? __umulhi(w1[t >> 1], 0x10000u) : w1[t >> 1];
-        uint32_t a0, a1, a2, a3;
-        lookup4(t0, s0, a0, a2);
-        lookup4(t1, s1, a1, a3);
-        const uint32_t xo = ((uint32_t(t >> 1) ^ uint32_t(g)) << 4) + uint32_t(t & 1) * 8u;
+      for (int i = 0; i < 8; ++i) {
+        // word i: weights 8i .. 8i + 7 of the block, MMAs 2i and 2i + 1
+        uint32_t p0, p1, p2, p3, q0, q1, q2, q3;
+        lookup8(t0, w0[i], P.km, p0, p1, p2, p3);
+        lookup8(t1, w1[i], P.km, q0, q1, q2, q3);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          const uint2 b = lds64(xb + uint32_t(nt) * 1024u + xo);
-          mma16816<F16>(acc[nt], a0, a1, a2, a3, b.x, b.y);
+          const uint4 b = lds128((xb ^ uint32_t(i << 4)) + uint32_t(nt) * 1024u);
+          mma16816<F16>(acc[nt], p0, q0, p1, q1, b.x, b.y);
+          mma16816<F16>(acc2[nt], p2, q2, p3, q3, b.z, b.w);
         }
       }
       // the stage is refilled by TMA (async proxy): order these reads first
@@ -254,12 +258,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) nf4_decode_kernel(const __grid
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const int tk = nt * 8 + 2 * c;
-      red[tk * kDecTileRows + row0] = acc[nt][0];
-      red[(tk + 1) * kDecTileRows + row0] = acc[nt][1];
-      red[tk * kDecTileRows + row0 + 8] = acc[nt][2];
-      red[(tk + 1) * kDecTileRows + row0 + 8] = acc[nt][3];
+      red[tk * kDecTileRows + row0] = acc[nt][0] + acc2[nt][0];
+      red[(tk + 1) * kDecTileRows + row0] = acc[nt][1] + acc2[nt][1];
+      red[tk * kDecTileRows + row0 + 8] = acc[nt][2] + acc2[nt][2];
+      red[(tk + 1) * kDecTileRows + row0 + 8] = acc[nt][3] + acc2[nt][3];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) acc[nt][q] = 0.0f;
+      for (int q = 0; q < 4; ++q) acc[nt][q] = acc2[nt][q] = 0.0f;
     }
     consumer_sync();
     const int tid = threadIdx.x;   // 0 .. 511
@@ -351,8 +355,11 @@ DecodePlan plan_decode(int64_t M, int64_t N, int64_t K, int num_sms) {
   return d;
 }
 
+uint32_t decode_xrows(int64_t M) { return uint32_t(cdiv(M, 8)) * 8u + 6u; }
+uint32_t decode_xbox_bytes(int64_t M) { return uint32_t(cdiv(decode_xrows(M) * 128, 1024)) * 1024u; }
+
 size_t decode_smem_bytes(int64_t M) {
-  const uint32_t xbox = uint32_t(cdiv(M, 8)) * 1024u;
+  const uint32_t xbox = decode_xbox_bytes(M);
   const size_t stage = kPkBytes + 4 * size_t(xbox);
   return 1024 + kDecStages * stage + 16 * kDecTileRows * 4 + 2 * kDecStages * 8 + 16;
 }
@@ -367,14 +374,16 @@ cudaError_t launch_nf4_decode(const DecodePlan& plan, const Nf4DecodeArgs& a, co
   P.tiles = plan.tiles;
   P.nk = plan.nk;
   P.units = plan.units;
-  P.xbox_bytes = uint32_t(cdiv(a.M, 8)) * 1024u;
+  P.km = make_shift_muls();
+  P.xrows = decode_xrows(a.M);
+  P.xbox_bytes = decode_xbox_bytes(a.M);
   P.stage_bytes = kPkBytes + 4 * P.xbox_bytes;
   const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
   const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;   // 2-byte elements (bf16 or fp16)
   const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
   const uint64_t M = a.M, N = a.N, K = a.K;
   bool ok = encode_tmap_2d(&P.tm_pk, U8, a.packed, K / 2, N, K / 2, 128, kDecTileRows, SW);
-  ok &= encode_tmap_2d(&P.tm_x, BF, a.X, K, M, K * 2, 64, uint32_t(M), SW);
+  ok &= encode_tmap_2d(&P.tm_x, BF, a.X, K, M, K * 2, 64, P.xrows, SW);
   if (!ok) return cudaErrorInvalidValue;
   const size_t smem = decode_smem_bytes(a.M);
   void (*kern)(const DecodeParams);

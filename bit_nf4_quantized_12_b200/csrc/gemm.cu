@@ -46,11 +46,12 @@ constexpr int kSkinnyStages = 2;
 
 struct Nf4GemmParams {
   CUtensorMap tm_act;   // X [M,K] / dY [M,N], bf16, box {64, bt}, 128B swizzle
-  CUtensorMap tm_pk;    // packed [N, K/2] bytes; box {32,128} fwd, {64,64} bwd
+  CUtensorMap tm_pk;    // packed [N, K/2] bytes; box {32,128} fwd (32-byte swizzle), {64,64} bwd (64-byte)
   CUtensorMap tm_lact;  // hi/lo [M, 2rp] bf16, box {64, bt}, 128B swizzle
   CUtensorMap tm_lw;    // forward: B [r, N], box {64, 64}; backward: A [K, r], box {64, 128}; 128B swizzle
   Nf4GemmArgs a;
   CodeTable code;
+  ShiftMuls km;
   int bt;
   int splits;
   int64_t main_steps;   // total 64-wide steps of the main reduction
@@ -174,19 +175,17 @@ __device__ __forceinline__ void load_codes64(const uint8_t* packed, int64_t pack
 // 64 codes -> 32 bf16x2 (or f16x2) words in element order, each element taking
 // its value from t0 or, where its lane of masks[group] is set, from t1.
 __device__ __forceinline__ void dequant64_two(const BlockTable& t0, const BlockTable& t1, const uint32_t (&w)[8],
-                                              const uint2* masks, uint32_t (&o)[32]) {
+                                              const uint2* masks, const ShiftMuls& km, uint32_t (&o)[32]) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const uint32_t s = h ? (w[i] >> 16) : w[i];
-      uint32_t a01, a23, b01, b23;
-      lookup4(t0, s, a01, a23);
-      lookup4(t1, s, b01, b23);
-      const uint2 m = masks[2 * i + h];
-      o[4 * i + 2 * h] = (a01 & ~m.x) | (b01 & m.x);
-      o[4 * i + 2 * h + 1] = (a23 & ~m.y) | (b23 & m.y);
-    }
+    lookup8(t0, w[i], km, o[4 * i + 0], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+    uint32_t b[4];
+    lookup8(t1, w[i], km, b[0], b[1], b[2], b[3]);
+    const uint4 m = *reinterpret_cast<const uint4*>(masks + 2 * i);
+    o[4 * i + 0] = (o[4 * i + 0] & ~m.x) | (b[0] & m.x);
+    o[4 * i + 1] = (o[4 * i + 1] & ~m.y) | (b[1] & m.y);
+    o[4 * i + 2] = (o[4 * i + 2] & ~m.z) | (b[2] & m.z);
+    o[4 * i + 3] = (o[4 * i + 3] & ~m.w) | (b[3] & m.w);
   }
 }
 
@@ -430,15 +429,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
           if (!RAGGED) {
             const int sp = int(ks % SP);
             if (!(ok = mbar_wait(&p_full[sp], uint32_t(ks / SP) & 1u, a.status, abort_flag))) break;
-            const uint32_t pa = BWD ? smem_u32(pk_s + sp * 4096 + (t & 63) * 64 + (t >> 6) * 32)
-                                    : smem_u32(pk_s + sp * 4096 + t * 32);
-            const uint4 p0 = lds128(pa), p1 = lds128(pa + 16);
+            // The packed box is swizzled (32-byte mode forward, 64-byte mode
+            // backward): 16-byte chunk c of a row sits at c ^ (address bits 7
+            // and up), so the 8 lanes of each load phase hit 8 different bank
+            // groups.  Forward: row t, 32 bytes, chunks 0 and 1; backward: row
+            // t % 64, 64 bytes, chunks 2 (t / 64) and 2 (t / 64) + 1.
+            const uint32_t row = smem_u32(pk_s + sp * 4096) + (BWD ? uint32_t(t & 63) * 64u : uint32_t(t) * 32u);
+            const uint32_t c0 = BWD ? uint32_t(2 * (t >> 6)) ^ ((uint32_t(t & 63) >> 1) & 3u) : (uint32_t(t) >> 2) & 1u;
+            const uint4 p0 = lds128(row + (c0 << 4)), p1 = lds128(row + ((c0 ^ 1u) << 4));
             // The slot is refilled by TMA, an async-proxy write: order these
             // generic-proxy reads before it, or the refill can land first.
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_empty[sp]);
-            dequant64(make_table(P.code, scale_from_parts(a.dq, cq[j], cc[j]), f16), p0, p1, o);
+            dequant64(make_table(P.code, scale_from_parts(a.dq, cq[j], cc[j]), f16), p0, p1, P.km, o);
           } else {
             const int64_t e0 = seg_of(ks);
             uint32_t wv[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
@@ -446,7 +450,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
               load_codes64(a.packed, a.packed_bytes, e0, smem_u32(pk_s) + uint32_t(threadIdx.x - 128) * 48u, wv);
             const uint2* masks = reinterpret_cast<const uint2*>(pk_s + kRaggedMaskOffset) + (e0 >= 0 ? (e0 & 63) : 0) * 16;
             dequant64_two(make_table(P.code, scale_from_parts(a.dq, cq[j], cc[j]), f16),
-                          make_table(P.code, scale_from_parts(a.dq, cq2[j], cc2[j]), f16), wv, masks, o);
+                          make_table(P.code, scale_from_parts(a.dq, cq2[j], cc2[j]), f16), wv, masks, P.km, o);
           }
           if (!BWD && kTmemA) {
             // forward: row t of Wd into tensor memory, lane t (this warp's
@@ -987,11 +991,11 @@ cudaError_t launch_nf4_gemm(const Nf4GemmPlan& plan, const Nf4GemmArgs& a, cudaS
   P.lora_steps = plan.lora_steps;
   const Codebook& cb = host_codebook(a.quant_type);
   for (int i = 0; i < 16; ++i) P.code.v[i] = cb.code[i];
+  P.km = make_shift_muls();
   // 2-byte elements; TMA only moves them, so bf16 and fp16 share the map type
   const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
   const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
-  const auto NOSW = CU_TENSOR_MAP_SWIZZLE_NONE;
   bool ok = true;
   const uint64_t M = a.M, N = a.N, K = a.K;
   const uint64_t hw = 2 * uint64_t(a.rp);
@@ -1003,11 +1007,11 @@ cudaError_t launch_nf4_gemm(const Nf4GemmPlan& plan, const Nf4GemmArgs& a, cudaS
   const uint64_t lda = uint64_t(a.ld_act), ldl = uint64_t(a.ld_lw);
   if (!plan.backward) {
     ok &= encode_tmap_2d(&P.tm_act, BF, a.act, K, M, lda * 2, 64, act_box, SW);
-    if (!ragged) ok &= encode_tmap_2d(&P.tm_pk, U8, a.packed, K / 2, N, K / 2, 32, 128, NOSW);
+    if (!ragged) ok &= encode_tmap_2d(&P.tm_pk, U8, a.packed, K / 2, N, K / 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_32B);
     ok &= encode_tmap_2d(&P.tm_lw, BF, a.lora_w, N, uint64_t(a.r), ldl * 2, 64, 64, SW);
   } else {
     ok &= encode_tmap_2d(&P.tm_act, BF, a.act, N, M, lda * 2, 64, act_box, SW);
-    if (!ragged) ok &= encode_tmap_2d(&P.tm_pk, U8, a.packed, K / 2, N, K / 2, 64, 64, NOSW);
+    if (!ragged) ok &= encode_tmap_2d(&P.tm_pk, U8, a.packed, K / 2, N, K / 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_64B);
     ok &= encode_tmap_2d(&P.tm_lw, BF, a.lora_w, uint64_t(a.r), K, uint64_t(a.r) * 2, 64, 128, SW);
   }
   ok &= encode_tmap_2d(&P.tm_lact, BF, a.lora_act, hw, M, hw * 2, 64, act_box, SW);

@@ -49,15 +49,54 @@ __device__ __forceinline__ void lookup4(const BlockTable& t, uint32_t s, uint32_
   o23 = prmt(lo, hi, 0x7362);
 }
 
+// Multipliers of the high-multiply shifts below.  They reach the kernels as
+// launch parameters, so the compiler cannot turn a multiply by a power of two
+// back into a shift: the shifts then run on the FMA pipe as integer
+// multiply-adds, next to the integer pipe that the byte permutes keep busy.
+struct ShiftMuls {
+  uint32_t k16;   // 2^16: x >> 16
+  uint32_t k15;   // 2^15: x >> 17
+  uint32_t k31;   // 2^31: x >> 1
+};
+inline ShiftMuls make_shift_muls() { return ShiftMuls{1u << 16, 1u << 15, 1u << 31}; }
+
+__device__ __forceinline__ uint32_t mulhi_add(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("mad.hi.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// Eight nibbles (one packed word, element j in nibble j) -> four bf16x2 words
+// (elements 0-1, 2-3, 4-5, 6-7).  The flip of bit 3 and its mask are taken
+// once for the eight nibbles; the upper four nibbles' selectors come from
+// them by high multiplies.
+__device__ __forceinline__ void lookup8(const BlockTable& t, uint32_t w, const ShiftMuls& k, uint32_t& o0,
+                                        uint32_t& o1, uint32_t& o2, uint32_t& o3) {
+  const uint32_t wb = w ^ 0x88888888u;     // selectors into entries 8-15
+  const uint32_t m = w & 0x88888888u;      // bit 3 of every nibble
+  const uint32_t sel2_lo = mulhi_add(m, k.k31, 0x3210u);   // ((m >> 1) & 0x4444) | 0x3210 (bits 16+ unused)
+  const uint32_t sel2_hi = mulhi_add(m, k.k15, 0x3210u);   // the same for nibbles 4-7
+  const uint32_t wa_hi = mulhi_add(w, k.k16, 0u), wb_hi = mulhi_add(wb, k.k16, 0u);   // >> 16
+  {
+    const uint32_t lo = prmt(prmt(t.lo[0], t.lo[1], w), prmt(t.lo[2], t.lo[3], wb), sel2_lo);
+    const uint32_t hi = prmt(prmt(t.hi[0], t.hi[1], w), prmt(t.hi[2], t.hi[3], wb), sel2_lo);
+    o0 = prmt(lo, hi, 0x5140);
+    o1 = prmt(lo, hi, 0x7362);
+  }
+  {
+    const uint32_t lo = prmt(prmt(t.lo[0], t.lo[1], wa_hi), prmt(t.lo[2], t.lo[3], wb_hi), sel2_hi);
+    const uint32_t hi = prmt(prmt(t.hi[0], t.hi[1], wa_hi), prmt(t.hi[2], t.hi[3], wb_hi), sel2_hi);
+    o2 = prmt(lo, hi, 0x5140);
+    o3 = prmt(lo, hi, 0x7362);
+  }
+}
+
 // 32 packed bytes (64 weights) -> 32 bf16x2 words in element order.
-__device__ __forceinline__ void dequant64(const BlockTable& t, const uint4& p0, const uint4& p1,
+__device__ __forceinline__ void dequant64(const BlockTable& t, const uint4& p0, const uint4& p1, const ShiftMuls& km,
                                           uint32_t (&o)[32]) {
   const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    lookup4(t, w[i] & 0xFFFFu, o[4 * i + 0], o[4 * i + 1]);
-    lookup4(t, w[i] >> 16, o[4 * i + 2], o[4 * i + 3]);
-  }
+  for (int i = 0; i < 8; ++i) lookup8(t, w[i], km, o[4 * i + 0], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
 }
 
 }  // namespace nf4

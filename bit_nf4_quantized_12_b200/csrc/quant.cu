@@ -22,10 +22,13 @@
 // bf16: the table, the per-block constant and the final rounding change,
 // nothing else.
 //
-// Both kernels are HBM-bandwidth bound: 16-byte coalesced loads and stores,
-// the per-block absmax by warp shuffles across the 8 lanes that own a block,
-// and the code decision as one lookup in a 33-cell shared-memory table plus
-// one compare (about 8 instructions per weight, most on the FMA pipe).
+// Both kernels are meant to be HBM-bandwidth bound, so both keep the
+// instructions per weight low.  Quantize: 16-byte coalesced loads and
+// stores, the per-block absmax by warp shuffles across the 8 lanes that own a
+// block, and the code decision as one lookup in a 33-cell shared-memory table
+// plus one compare.  Dequantize: one lane per block, the block's 16 values
+// formed once and the codes looked up with byte permutes (about 2.3 integer
+// operations per weight), the output leaving through TMA tile stores.
 #include <cstdint>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -36,9 +39,17 @@
 namespace nf4 {
 namespace {
 
-constexpr int kQuantThreads = 512;   // one group (16384 weights) per CTA iteration
-constexpr int kQuantIters = kGroupElems / (kQuantThreads * 8);   // 16-byte loads per thread per group: 4
-static_assert(kQuantIters * kQuantThreads * 8 == kGroupElems, "a group is an exact number of passes");
+// A CTA of four warps quantizes one group (16384 weights) at a time.  A pass
+// is one 16-byte load per lane: 256 weights, four blocks of 8 lanes each.
+// Warp w takes passes 16 w .. 16 w + 15 of the group as two batches of 8,
+// and within a batch lane j of each 8-lane block group owns pass j (its
+// block's reciprocal is taken once and shuffled to the other lanes).
+constexpr int kQuantWarps = 4;
+constexpr int kQuantThreads = kQuantWarps * 32;
+constexpr int kQuantBatch = 8;                                      // passes per batch
+constexpr int kPassElems = 32 * 8;                                  // weights per pass
+constexpr int kWarpBatches = kGroupElems / (kPassElems * kQuantBatch * kQuantWarps);   // 2
+static_assert(kWarpBatches * kPassElems * kQuantBatch * kQuantWarps == kGroupElems, "whole batches per group");
 constexpr int kCells = 33;           // cells of 16 x: floor(16 x) = -16 .. 16
 
 // Code decision by cells of width 1/16 in x = w / absmax: cell c holds
@@ -74,13 +85,19 @@ __device__ __forceinline__ uint32_t classify16(const uint2* cells, float x16) {
 // is the integer 2^23 + 16 + floor(x16), so the low bits of its pattern are
 // the cell index 0..32: one round-down add on the FMA pipe instead of a
 // float-to-int conversion.  cells_biased is the cell table's shared address
-// minus 8 * 0x4B000000 (mod 2^32), so the pattern times 8 addresses the cell
-// directly.  The comparison x16 > 16 T is the sign bit of 16 T - x16, which is
-// +0 for x16 == 16 T (ties go to the lower code) and +inf where the cell holds
-// no threshold.
-__device__ __forceinline__ uint32_t classify_fast(uint32_t cells_biased, float x16) {
+// minus 8 * 0x4B000000 (mod 2^32), so the pattern times 8 (one integer
+// multiply-add by the runtime constant k8 = 8, on the FMA pipe) addresses the
+// cell directly.  The comparison x16 > 16 T is the sign bit of 16 T - x16,
+// which is +0 for x16 == 16 T (ties go to the lower code) and +inf where the
+// cell holds no threshold.
+__device__ __forceinline__ uint32_t mad_lo(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ uint32_t classify_fast(uint32_t cells_biased, float x16, uint32_t k8) {
   const float r = __fadd_rd(x16, 8388624.0f);
-  const uint32_t addr = cells_biased + (__float_as_uint(r) << 3);
+  const uint32_t addr = mad_lo(__float_as_uint(r), k8, cells_biased);
   uint32_t t, base;
   asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(t), "=r"(base) : "r"(addr));
   return base + (__float_as_uint(__uint_as_float(t) - x16) >> 31);
@@ -103,29 +120,33 @@ __device__ __forceinline__ uint32_t classify_exact(const uint2* cells, float x16
 // inv16 = 16 / scale1 (of the weights first scaled by pre, a power of two,
 // on the careful path for extreme or non-finite blocks); c1 = scale1 * pre.
 // MODE 0: fast cells (NF4 blocks with a normal scale1); 1: clamped cells (any
-// input); 2: exact comparison (dyadic thresholds).
+// input); 2: exact comparison (dyadic thresholds).  km holds runtime copies
+// of 8 and 2^16, so that those products stay integer multiply-adds.
 template <int MODE>
 __device__ __forceinline__ uint32_t quantize8(const uint2* cells, uint32_t cells_biased, const uint4& v,
-                                              float inv16, float pre, float c1) {
+                                              float inv16, float pre, float c1, uint32_t k8 = 8u,
+                                              uint32_t k65536 = 65536u) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   uint32_t out = 0;
+  if constexpr (MODE == 0) {   // each byte's two codes ORed in at fixed positions: no serial chain
 #pragma unroll
-  for (int j = 3; j >= 0; --j) {
-    float hi = bf16hi_to_f32(w[j]), lo = bf16lo_to_f32(w[j]);
-    if (MODE != 0) {
-      hi *= pre;
-      lo *= pre;
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t lo = classify_fast(cells_biased, __uint_as_float(mad_lo(w[j], k65536, 0u)) * inv16, k8);
+      const uint32_t hi = classify_fast(cells_biased, bf16hi_to_f32(w[j]) * inv16, k8);
+      out |= (lo | (hi << 4)) << (8 * j);
     }
-    const float xh = hi * inv16, xl = lo * inv16;
-    if (MODE == 0) {
-      out = out * 16u + classify_fast(cells_biased, xh);
-      out = out * 16u + classify_fast(cells_biased, xl);
-    } else if (MODE == 1) {
-      out = out * 16u + classify16(cells, xh);
-      out = out * 16u + classify16(cells, xl);
-    } else {
-      out = out * 16u + classify_exact(cells, xh, hi, c1);
-      out = out * 16u + classify_exact(cells, xl, lo, c1);
+  } else {
+#pragma unroll
+    for (int j = 3; j >= 0; --j) {
+      float hi = bf16hi_to_f32(w[j]) * pre, lo = bf16lo_to_f32(w[j]) * pre;
+      const float xh = hi * inv16, xl = lo * inv16;
+      if (MODE == 1) {
+        out = out * 16u + classify16(cells, xh);
+        out = out * 16u + classify16(cells, xl);
+      } else {
+        out = out * 16u + classify_exact(cells, xh, hi, c1);
+        out = out * 16u + classify_exact(cells, xl, lo, c1);
+      }
     }
   }
   return out;
@@ -154,36 +175,50 @@ struct QuantArgs {
   int dq;              // DqFormat
   int exact;           // exact comparisons (tables with dyadic thresholds)
   uint32_t zero8;      // eight nibbles of the table's 0.0 code (all-zero blocks)
+  uint32_t k8, k65536; // 8 and 2^16 (runtime values: see quantize8)
   float thr[15];
 };
 
-// Pass i of a group covers weights i * 4096 .. i * 4096 + 4095; thread tid
-// loads 8 of them (tid * 8 ..), so the 8 lanes tid & ~7 .. tid | 7 hold one
-// 64-weight block.
-__device__ __forceinline__ void load_group(const QuantArgs& p, int64_t g, uint4 (&v)[kQuantIters]) {
-  const int64_t gbase = g * kGroupElems;
-  const bool full = gbase + kGroupElems <= p.numel;
+// Batch b (0 .. kWarpBatches - 1) of this warp in group g: passes
+// P = (kWarpBatches w + b) 8 + i for i = 0..7; pass P covers weights
+// P * 256 + lane * 8 .. + 7 of the group.  Elements past the end read as 0.
+__device__ __forceinline__ int64_t batch_first(int64_t g, int b) {
+  const int warp = threadIdx.x >> 5;
+  return g * kGroupElems + int64_t((kWarpBatches * warp + b) * kQuantBatch) * kPassElems;
+}
+__device__ __forceinline__ void load_batch(const QuantArgs& p, int64_t e_first, uint4 (&v)[kQuantBatch]) {
+  const int lane = threadIdx.x & 31;
+  if (e_first + kQuantBatch * kPassElems <= p.numel) {   // one base pointer, constant offsets
+    const uint4* src = reinterpret_cast<const uint4*>(p.W + e_first) + lane;
 #pragma unroll
-  for (int i = 0; i < kQuantIters; ++i) {
-    const int64_t e0 = gbase + int64_t(i) * (kQuantThreads * 8) + threadIdx.x * 8;
-    if (full || e0 + 8 <= p.numel) {
+    for (int i = 0; i < kQuantBatch; ++i) v[i] = __ldcs(src + i * 32);
+    return;
+  }
+#pragma unroll
+  for (int i = 0; i < kQuantBatch; ++i) {
+    const int64_t e0 = e_first + int64_t(i) * kPassElems + lane * 8;
+    if (e0 + 8 <= p.numel) {
       v[i] = __ldcs(reinterpret_cast<const uint4*>(p.W + e0));
     } else {
       uint16_t t[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) t[j] = (e0 + j < p.numel) ? p.W[e0 + j] : uint16_t(0);
+      for (int k = 0; k < 8; ++k) t[k] = (e0 + k < p.numel) ? p.W[e0 + k] : uint16_t(0);
       v[i] = make_uint4(t[0] | (uint32_t(t[1]) << 16), t[2] | (uint32_t(t[3]) << 16),
                         t[4] | (uint32_t(t[5]) << 16), t[6] | (uint32_t(t[7]) << 16));
     }
   }
 }
 
-// Persistent CTAs walk the groups; the next group's 32 KB are loaded while
-// the current one is classified.
-__global__ void __launch_bounds__(kQuantThreads, 2) nf4_quantize_kernel(const __grid_constant__ QuantArgs p) {
+// Persistent CTAs walk the groups; each warp loads its next batch (of this
+// group or of the CTA's next one) while it classifies the current one.  The
+// 4-bit codes depend only on their own block's absmax, so they are written
+// before the group's maximum is known; the four warps then meet once per
+// group for scale2 and each writes the 8-bit codes of its own 64 blocks.
+__global__ void __launch_bounds__(kQuantThreads, 5) nf4_quantize_kernel(const __grid_constant__ QuantArgs p) {
   __shared__ uint2 cells[kCells];
   __shared__ float thr_s[16];
-  __shared__ __align__(16) uint32_t warp_max[2][kQuantThreads / 32];
+  __shared__ uint32_t warp_max[2][kQuantWarps];
+  __shared__ uint32_t keep_s[kQuantWarps][kWarpBatches * 32];   // block maxima, block order within the warp
   if (threadIdx.x < 15) thr_s[threadIdx.x] = p.thr[threadIdx.x];
   __syncthreads();
   build_cells(cells, thr_s);
@@ -191,184 +226,214 @@ __global__ void __launch_bounds__(kQuantThreads, 2) nf4_quantize_kernel(const __
   const uint32_t cells_biased = smem_u32(cells) - (0x4B000000u << 3);
 
   const int tid = threadIdx.x;
-  const int lane = tid & 31, warp = tid >> 5;
+  const int lane = tid & 31, warp = tid >> 5, j = lane & 7;
   const int64_t nblk_total = nblocks_of(p.numel);
   uint32_t bad = 0;
 
   int64_t g = blockIdx.x;
-  uint4 v[kQuantIters];
-  if (g < p.ngroups) load_group(p, g, v);
+  uint4 v[kQuantBatch];
+  if (g < p.ngroups) load_batch(p, batch_first(g, 0), v);
   for (int parity = 0; g < p.ngroups; g += gridDim.x, parity ^= 1) {
-    const int64_t gbase = g * kGroupElems;
-    // first level: absmax of each block (8 lanes x 8 weights)
-    uint32_t bm[kQuantIters];
     uint32_t gm = 0;
-#pragma unroll
-    for (int i = 0; i < kQuantIters; ++i) {
-      uint32_t m = absmax_bits8(v[i]);
-      m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-      m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
-      m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
-      bm[i] = m;
-      gm = max(gm, m);
-    }
-#pragma unroll
-    for (int o = 8; o < 32; o <<= 1) gm = max(gm, __shfl_xor_sync(0xffffffffu, gm, o));
-    if (lane == 0) warp_max[parity][warp] = gm;
-
-    // prefetch the next group while this one is finished
-    const int64_t gn = g + gridDim.x;
-    uint4 vn[kQuantIters];
-    if (gn < p.ngroups) load_group(p, gn, vn);
-
-    // 4-bit codes first: a code depends only on its own block's absmax, so
-    // this work needs no other warp and comes before the group barrier.
-    // Lane j < kQuantIters of each 8-lane block group owns pass j: it takes
-    // that block's reciprocal once; the others receive it by shuffle.
-    const int j = lane & 7;
-    uint32_t my_bm = bm[0];
-#pragma unroll
-    for (int i = 1; i < kQuantIters; ++i) my_bm = (j == i) ? bm[i] : my_bm;
-    const float my_c1 = __uint_as_float(my_bm << 16);
-    // 16 / scale1 must stay a finite normal number: scale1 in [2^-122, 2^125]
-    const bool normal = (my_c1 >= 0x1p-122f && my_c1 <= 0x1p125f) || my_c1 == 0.0f;
-    const float my_inv = (my_c1 == 0.0f) ? 0.0f : (normal ? __frcp_rn(my_c1) : 0.0f);
-    const bool fast = __all_sync(0xffffffffu, normal);
-    const int64_t ebase = gbase + tid * 8;
-    const bool full = gbase + kGroupElems <= p.numel;   // no element of this group is past the end
-#pragma unroll
-    for (int i = 0; i < kQuantIters; ++i) {
-      const int64_t e0 = ebase + i * (kQuantThreads * 8);
-      const float inv = __shfl_sync(0xffffffffu, my_inv, (lane & ~7) | i);
-      if (!full && e0 >= p.numel) continue;
-      const float c1 = __uint_as_float(bm[i] << 16);
-      uint32_t q8;
-      if (c1 == 0.0f) {
-        q8 = p.zero8;                            // all-zero block: the 0.0 code
-      } else if (p.exact) {                      // dyadic thresholds: exact comparisons
-        const bool nrm = c1 >= 0x1p-122f && c1 <= 0x1p125f;
-        const float pre = nrm ? 1.0f : ((c1 < 1.0f) ? 0x1p64f : 0x1p-64f);
-        q8 = quantize8<2>(cells, cells_biased, v[i], __frcp_rn(c1 * pre) * 16.0f, pre, c1 * pre);
-      } else if (fast) {
-        q8 = quantize8<0>(cells, cells_biased, v[i], inv * 16.0f, 1.0f, c1);
-      } else if (c1 >= 0x1p-122f && c1 <= 0x1p125f) {
-        q8 = quantize8<1>(cells, cells_biased, v[i], __frcp_rn(c1) * 16.0f, 1.0f, c1);
-      } else {                                   // keep 16/c1 a normal number
-        const float pre = (c1 < 1.0f) ? 0x1p64f : 0x1p-64f;
-        q8 = quantize8<1>(cells, cells_biased, v[i], __frcp_rn(c1 * pre) * 16.0f, pre, c1);
+#pragma unroll 1
+    for (int b = 0; b < kWarpBatches; ++b) {
+      const int64_t e_first = batch_first(g, b);
+      // prefetch: the next batch of this group, or the first of the next group
+      uint4 vn[kQuantBatch];
+      {
+        const int64_t gn = (b + 1 < kWarpBatches) ? g : g + gridDim.x;
+        if (gn < p.ngroups) load_batch(p, batch_first(gn, (b + 1) % kWarpBatches), vn);
       }
-      uint8_t* dst = p.packed + (e0 >> 1);
-      if (full || e0 + 8 <= p.numel) {
-        __stcs(reinterpret_cast<unsigned int*>(dst), q8);
-      } else {
-        const int valid = int(p.numel - e0);
+      // first level: absmax of each block (8 lanes x 8 weights)
+      uint32_t bm[kQuantBatch];
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          if (2 * jj < valid) {
-            uint32_t byte = (q8 >> (8 * jj)) & 0xFFu;
-            if (2 * jj + 1 >= valid) byte &= 0x0Fu;   // pad nibble of an odd tail
-            dst[jj] = uint8_t(byte);
+      for (int i = 0; i < kQuantBatch; ++i) {
+        uint32_t m = absmax_bits8(v[i]);
+        m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
+        bm[i] = m;
+        gm = max(gm, m);
+      }
+      uint32_t my_bm = bm[0];   // this lane's pass: i == j
+#pragma unroll
+      for (int i = 1; i < kQuantBatch; ++i) my_bm = (j == i) ? bm[i] : my_bm;
+      keep_s[warp][b * 32 + j * 4 + (lane >> 3)] = my_bm;   // block 4 i + lane / 8 of the batch
+      const float my_c1 = __uint_as_float(my_bm << 16);
+      // 16 / scale1 must stay a finite normal number: scale1 in [2^-122, 2^125]
+      const bool normal = (my_c1 >= 0x1p-122f && my_c1 <= 0x1p125f) || my_c1 == 0.0f;
+      const float my_inv = (my_c1 == 0.0f) ? 0.0f : (normal ? __frcp_rn(my_c1) : 0.0f);
+      const bool fast = __all_sync(0xffffffffu, normal);
+      const bool full = e_first + kQuantBatch * kPassElems <= p.numel;
+      if (fast && full && !p.exact) {
+        // the common case in straight-line code: every block of the batch
+        // has a normal (or zero) scale1, no element is past the end and the
+        // table's thresholds are not dyadic.  A zero block has inv16 = 0, so
+        // x16 = 0 and its codes come out as the 0.0 code of the table.
+        const float my_inv16 = my_inv * 16.0f;
+        uint32_t* dst = reinterpret_cast<uint32_t*>(p.packed + (e_first >> 1)) + lane;
+#pragma unroll
+        for (int i = 0; i < kQuantBatch; ++i) {
+          const float inv16 = __shfl_sync(0xffffffffu, my_inv16, (lane & ~7) | i);
+          __stcs(dst + i * 32, quantize8<0>(cells, cells_biased, v[i], inv16, 1.0f, 0.0f, p.k8, p.k65536));
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < kQuantBatch; ++i) {
+          const int64_t e0 = e_first + int64_t(i) * kPassElems + lane * 8;
+          const float inv = __shfl_sync(0xffffffffu, my_inv, (lane & ~7) | i);
+          if (e0 >= p.numel) continue;
+          const float c1 = __uint_as_float(bm[i] << 16);
+          uint32_t q8;
+          if (c1 == 0.0f) {
+            q8 = p.zero8;                            // all-zero block: the 0.0 code
+          } else if (p.exact) {                      // dyadic thresholds: exact comparisons
+            const bool nrm = c1 >= 0x1p-122f && c1 <= 0x1p125f;
+            const float pre = nrm ? 1.0f : ((c1 < 1.0f) ? 0x1p64f : 0x1p-64f);
+            q8 = quantize8<2>(cells, cells_biased, v[i], __frcp_rn(c1 * pre) * 16.0f, pre, c1 * pre);
+          } else if (fast) {
+            q8 = quantize8<0>(cells, cells_biased, v[i], inv * 16.0f, 1.0f, c1, p.k8, p.k65536);
+          } else if (c1 >= 0x1p-122f && c1 <= 0x1p125f) {
+            q8 = quantize8<1>(cells, cells_biased, v[i], __frcp_rn(c1) * 16.0f, 1.0f, c1);
+          } else {                                   // keep 16/c1 a normal number
+            const float pre = (c1 < 1.0f) ? 0x1p64f : 0x1p-64f;
+            q8 = quantize8<1>(cells, cells_biased, v[i], __frcp_rn(c1 * pre) * 16.0f, pre, c1);
+          }
+          uint8_t* dst = p.packed + (e0 >> 1);
+          if (e0 + 8 <= p.numel) {
+            __stcs(reinterpret_cast<unsigned int*>(dst), q8);
+          } else {
+            const int valid = int(p.numel - e0);
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+              if (2 * jj < valid) {
+                uint32_t byte = (q8 >> (8 * jj)) & 0xFFu;
+                if (2 * jj + 1 >= valid) byte &= 0x0Fu;   // pad nibble of an odd tail
+                dst[jj] = uint8_t(byte);
+              }
+            }
           }
         }
       }
+#pragma unroll
+      for (int i = 0; i < kQuantBatch; ++i) v[i] = vn[i];
     }
 
-    // second level: fp32 scale2 for the group (needs every warp's maximum),
-    // then the 8-bit codes of scale1 / scale2 (lane j < kQuantIters of each
-    // block group stores its block's)
-    __syncthreads();
-    {   // the group maximum over the warps' maxima, four per 16-byte load
-      const uint4* wm = reinterpret_cast<const uint4*>(warp_max[parity]);
-      gm = 0;
+    // second level: fp32 scale2 of the group (the four warps' maxima), then
+    // the 8-bit codes of scale1 / scale2 of this warp's 64 blocks
 #pragma unroll
-      for (int w = 0; w < kQuantThreads / 128; ++w) {
-        const uint4 q = wm[w];
-        gm = max(gm, max(max(q.x, q.y), max(q.z, q.w)));
-      }
-    }
+    for (int o = 8; o < 32; o <<= 1) gm = max(gm, __shfl_xor_sync(0xffffffffu, gm, o));
+    if (lane == 0) warp_max[parity][warp] = gm;
+    __syncthreads();
+    gm = max(max(warp_max[parity][0], warp_max[parity][1]), max(warp_max[parity][2], warp_max[parity][3]));
     if (gm >= 0x7F80u) bad = 1;
     const float gmax = __uint_as_float(gm << 16);
     const float s2 = __fdiv_rn(gmax, p.dq == kDqU8 ? 255.0f : 448.0f);
     if (tid == 0 && p.dq != kDqNone) p.c2[g] = s2;
-    if (j < kQuantIters) {
-      const int64_t b = g * kGroup + int64_t(j) * (kQuantThreads / 8) + (tid >> 3);
-      if (b < nblk_total) {
+#pragma unroll
+    for (int k = 0; k < kWarpBatches; ++k) {
+      const int64_t blk = g * kGroup + int64_t(warp) * (kWarpBatches * 32) + k * 32 + lane;
+      const float c1 = __uint_as_float(keep_s[warp][k * 32 + lane] << 16);
+      if (blk < nblk_total) {
         if (p.dq == kDqNone) {
-          reinterpret_cast<float*>(p.c1q)[b] = my_c1;
-        } else if (my_c1 == 0.0f) {
-          p.c1q[b] = 0;
+          reinterpret_cast<float*>(p.c1q)[blk] = c1;
+        } else if (c1 == 0.0f) {
+          p.c1q[blk] = 0;
         } else {
-          const float t = __fdiv_rn(my_c1, s2);
-          p.c1q[b] = uint8_t(p.dq == kDqU8 ? min(__float2uint_rn(t), 255u) : f32_to_e4m3_satfinite(t));
+          const float t = __fdiv_rn(c1, s2);
+          p.c1q[blk] = uint8_t(p.dq == kDqU8 ? min(__float2uint_rn(t), 255u) : f32_to_e4m3_satfinite(t));
         }
       }
     }
-#pragma unroll
-    for (int i = 0; i < kQuantIters; ++i) v[i] = vn[i];
+    __syncwarp();   // keep_s is rewritten by other lanes in the next group
   }
   if (bad && p.status != nullptr && tid == 0) atomicOr(p.status, kStatusNonfinite);
 }
 
 // ---------------------------------------------------------------- dequantize
 struct DequantArgs {
+  CUtensorMap tm_out;   // out as [nfull rows x 64] 2-byte, box {64, 32}, 128-byte swizzle
   const uint8_t* packed;
   const uint8_t* c1q;   // first-level constants (bytes, or fp32 for kDqNone)
   const float* c2;
   uint16_t* out;
   int64_t numel;
+  int64_t nfull;        // complete 64-weight blocks
   int dq;               // DqFormat
   int f16;              // output fp16 (else bf16)
-  float code[16];
+  CodeTable code;
+  ShiftMuls km;
 };
 
-// Eight lanes per 64-weight block, eight weights (four packed bytes) per
-// lane and unit, so that every warp load covers 128 contiguous packed bytes
-// and every warp store 512 contiguous bytes of bf16; four units per lane per
-// iteration keep enough bytes in flight.  code[q] comes from a 16-word shared
-// table (one bank per entry), times the block scale in fp32, rounded to bf16.
-constexpr int kDqUnits = 4;
-__global__ void __launch_bounds__(256) nf4_dequant_kernel(const __grid_constant__ DequantArgs p) {
-  __shared__ float code_s[16];
-  if (threadIdx.x < 16) code_s[threadIdx.x] = p.code[threadIdx.x];
-  __syncthreads();
-  const int lane = threadIdx.x & 31;
-  const int64_t nunits = p.numel / 8;                        // complete 8-weight units
-  const int64_t warp_id = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
-  for (int64_t base = warp_id * (32 * kDqUnits); base < nunits; base += nwarps * (32 * kDqUnits)) {
-    uint32_t w[kDqUnits];
-    float s1[kDqUnits];
-#pragma unroll
-    for (int i = 0; i < kDqUnits; ++i) {
-      const int64_t u = base + i * 32 + lane;
-      if (u < nunits) {
-        w[i] = __ldcs(reinterpret_cast<const unsigned int*>(p.packed) + u);
-        s1[i] = block_scale(p.dq, p.c1q, p.c2, u >> 3);
-      } else {
-        w[i] = 0u;
-        s1[i] = 0.0f;
-      }
+// One lane per 64-weight block: the lane loads the block's 32 packed bytes and
+// its constants, forms the block's 16 values once (code[q] * scale1 in fp32,
+// rounded to bf16 or fp16) and looks the 64 codes up with byte permutes.  A
+// warp's 32 blocks (4 KB of output, contiguous in memory) are written into
+// shared memory as a 32 x 128-byte tile in the 128-byte swizzle (lane l's
+// 16-byte chunk k at position k ^ (l mod 8): no bank conflicts) and leave by
+// one TMA store, which also clips the last, partial tile.  The next blocks'
+// bytes are loaded before the current ones are decoded.
+constexpr int kDqWarps = 8;
+__global__ void __launch_bounds__(kDqWarps * 32, 4) nf4_dequant_kernel(const __grid_constant__ DequantArgs p) {
+  __shared__ __align__(1024) uint4 stage[kDqWarps][32 * 8];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint4* st = stage[warp];
+  const int64_t nchunks = (p.nfull + 31) / 32;
+  const int64_t nw = int64_t(gridDim.x) * kDqWarps;
+  const bool h = p.f16 != 0;
+  auto load = [&](int64_t ch, uint4& a, uint4& b, uint32_t& q, float& s2) {
+    const int64_t blk = ch * 32 + lane;
+    if (ch < nchunks && blk < p.nfull) {
+      const uint4* src = reinterpret_cast<const uint4*>(p.packed) + blk * 2;
+      a = __ldcs(src);
+      b = __ldcs(src + 1);
+      load_scale_parts(p.dq, p.c1q, p.c2, blk, q, s2);
+    } else {
+      a = b = make_uint4(0u, 0u, 0u, 0u);
+      q = 0u;
+      s2 = 0.0f;
     }
+  };
+  int64_t ch = int64_t(blockIdx.x) * kDqWarps + warp;
+  uint4 a, b;
+  uint32_t q;
+  float s2;
+  load(ch, a, b, q, s2);
+  for (; ch < nchunks; ch += nw) {
+    uint4 na, nb;
+    uint32_t nq;
+    float ns2;
+    load(ch + nw, na, nb, nq, ns2);
+    const BlockTable t = make_table(p.code, scale_from_parts(p.dq, q, s2), h);
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    // the previous tile's TMA store must have read the staging buffer
+    if (lane == 0) bulk_wait_read_all();
+    __syncwarp();
 #pragma unroll
-    for (int i = 0; i < kDqUnits; ++i) {
-      const int64_t u = base + i * 32 + lane;
-      if (u >= nunits) break;
-      const bool h = p.f16 != 0;
+    for (int k = 0; k < 8; ++k) {   // 16-byte chunk k: weights 8k .. 8k + 7
       uint4 o;
-      o.x = pack2(h, code_s[w[i] & 0xFu] * s1[i], code_s[(w[i] >> 4) & 0xFu] * s1[i]);
-      o.y = pack2(h, code_s[(w[i] >> 8) & 0xFu] * s1[i], code_s[(w[i] >> 12) & 0xFu] * s1[i]);
-      o.z = pack2(h, code_s[(w[i] >> 16) & 0xFu] * s1[i], code_s[(w[i] >> 20) & 0xFu] * s1[i]);
-      o.w = pack2(h, code_s[(w[i] >> 24) & 0xFu] * s1[i], code_s[w[i] >> 28] * s1[i]);
-      __stcs(reinterpret_cast<uint4*>(p.out) + u, o);
+      lookup8(t, w[k], p.km, o.x, o.y, o.z, o.w);
+      st[lane * 8 + (k ^ (lane & 7))] = o;
     }
+    fence_proxy_async_smem();   // generic-proxy writes, read next by the TMA engine
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(&p.tm_out, st, 0, int32_t(ch * 32));
+      bulk_commit();
+    }
+    a = na;
+    b = nb;
+    q = nq;
+    s2 = ns2;
   }
-  // ragged tail: the last numel % 8 weights, one thread
+  if (lane == 0) bulk_wait_all();
+  // the last numel % 64 weights (a partial block), one thread
   if (blockIdx.x == 0 && threadIdx.x == 0) {
-    for (int64_t e = nunits * 8; e < p.numel; ++e) {
-      const float s = block_scale(p.dq, p.c1q, p.c2, e / kBlock);
+    for (int64_t e = p.nfull * kBlock; e < p.numel; ++e) {
+      const float sc = block_scale(p.dq, p.c1q, p.c2, e / kBlock);
       const uint32_t byte = p.packed[e >> 1];
-      const uint32_t q = (e & 1) ? (byte >> 4) : (byte & 0xFu);
-      p.out[e] = uint16_t(pack2(p.f16 != 0, code_s[q] * s, 0.0f) & 0xFFFFu);
+      const uint32_t c = (e & 1) ? (byte >> 4) : (byte & 0xFu);
+      p.out[e] = uint16_t(pack2(h, p.code.v[c] * sc, 0.0f) & 0xFFFFu);
     }
   }
 }
@@ -388,10 +453,12 @@ cudaError_t launch_quantize(const uint16_t* W, int64_t numel, int quant_type, in
   a.dq = dq;
   a.zero8 = 0x11111111u * uint32_t(zero_code(quant_type));
   a.exact = quant_type == kQuantInt4 ? 1 : 0;
+  a.k8 = 8u;
+  a.k65536 = 65536u;
   const Codebook& cb = host_codebook(quant_type);
   for (int i = 0; i < 15; ++i) a.thr[i] = cb.thr[i];
   int64_t grid = a.ngroups;
-  const int64_t cap = int64_t(num_sms) * 2;
+  const int64_t cap = int64_t(num_sms) * 5;
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
   nf4_quantize_kernel<<<dim3(unsigned(grid)), kQuantThreads, 0, stream>>>(a);
@@ -406,24 +473,31 @@ cudaError_t launch_dequant(const uint8_t* packed, const uint8_t* c1, const float
   a.c2 = c2;
   a.out = out;
   a.numel = numel;
+  a.nfull = numel / kBlock;
   a.dq = dq;
   a.f16 = f16;
   const Codebook& cb = host_codebook(quant_type);
-  for (int i = 0; i < 16; ++i) a.code[i] = cb.code[i];
-  const int64_t nunits = numel / 8;
-  int64_t grid = (nunits / (32 * kDqUnits) + 7) / 8;   // 8 warps per CTA
+  for (int i = 0; i < 16; ++i) a.code.v[i] = cb.code[i];
+  a.km = make_shift_muls();
+  if (a.nfull >= (int64_t(1) << 31)) return cudaErrorInvalidValue;   // tile rows are int32 coordinates
+  if (a.nfull > 0 && !encode_tmap_2d(&a.tm_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, 64, uint64_t(a.nfull), 128, 64,
+                                     32, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  int64_t grid = (a.nfull + 32 * kDqWarps - 1) / (32 * kDqWarps);
   // one wave: no more CTAs than fit on the SMs at once (the loop is
   // grid-stride, so any grid covers the weight), or a partial second wave
   // of short-lived CTAs would add a tail to every call
   static const int per_sm = [] {
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, nf4_dequant_kernel, 256, 0) != cudaSuccess || n < 1) n = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, nf4_dequant_kernel, kDqWarps * 32, 0) != cudaSuccess ||
+        n < 1)
+      n = 1;
     return n;
   }();
   const int64_t cap = int64_t(num_sms) * per_sm;
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
-  nf4_dequant_kernel<<<dim3(unsigned(grid)), 256, 0, stream>>>(a);
+  nf4_dequant_kernel<<<dim3(unsigned(grid)), kDqWarps * 32, 0, stream>>>(a);
   return cudaGetLastError();
 }
 

@@ -138,7 +138,8 @@ nf4_status nf4_dequant_bf16(nf4_weight w, uint16_t* out, void* stream);
 /* Dequantization of any storage format into a compute type (QLORA_BF16 or
  * QLORA_F16): scale1' = the FP32 scale1, or fp32(decoded 8-bit code *
  * scale2); out = round(fp32(code * scale1')) to the compute type.
- * nf4_dequant_bf16(w, out) is nf4_dequant(w, QLORA_BF16, out). */
+ * nf4_dequant_bf16(w, out) is nf4_dequant(w, QLORA_BF16, out).
+ * NF4_ERR_UNSUPPORTED above 2^37 weights (beyond any one GPU's memory). */
 nf4_status nf4_dequant(nf4_weight w, int32_t dtype, uint16_t* out, void* stream);
 
 /* Merge the adapter into the frozen weight for serving ([P2] §2.5: merged
