@@ -155,13 +155,29 @@ __device__ __forceinline__ uint32_t quantize8(const uint2* cells, uint32_t cells
 __device__ __forceinline__ __nv_bfloat162 as_bf162(uint32_t u) {
   return *reinterpret_cast<const __nv_bfloat162*>(&u);
 }
-// Largest |w| of 8 bf16 as a bf16 bit pattern (NaN propagates, so Inf/NaN
-// inputs give a pattern >= 0x7F80).
-__device__ __forceinline__ uint32_t absmax_bits8(const uint4& v) {
+// Largest |w| of each half of 8 bf16 as a bf16x2 pattern (NaN propagates, so
+// Inf/NaN inputs give a pattern >= 0x7F80 in that half).
+__device__ __forceinline__ uint32_t absmax_pair8(const uint4& v) {
   const __nv_bfloat162 m = __hmax2_nan(__hmax2_nan(__habs2(as_bf162(v.x)), __habs2(as_bf162(v.y))),
                                        __hmax2_nan(__habs2(as_bf162(v.z)), __habs2(as_bf162(v.w))));
-  const uint32_t u = *reinterpret_cast<const uint32_t*>(&m);
-  return max(u & 0xFFFFu, u >> 16);
+  return *reinterpret_cast<const uint32_t*>(&m);
+}
+__device__ __forceinline__ uint32_t hmax2_bits(uint32_t a, uint32_t b) {
+  const __nv_bfloat162 m = __hmax2_nan(as_bf162(a), as_bf162(b));
+  return *reinterpret_cast<const uint32_t*>(&m);
+}
+// Block maxima of two passes at once: the per-lane maxima of passes i and
+// i + 1 are folded into one bf16x2 word (max of pass i in the low half, of
+// pass i + 1 in the high half) and reduced over the block's 8 lanes with one
+// set of shuffles.  All values are |w| patterns (non-negative), so the bf16
+// maximum orders them as their bit patterns do.
+__device__ __forceinline__ uint32_t block_absmax2(const uint4& vi, const uint4& vj) {
+  const uint32_t mi = absmax_pair8(vi), mj = absmax_pair8(vj);
+  uint32_t m = hmax2_bits(prmt(mi, mj, 0x5410u), prmt(mi, mj, 0x7632u));
+  m = hmax2_bits(m, __shfl_xor_sync(0xffffffffu, m, 1));
+  m = hmax2_bits(m, __shfl_xor_sync(0xffffffffu, m, 2));
+  m = hmax2_bits(m, __shfl_xor_sync(0xffffffffu, m, 4));
+  return m;
 }
 
 struct QuantArgs {
@@ -234,7 +250,7 @@ __global__ void __launch_bounds__(kQuantThreads, 5) nf4_quantize_kernel(const __
   uint4 v[kQuantBatch];
   if (g < p.ngroups) load_batch(p, batch_first(g, 0), v);
   for (int parity = 0; g < p.ngroups; g += gridDim.x, parity ^= 1) {
-    uint32_t gm = 0;
+    uint32_t gm2 = 0;   // group maximum so far, as a bf16x2 pattern
 #pragma unroll 1
     for (int b = 0; b < kWarpBatches; ++b) {
       const int64_t e_first = batch_first(g, b);
@@ -247,13 +263,11 @@ __global__ void __launch_bounds__(kQuantThreads, 5) nf4_quantize_kernel(const __
       // first level: absmax of each block (8 lanes x 8 weights)
       uint32_t bm[kQuantBatch];
 #pragma unroll
-      for (int i = 0; i < kQuantBatch; ++i) {
-        uint32_t m = absmax_bits8(v[i]);
-        m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-        m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
-        m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
-        bm[i] = m;
-        gm = max(gm, m);
+      for (int i = 0; i < kQuantBatch; i += 2) {
+        const uint32_t m = block_absmax2(v[i], v[i + 1]);
+        bm[i] = m & 0xFFFFu;
+        bm[i + 1] = m >> 16;
+        gm2 = hmax2_bits(gm2, m);
       }
       uint32_t my_bm = bm[0];   // this lane's pass: i == j
 #pragma unroll
@@ -321,6 +335,7 @@ __global__ void __launch_bounds__(kQuantThreads, 5) nf4_quantize_kernel(const __
 
     // second level: fp32 scale2 of the group (the four warps' maxima), then
     // the 8-bit codes of scale1 / scale2 of this warp's 64 blocks
+    uint32_t gm = max(gm2 & 0xFFFFu, gm2 >> 16);
 #pragma unroll
     for (int o = 8; o < 32; o <<= 1) gm = max(gm, __shfl_xor_sync(0xffffffffu, gm, o));
     if (lane == 0) warp_max[parity][warp] = gm;
