@@ -339,23 +339,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
     // A operand layouts: forward main steps K-major (rows of W), backward
     // main steps MN-major (columns of W), forward low-rank steps MN-major
     // (B^T by TMA), backward low-rank steps K-major (A by TMA).
-    const uint32_t idesc_k = make_idesc(128, bt, 0, 0, a.f16 != 0);
-    const uint32_t idesc_mn = make_idesc(128, bt, 1, 0, a.f16 != 0);
-    for (int64_t ks = 0; ks < nsteps; ++ks) {
-      const int sx = int(ks % SX);
-      // operand slot: forward main steps in the tensor-memory ring, every
-      // other step in the shared-memory ring (the forward's low-rank steps
-      // counted from the first of them)
-      const bool a_in_tmem = !BWD && kTmemA && ks < my_main;
-      const int64_t ls = (!BWD && kTmemA) ? ks - my_main : ks;
-      const int sa = a_in_tmem ? int(ks % SAT) : int(ls % SA);
-      const uint32_t aph = a_in_tmem ? uint32_t(ks / SAT) & 1u : uint32_t(ls / SA) & 1u;
-      if (!mbar_wait(&x_full[sx], uint32_t(ks / SX) & 1u, a.status, abort_flag)) break;
-      if (!mbar_wait(a_in_tmem ? &t_full[sa] : &a_full[sa], aph, a.status, abort_flag)) break;
-      tc_fence_after();
-      if (elect_one()) {
-        const uint32_t act_addr = smem_u32(act_s + sx * act_bytes);
-        const uint32_t a_addr = smem_u32(a_s + sa * 16384);
+    // One thread runs the whole loop, waits included: a warp that loops and
+    // elects a lane per step to issue the MMAs (with a warp sync after them)
+    // takes ~1000 cycles per step on this part, against ~550 for the four
+    // 128 x 256 x 16 MMAs themselves.  Ring slots and phases advance by one
+    // per step (the activation ring's size is not a power of two).
+    if (elect_one()) {
+      const uint32_t idesc_k = make_idesc(128, bt, 0, 0, a.f16 != 0);
+      const uint32_t idesc_mn = make_idesc(128, bt, 1, 0, a.f16 != 0);
+      const uint32_t act_base = smem_u32(act_s), a_base = smem_u32(a_s);
+      int sx = 0, st = 0, ss = 0;               // activation, tensor-memory and shared operand slots
+      uint32_t xph = 0, tph = 0, sph = 0;
+      for (int64_t ks = 0; ks < nsteps; ++ks) {
+        // operand slot: forward main steps in the tensor-memory ring, every
+        // other step in the shared-memory ring (the forward's low-rank steps
+        // counted from the first of them)
+        const bool a_in_tmem = !BWD && kTmemA && ks < my_main;
+        const int sa = a_in_tmem ? st : ss;
+        if (!mbar_wait(&x_full[sx], xph, a.status, abort_flag)) break;
+        if (!mbar_wait(a_in_tmem ? &t_full[sa] : &a_full[sa], a_in_tmem ? tph : sph, a.status, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t act_addr = act_base + uint32_t(sx) * act_bytes;
+        const uint32_t a_addr = a_base + uint32_t(sa) * 16384u;
         const bool a_mn = (ks < my_main) == BWD;
         const uint32_t idesc = a_mn ? idesc_mn : idesc_k;
 #pragma unroll
@@ -372,10 +377,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
         }
         mma_commit(&x_empty[sx]);
         mma_commit(a_in_tmem ? &t_empty[sa] : &a_empty[sa]);
+        if (++sx == SX) { sx = 0; xph ^= 1u; }
+        if (a_in_tmem) {
+          if (++st == SAT) { st = 0; tph ^= 1u; }
+        } else {
+          if (++ss == SA) { ss = 0; sph ^= 1u; }
+        }
       }
-      __syncwarp();
-    }
-    if (elect_one()) {
       mma_commit(accf);
       if (*abort_flag) mbar_drain(accf, 0);
     }
@@ -768,13 +776,14 @@ __global__ void __launch_bounds__(kSkinnyThreads, 2) skinny_gemm_kernel(const __
     }
     __syncwarp();
   } else if (warp == 1) {
-    const uint32_t idesc = make_idesc(128, rp, P.a_mn, P.b_mn, a.f16 != 0);
-    for (int64_t ks = 0; ks < nsteps; ++ks) {
-      const int s = int(ks % kSkinnyStages);
-      const uint32_t ph = uint32_t(ks / kSkinnyStages) & 1u;
-      if (!mbar_wait(&full[s], ph, a.status, abort_flag)) break;
-      tc_fence_after();
-      if (elect_one()) {
+    // one thread runs the whole MMA loop (see the fused kernel's issuer)
+    if (elect_one()) {
+      const uint32_t idesc = make_idesc(128, rp, P.a_mn, P.b_mn, a.f16 != 0);
+      int s = 0;
+      uint32_t ph = 0;
+      for (int64_t ks = 0; ks < nsteps; ++ks) {
+        if (!mbar_wait(&full[s], ph, a.status, abort_flag)) break;
+        tc_fence_after();
         const uint32_t aa = smem_u32(smem + s * stage_bytes);
         const uint32_t ba = aa + a_bytes;
 #pragma unroll
@@ -786,10 +795,8 @@ __global__ void __launch_bounds__(kSkinnyThreads, 2) skinny_gemm_kernel(const __
           mma_ss(tmem_base, ad, bd, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(&empty[s]);
+        if (++s == kSkinnyStages) { s = 0; ph ^= 1u; }
       }
-      __syncwarp();
-    }
-    if (elect_one()) {
       mma_commit(accf);
       if (*abort_flag) mbar_drain(accf, 0);
     }
