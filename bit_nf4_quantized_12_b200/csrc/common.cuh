@@ -193,6 +193,50 @@ NF4_DEV void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t 
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// The four MMAs of one 64-wide K step (K = 16 each) in one statement: A from
+// tensor memory at columns a, a + 8, a + 16, a + 24, or from shared memory
+// with its descriptor's address field advanced by a_inc per MMA; B's
+// descriptor address field advanced by 2 (32 bytes) per MMA.  The address
+// field (bits 0-13, address / 16) never carries into the next field for
+// shared addresses below 256 KB.  The first MMA accumulates when acc != 0,
+// the other three always.  One statement keeps the issuing thread's
+// instruction count per step low: its loop paces the tensor pipe.
+NF4_DEV void mma_ts_k64(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p, t;\n\t.reg .b32 bl, bh, b1l, b2l, b3l, a1, a2, a3;\n\t.reg .b64 b1, b2, b3;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 t, %4, %4;\n\t"
+      "mov.b64 {bl, bh}, %2;\n\t"
+      "add.u32 b1l, bl, 2;\n\tadd.u32 b2l, bl, 4;\n\tadd.u32 b3l, bl, 6;\n\t"
+      "mov.b64 b1, {b1l, bh};\n\tmov.b64 b2, {b2l, bh};\n\tmov.b64 b3, {b3l, bh};\n\t"
+      "add.u32 a1, %1, 8;\n\tadd.u32 a2, %1, 16;\n\tadd.u32 a3, %1, 24;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, t;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], b2, %3, t;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a3], b3, %3, t;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(acc)
+      : "memory");
+}
+NF4_DEV void mma_ss_k64(uint32_t d_tmem, uint64_t a_desc, uint32_t a_inc, uint64_t b_desc, uint32_t b_inc,
+                        uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p, t;\n\t.reg .b32 al, ah, bl, bh, x1, x2, x3, y1, y2, y3;\n\t"
+      ".reg .b64 a1, a2, a3, b1, b2, b3;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "setp.eq.b32 t, %6, %6;\n\t"
+      "mov.b64 {al, ah}, %1;\n\tmov.b64 {bl, bh}, %3;\n\t"
+      "add.u32 x1, al, %2;\n\tadd.u32 x2, x1, %2;\n\tadd.u32 x3, x2, %2;\n\t"
+      "add.u32 y1, bl, %4;\n\tadd.u32 y2, y1, %4;\n\tadd.u32 y3, y2, %4;\n\t"
+      "mov.b64 a1, {x1, ah};\n\tmov.b64 a2, {x2, ah};\n\tmov.b64 a3, {x3, ah};\n\t"
+      "mov.b64 b1, {y1, bh};\n\tmov.b64 b2, {y2, bh};\n\tmov.b64 b3, {y3, bh};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %3, %5, p;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %5, t;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a2, b2, %5, t;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a3, b3, %5, t;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "r"(a_inc), "l"(b_desc), "r"(b_inc), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
 // 32 lanes x 32 columns of 32 bit from registers into tensor memory (thread i
 // of the warp -> lane base + i), then wait until the stores are done.
 NF4_DEV void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&v)[32]) {

@@ -347,7 +347,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
     if (elect_one()) {
       const uint32_t idesc_k = make_idesc(128, bt, 0, 0, a.f16 != 0);
       const uint32_t idesc_mn = make_idesc(128, bt, 1, 0, a.f16 != 0);
-      const uint32_t act_base = smem_u32(act_s), a_base = smem_u32(a_s);
+      // descriptors and tensor-memory addresses of slot 0; a slot adds its
+      // byte offset / 16 to a descriptor's address field
+      const uint64_t bdesc0 = make_sdesc_sw128(smem_u32(act_s), 16, 1024);
+      const uint64_t adesc0_k = make_sdesc_sw128(smem_u32(a_s), 16, 1024);
+      const uint64_t adesc0_mn = make_sdesc_sw128(smem_u32(a_s), 8192, 1024);
+      const uint32_t ta0 = tmem_base + a_tmem_col;
       int sx = 0, st = 0, ss = 0;               // activation, tensor-memory and shared operand slots
       uint32_t xph = 0, tph = 0, sph = 0;
       for (int64_t ks = 0; ks < nsteps; ++ks) {
@@ -359,21 +364,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
         if (!mbar_wait(&x_full[sx], xph, a.status, abort_flag)) break;
         if (!mbar_wait(a_in_tmem ? &t_full[sa] : &a_full[sa], a_in_tmem ? tph : sph, a.status, abort_flag)) break;
         tc_fence_after();
-        const uint32_t act_addr = act_base + uint32_t(sx) * act_bytes;
-        const uint32_t a_addr = a_base + uint32_t(sa) * 16384u;
-        const bool a_mn = (ks < my_main) == BWD;
-        const uint32_t idesc = a_mn ? idesc_mn : idesc_k;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bdesc = make_sdesc_sw128(act_addr + kk * 32, 16, 1024);
-          if (a_in_tmem) {   // 16 K-elements = 8 columns per MMA
-            mma_ts(tmem_base, tmem_base + a_tmem_col + uint32_t(sa) * 32u + uint32_t(kk) * 8u, bdesc, idesc,
-                   (ks > 0 || kk > 0) ? 1u : 0u);
-          } else {
-            const uint64_t adesc = a_mn ? make_sdesc_sw128(a_addr + kk * 2048, 8192, 1024)
-                                        : make_sdesc_sw128(a_addr + kk * 32, 16, 1024);
-            mma_ss(tmem_base, adesc, bdesc, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
-          }
+        const uint64_t bdesc = bdesc0 + uint32_t(sx) * (act_bytes >> 4);
+        const uint32_t acc = ks > 0 ? 1u : 0u;
+        if (a_in_tmem) {
+          mma_ts_k64(tmem_base, ta0 + uint32_t(sa) * 32u, bdesc, idesc_k, acc);
+        } else {
+          const bool a_mn = (ks < my_main) == BWD;   // backward main steps: MN-major operand
+          mma_ss_k64(tmem_base, (a_mn ? adesc0_mn : adesc0_k) + uint32_t(sa) * 1024u, a_mn ? 128u : 2u, bdesc, 2u,
+                     a_mn ? idesc_mn : idesc_k, acc);
         }
         mma_commit(&x_empty[sx]);
         mma_commit(a_in_tmem ? &t_empty[sa] : &a_empty[sa]);
@@ -786,14 +784,8 @@ __global__ void __launch_bounds__(kSkinnyThreads, 2) skinny_gemm_kernel(const __
         tc_fence_after();
         const uint32_t aa = smem_u32(smem + s * stage_bytes);
         const uint32_t ba = aa + a_bytes;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t ad = P.a_mn ? make_sdesc_sw128(aa + kk * 2048, 8192, 1024)
-                                     : make_sdesc_sw128(aa + kk * 32, 16, 1024);
-          const uint64_t bd = P.b_mn ? make_sdesc_sw128(ba + kk * 2048, 8192, 1024)
-                                     : make_sdesc_sw128(ba + kk * 32, 16, 1024);
-          mma_ss(tmem_base, ad, bd, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
-        }
+        mma_ss_k64(tmem_base, make_sdesc_sw128(aa, P.a_mn ? 8192 : 16, 1024), P.a_mn ? 128u : 2u,
+                   make_sdesc_sw128(ba, P.b_mn ? 8192 : 16, 1024), P.b_mn ? 128u : 2u, idesc, ks > 0 ? 1u : 0u);
         mma_commit(&empty[s]);
         if (++s == kSkinnyStages) { s = 0; ph ^= 1u; }
       }
