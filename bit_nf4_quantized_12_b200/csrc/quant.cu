@@ -41,14 +41,18 @@ namespace {
 
 // A CTA of four warps quantizes one group (16384 weights) at a time.  A pass
 // is one 16-byte load per lane: 256 weights, four blocks of 8 lanes each.
-// Warp w takes passes 16 w .. 16 w + 15 of the group as two batches of 8,
-// and within a batch lane j of each 8-lane block group owns pass j (its
-// block's reciprocal is taken once and shuffled to the other lanes).
+// Warp w takes passes 16 w .. 16 w + 15 of the group as four batches of 4,
+// and within a batch lane j < 4 of each 8-lane block group owns pass j (its
+// block's reciprocal is taken once and shuffled to the other lanes).  Small
+// batches keep a warp's registers low enough for 8 CTAs per SM, so that the
+// 1024 groups of a 4096 x 4096 weight run in one round.
 constexpr int kQuantWarps = 4;
 constexpr int kQuantThreads = kQuantWarps * 32;
-constexpr int kQuantBatch = 8;                                      // passes per batch
+constexpr int kQuantBatch = 4;                                      // passes per batch
 constexpr int kPassElems = 32 * 8;                                  // weights per pass
-constexpr int kWarpBatches = kGroupElems / (kPassElems * kQuantBatch * kQuantWarps);   // 2
+constexpr int kWarpBatches = kGroupElems / (kPassElems * kQuantBatch * kQuantWarps);   // 4
+constexpr int kWarpBlocks = kWarpBatches * kQuantBatch * 4;         // blocks per warp and group: 64
+constexpr int kQuantCtasPerSm = 8;
 static_assert(kWarpBatches * kPassElems * kQuantBatch * kQuantWarps == kGroupElems, "whole batches per group");
 constexpr int kCells = 33;           // cells of 16 x: floor(16 x) = -16 .. 16
 
@@ -196,7 +200,7 @@ struct QuantArgs {
 };
 
 // Batch b (0 .. kWarpBatches - 1) of this warp in group g: passes
-// P = (kWarpBatches w + b) 8 + i for i = 0..7; pass P covers weights
+// P = (kWarpBatches w + b) 4 + i for i = 0..3; pass P covers weights
 // P * 256 + lane * 8 .. + 7 of the group.  Elements past the end read as 0.
 __device__ __forceinline__ int64_t batch_first(int64_t g, int b) {
   const int warp = threadIdx.x >> 5;
@@ -230,11 +234,11 @@ __device__ __forceinline__ void load_batch(const QuantArgs& p, int64_t e_first, 
 // 4-bit codes depend only on their own block's absmax, so they are written
 // before the group's maximum is known; the four warps then meet once per
 // group for scale2 and each writes the 8-bit codes of its own 64 blocks.
-__global__ void __launch_bounds__(kQuantThreads, 5) nf4_quantize_kernel(const __grid_constant__ QuantArgs p) {
+__global__ void __launch_bounds__(kQuantThreads, kQuantCtasPerSm) nf4_quantize_kernel(const __grid_constant__ QuantArgs p) {
   __shared__ uint2 cells[kCells];
   __shared__ float thr_s[16];
   __shared__ uint32_t warp_max[2][kQuantWarps];
-  __shared__ uint32_t keep_s[kQuantWarps][kWarpBatches * 32];   // block maxima, block order within the warp
+  __shared__ uint32_t keep_s[kQuantWarps][kWarpBlocks];   // block maxima, block order within the warp
   if (threadIdx.x < 15) thr_s[threadIdx.x] = p.thr[threadIdx.x];
   __syncthreads();
   build_cells(cells, thr_s);
@@ -269,10 +273,11 @@ __global__ void __launch_bounds__(kQuantThreads, 5) nf4_quantize_kernel(const __
         bm[i + 1] = m >> 16;
         gm2 = hmax2_bits(gm2, m);
       }
-      uint32_t my_bm = bm[0];   // this lane's pass: i == j
+      uint32_t my_bm = bm[0];   // this lane's pass: i == j (lanes j >= 4: pass 0, unused)
 #pragma unroll
       for (int i = 1; i < kQuantBatch; ++i) my_bm = (j == i) ? bm[i] : my_bm;
-      keep_s[warp][b * 32 + j * 4 + (lane >> 3)] = my_bm;   // block 4 i + lane / 8 of the batch
+      if (j < kQuantBatch)   // block 4 j + lane / 8 of the batch
+        keep_s[warp][b * (kQuantBatch * 4) + j * 4 + (lane >> 3)] = my_bm;
       const float my_c1 = __uint_as_float(my_bm << 16);
       // 16 / scale1 must stay a finite normal number: scale1 in [2^-122, 2^125]
       const bool normal = (my_c1 >= 0x1p-122f && my_c1 <= 0x1p125f) || my_c1 == 0.0f;
@@ -346,8 +351,8 @@ __global__ void __launch_bounds__(kQuantThreads, 5) nf4_quantize_kernel(const __
     const float s2 = __fdiv_rn(gmax, p.dq == kDqU8 ? 255.0f : 448.0f);
     if (tid == 0 && p.dq != kDqNone) p.c2[g] = s2;
 #pragma unroll
-    for (int k = 0; k < kWarpBatches; ++k) {
-      const int64_t blk = g * kGroup + int64_t(warp) * (kWarpBatches * 32) + k * 32 + lane;
+    for (int k = 0; k < kWarpBlocks / 32; ++k) {
+      const int64_t blk = g * kGroup + int64_t(warp) * kWarpBlocks + k * 32 + lane;
       const float c1 = __uint_as_float(keep_s[warp][k * 32 + lane] << 16);
       if (blk < nblk_total) {
         if (p.dq == kDqNone) {
@@ -473,7 +478,7 @@ cudaError_t launch_quantize(const uint16_t* W, int64_t numel, int quant_type, in
   const Codebook& cb = host_codebook(quant_type);
   for (int i = 0; i < 15; ++i) a.thr[i] = cb.thr[i];
   int64_t grid = a.ngroups;
-  const int64_t cap = int64_t(num_sms) * 5;
+  const int64_t cap = int64_t(num_sms) * kQuantCtasPerSm;
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
   nf4_quantize_kernel<<<dim3(unsigned(grid)), kQuantThreads, 0, stream>>>(a);
