@@ -124,21 +124,29 @@ __device__ __forceinline__ uint32_t classify_exact(const uint2* cells, float x16
 // inv16 = 16 / scale1 (of the weights first scaled by pre, a power of two,
 // on the careful path for extreme or non-finite blocks); c1 = scale1 * pre.
 // MODE 0: fast cells (NF4 blocks with a normal scale1); 1: clamped cells (any
-// input); 2: exact comparison (dyadic thresholds).  km holds runtime copies
-// of 8 and 2^16, so that those products stay integer multiply-adds.
+// input); 2: exact comparison (dyadic thresholds).  k holds runtime copies of
+// 8, 16, 256 and 2^16, so that those products stay integer multiply-adds on
+// the FMA pipe (the integer pipe carries the rest of the classification).
+struct PackMuls {
+  uint32_t k8, k16, k256, k65536;
+};
 template <int MODE>
 __device__ __forceinline__ uint32_t quantize8(const uint2* cells, uint32_t cells_biased, const uint4& v,
-                                              float inv16, float pre, float c1, uint32_t k8 = 8u,
-                                              uint32_t k65536 = 65536u) {
+                                              float inv16, float pre, float c1,
+                                              const PackMuls& k = PackMuls{8u, 16u, 256u, 65536u}) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   uint32_t out = 0;
-  if constexpr (MODE == 0) {   // each byte's two codes ORed in at fixed positions: no serial chain
+  if constexpr (MODE == 0) {
+    // byte j = lo + 16 hi; bytes 0-1 and 2-3 joined by x 256, the halves by
+    // x 2^16: seven multiply-adds for the eight codes, no serial chain
+    uint32_t b[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const uint32_t lo = classify_fast(cells_biased, __uint_as_float(mad_lo(w[j], k65536, 0u)) * inv16, k8);
-      const uint32_t hi = classify_fast(cells_biased, bf16hi_to_f32(w[j]) * inv16, k8);
-      out |= (lo | (hi << 4)) << (8 * j);
+      const uint32_t lo = classify_fast(cells_biased, __uint_as_float(mad_lo(w[j], k.k65536, 0u)) * inv16, k.k8);
+      const uint32_t hi = classify_fast(cells_biased, bf16hi_to_f32(w[j]) * inv16, k.k8);
+      b[j] = mad_lo(hi, k.k16, lo);
     }
+    out = mad_lo(mad_lo(b[3], k.k256, b[2]), k.k65536, mad_lo(b[1], k.k256, b[0]));
   } else {
 #pragma unroll
     for (int j = 3; j >= 0; --j) {
@@ -195,7 +203,7 @@ struct QuantArgs {
   int dq;              // DqFormat
   int exact;           // exact comparisons (tables with dyadic thresholds)
   uint32_t zero8;      // eight nibbles of the table's 0.0 code (all-zero blocks)
-  uint32_t k8, k65536; // 8 and 2^16 (runtime values: see quantize8)
+  PackMuls km;          // 8, 16, 256 and 2^16 as runtime values (see quantize8)
   float thr[15];
 };
 
@@ -294,7 +302,7 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantCtasPerSm) nf4_quantize_k
 #pragma unroll
         for (int i = 0; i < kQuantBatch; ++i) {
           const float inv16 = __shfl_sync(0xffffffffu, my_inv16, (lane & ~7) | i);
-          __stcs(dst + i * 32, quantize8<0>(cells, cells_biased, v[i], inv16, 1.0f, 0.0f, p.k8, p.k65536));
+          __stcs(dst + i * 32, quantize8<0>(cells, cells_biased, v[i], inv16, 1.0f, 0.0f, p.km));
         }
       } else {
 #pragma unroll
@@ -311,7 +319,7 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantCtasPerSm) nf4_quantize_k
             const float pre = nrm ? 1.0f : ((c1 < 1.0f) ? 0x1p64f : 0x1p-64f);
             q8 = quantize8<2>(cells, cells_biased, v[i], __frcp_rn(c1 * pre) * 16.0f, pre, c1 * pre);
           } else if (fast) {
-            q8 = quantize8<0>(cells, cells_biased, v[i], inv * 16.0f, 1.0f, c1, p.k8, p.k65536);
+            q8 = quantize8<0>(cells, cells_biased, v[i], inv * 16.0f, 1.0f, c1, p.km);
           } else if (c1 >= 0x1p-122f && c1 <= 0x1p125f) {
             q8 = quantize8<1>(cells, cells_biased, v[i], __frcp_rn(c1) * 16.0f, 1.0f, c1);
           } else {                                   // keep 16/c1 a normal number
@@ -473,8 +481,7 @@ cudaError_t launch_quantize(const uint16_t* W, int64_t numel, int quant_type, in
   a.dq = dq;
   a.zero8 = 0x11111111u * uint32_t(zero_code(quant_type));
   a.exact = quant_type == kQuantInt4 ? 1 : 0;
-  a.k8 = 8u;
-  a.k65536 = 65536u;
+  a.km = PackMuls{8u, 16u, 256u, 65536u};
   const Codebook& cb = host_codebook(quant_type);
   for (int i = 0; i < 15; ++i) a.thr[i] = cb.thr[i];
   int64_t grid = a.ngroups;
