@@ -406,9 +406,10 @@ nf4_status qlora_linear_bwd_ex(int32_t dtype, const uint16_t* dY, const uint16_t
   // Launch order and overlap: the first kernel waits for all earlier work of
   // the stream; each later one is a programmatic dependent of the one before.
   // G waits for the T recompute (both write the hi/lo buffer).  The fused
-  // GEMM waits for G at its start and then lets dA and dB start: they read
-  // only G and the inputs, so they fill the SMs the GEMM's last wave leaves
-  // idle, and wait for the GEMM only before they exit.
+  // GEMM starts its main product (dY Wd) while G is still running and waits
+  // for G before its low-rank steps; it lets dA and dB start once G is
+  // complete: they read only G and the inputs, so they fill the SMs the
+  // GEMM's last wave leaves idle, and wait for the GEMM only before they exit.
   const uint16_t* Tin = T;
   bool after_kernel = false;
   sa.pdl_mode = kPdlWaitFirst;
@@ -433,7 +434,7 @@ nf4_status qlora_linear_bwd_ex(int32_t dtype, const uint16_t* dY, const uint16_t
   ga.act = dYa; ga.lora_w = A; ga.lora_act = hilo; ga.out = dX;
   ga.ld_act = ldn; ga.ld_lw = r; ga.packed_bytes = packed_bytes_of(N * K);
   ga.status = status;
-  ga.pdl_mode = kPdlWaitFirst;
+  ga.pdl_mode = kPdlWaitLowRank;
   ga.quant_type = w.quant_type; ga.dq = w.double_quant; ga.f16 = f16;
   if (launch_nf4_gemm(plan_nf4_gemm(1, M, N, K, r, sms), ga, strm, true) != cudaSuccess) return NF4_ERR_CUDA;
 

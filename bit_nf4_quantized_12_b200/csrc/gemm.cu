@@ -272,7 +272,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   if (a.pdl_mode == kPdlWaitFirst) griddep_wait();
-  griddep_launch();
+  if (a.pdl_mode != kPdlWaitLowRank || my_lora == 0) griddep_launch();
 
   if (warp == 0) {
     // ------------------------------------------------------------ X producer
@@ -314,6 +314,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) nf4_gemm_kernel(const __grid_
       }
     }
     __syncwarp();
+  } else if (warp == 2) {
+    // A CTA with low-rank steps lets the next kernel start only once the
+    // previous one is complete: in the backward that kernel (dA = X^T G)
+    // reads G from the previous one.  This warp is idle while the others run
+    // the main product, so the wait delays nothing.
+    if (a.pdl_mode == kPdlWaitLowRank && my_lora > 0 && lane == 0) {
+      griddep_wait();
+      griddep_launch();
+    }
   } else if (warp == 3) {
     // ------------------------------------------------------------ packed-W producer
     if (!RAGGED && elect_one()) {

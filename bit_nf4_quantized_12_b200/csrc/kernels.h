@@ -11,7 +11,8 @@ namespace nf4 {
 enum PdlMode : int {
   kPdlWaitFirst = 0,    // wait for the previous kernel, then let the next one start
   kPdlWaitLast = 1,     // let the next kernel start, work, wait before exiting
-  kPdlWaitLowRank = 2,  // fused GEMM: main product first, wait before the low-rank operand
+  kPdlWaitLowRank = 2,  // fused GEMM: main product first, wait before the low-rank operand; a CTA with
+                        // low-rank steps releases the next kernel only after that wait
 };
 
 // Quantize W (numel bf16) into the storage format (quant_type: table;
