@@ -7,35 +7,23 @@
 // merge the adapter back, then re-quantize for inference).
 //
 // Per element: wd = round(fp32(code[q] * scale1')) exactly as the standalone
-// dequantization; p = sum_j A[k,j] B[j,n] in fp32 on the tensor cores
-// (mma.sync m16n8k16, exact products, fp32 accumulation); v = fma(s, p, wd)
-// in fp32; W' = round(v) to the compute type.  The kernel is bound by HBM:
-// it reads 0.5 byte of packed code per weight and writes the 2-byte result;
-// the rank-r product adds 2 r flops per weight, which the tensor cores absorb.
+// dequantization; p = sum_j A[k,j] B[j,n] in fp32 on the tensor cores (exact
+// products, fp32 accumulation); v = fma(s, p, wd) in fp32; W' = round(v) to
+// the compute type.  The bound is HBM: 0.5 byte of packed code read and the
+// 2-byte result written per weight; the rank-r product adds 2 r flops per
+// weight, which the tensor cores absorb.
 //
-// Two kernels.  nf4_merge_frag_kernel takes the common shapes (K a multiple
-// of 64, so every NF4 block lies in one row; N and r multiples of 8, so rows
-// of A and B are 16-byte aligned); nf4_merge_kernel takes every other shape.
-//
-// nf4_merge_frag_kernel: one CTA per 64 (rows of W) x 128 (columns) tile, 4
-// warps, each owning 32 rows x 64 columns -- one NF4 block per row.  The
-// tile's B slice [r x 64], A slice [128 x r] and packed codes arrive by
-// cp.async; p is formed 16 rows at a time with ldmatrix (.trans for B, which
-// is stored rank-major) and mma.sync, and the epilogue runs on the MMA
-// fragments where they are: a thread holds columns 2c, 2c+1 of each 8-column
-// tile of a row, i.e. byte c of each of the block's eight packed words, so
-// three byte permutes gather its 16 codes into two words and the block's
-// 16-entry table (byte permutes, as in the fused GEMM) decodes them.  The
-// results go to shared memory by stmatrix in the 128-byte-swizzled layout of
-// a TMA tile and leave as one TMA store per warp (rows and columns past the
-// weight are not written).
-//
-// nf4_merge_kernel: one CTA per 128 x 128 tile, 8 warps; B^T and A slices
-// staged in shared memory (zero padded), each warp forms a 32 x 64 part of p
-// with ldmatrix + mma.sync, the whole tile of p is parked in shared memory,
-// and the epilogue walks each row in 8-column pieces of element loads and
-// stores.
+// Two kernels.  nf4_merge_tc_kernel takes the common shapes (K a multiple of
+// 64, so every NF4 block lies in one row; N and r multiples of 8, so rows of
+// A and B can be TMA boxes): p on the tensor cores (tcgen05) and one row of
+// the tile per thread in the epilogue; see the kernel.  nf4_merge_kernel
+// takes every other shape: one CTA per 128 x 128 tile, 8 warps; B^T and A
+// slices staged in shared memory (zero padded), each warp forms a 32 x 64
+// part of p with ldmatrix + mma.sync, the whole tile of p is parked in
+// shared memory, and the epilogue walks each row in 8-column pieces of
+// element loads and stores.
 #include <cstdint>
+#include <cstring>
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
 #include "common.cuh"
@@ -275,181 +263,177 @@ __global__ void __launch_bounds__(kMergeThreads, 3) nf4_merge_kernel(const __gri
   }
 }
 
-// ---------------------------------------------------------------------------
-// nf4_merge_frag_kernel
-constexpr int kFragThreads = 128;
-constexpr int kFragRows = 64;           // rows of W per CTA
-constexpr int kFragCols = 128;          // columns of W per CTA (two NF4 blocks per row)
-constexpr int kFragStage = 4 * 4096;    // per warp a 32-row x 128-byte swizzled TMA tile
-constexpr int kFragBRow = kFragRows * 2 + 16;   // bytes per staged B row (ldmatrix conflict-free)
-constexpr int kFragPkRow = 80;          // bytes per staged row of packed codes (64 + 16)
-
-struct MergeFragParams {
-  MergeArgs a;
-  CodeTable code;
-  ShiftMuls km;
-  CUtensorMap tm_out;                   // out [N x K], 2-byte elements, box {64, 32}, 128-byte swizzle
-  int rp;                               // r rounded up to 16
-  uint32_t a_chunks;                    // 16-byte chunks per staged A row (rp / 8)
-  uint32_t a_magic;                     // ceil(2^32 / a_chunks): exact quotients for indices < 2^16
-  int64_t ktiles;                       // column tiles per row of tiles
-};
-
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(bytes) : "memory");
-}
+// ---------------------------------------------------------------------------
+// nf4_merge_tc_kernel: p on the tensor cores (tcgen05, accumulator in tensor
+// memory), the epilogue one row per thread.
+//
+// One CTA per 128 (rows of W) x 128 (columns) tile, 4 warps.  One thread
+// loads by TMA, per 64 ranks, the B slice as two rank-major boxes [64 ranks x
+// 64 rows of W] (the MMA's A operand, MN-major) and the A slice [128 columns
+// x 64 ranks] (its B operand, K-major), both with the 128-byte swizzle (ranks
+// past r read as zeros), and issues p[128 x 128] = B^T A^T as M128 N128 K16
+// MMAs into 128 tensor-memory columns.  Meanwhile every thread loads the
+// packed codes (64 bytes) and the two block constants of its row: warp w owns
+// tensor-memory lanes 32w .. 32w + 31, i.e. rows 32w + lane.  Per NF4 block a
+// thread then reads its row's 64 values of p (two 32-column loads), decodes
+// the block's 64 codes with its 16-entry table, forms round(fma(s, p, wd)),
+// and writes the 128-byte row piece into a 128-byte-swizzled TMA tile that
+// leaves as one TMA store per warp and block.  The waits are bounded: a lost
+// arrival leaves the output unspecified instead of hanging.
+constexpr int kTcThreads = 128;
+constexpr int kTcTile = 128;
+constexpr uint32_t kTcStage = 4 * 2 * 4096;   // per warp and block a 32-row x 128-byte tile
+constexpr uint32_t kTcChunk = 32768;          // per 64 ranks: B slice 2 x 8 KB, A slice 16 KB
 
-__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
-                                              uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void stsm_x4(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
-  asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(r0), "r"(r1),
-               "r"(r2), "r"(r3)
-               : "memory");
-}
-
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-  return v;
-}
+struct MergeTcParams {
+  MergeArgs a;
+  CodeTable code;
+  ShiftMuls km;
+  CUtensorMap tm_b;     // B [r x N], box {64 columns, 64 ranks}, 128-byte swizzle
+  CUtensorMap tm_a;     // A [K x r], box {64 ranks, 128 rows}, 128-byte swizzle
+  CUtensorMap tm_out;   // out [N x K], box {64, 32}, 128-byte swizzle
+  int nch;              // 64-rank chunks: ceil(r / 64)
+  int64_t ktiles;
+};
 
 template <bool F16>
-__global__ void __launch_bounds__(kFragThreads, 4) nf4_merge_frag_kernel(const __grid_constant__ MergeFragParams P) {
+__global__ void __launch_bounds__(kTcThreads, 1) nf4_merge_tc_kernel(const __grid_constant__ MergeTcParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const MergeArgs& a = P.a;
-  const int rp = P.rp;
-  const int a_row = rp * 2 + 16;                     // bytes per staged A row (ldmatrix conflict-free)
-  uint8_t* stage = smem;                             // 4 x 4 KB TMA tiles
-  uint8_t* bs = stage + kFragStage;                  // B slice [rp][64 columns of out's rows]
-  uint8_t* as = bs + rp * kFragBRow;                 // A slice [128 columns of W][rp]
-  uint8_t* pk = as + kFragCols * a_row;              // packed codes [64 rows][64 bytes]
+  uint8_t* stage = smem;
+  uint8_t* ops = smem + kTcStage;
+  uint64_t* full = reinterpret_cast<uint64_t*>(ops + P.nch * kTcChunk);
+  uint64_t* done = full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t nt_i = int64_t(blockIdx.x) / P.ktiles;
-  const int64_t n0 = nt_i * kFragRows;
-  const int64_t k0 = (int64_t(blockIdx.x) - nt_i * P.ktiles) * kFragCols;
+  const int64_t n0 = nt_i * kTcTile;
+  const int64_t k0 = (int64_t(blockIdx.x) - nt_i * P.ktiles) * kTcTile;
 
-  // ---- stage the B slice, the A slice and the packed codes (zero fill past
-  // r, N and K)
-  const uint32_t bs_u = smem_u32(bs), as_u = smem_u32(as), pk_u = smem_u32(pk);
-  for (int i = tid; i < rp * 8; i += kFragThreads) {         // B[j][n0 + 8c .. + 7]
-    const int j = i >> 3, c = i & 7;
-    const int64_t n = n0 + 8 * c;
-    const bool ok = j < a.r && n < a.N;
-    cp_async16(bs_u + j * kFragBRow + c * 16, ok ? a.B + int64_t(j) * a.N + n : a.B, ok ? 16u : 0u);
+  if (tid == 0) {
+    tma_prefetch_desc(&P.tm_b);
+    tma_prefetch_desc(&P.tm_a);
+    mbar_init(full, 1);
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
   }
-  for (int i = tid; i < kFragCols * int(P.a_chunks); i += kFragThreads) {   // A[k0 + row][8c .. 8c + 7]
-    const int row = int(__umulhi(uint32_t(i), P.a_magic));
-    const int c = i - row * int(P.a_chunks);
-    const int64_t k = k0 + row;
-    const bool ok = 8 * c < a.r && k < a.K;
-    cp_async16(as_u + row * a_row + c * 16, ok ? a.A + k * a.r + 8 * c : a.A, ok ? 16u : 0u);
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
   }
-  for (int i = tid; i < kFragRows * 4; i += kFragThreads) {   // row n0 + row, columns k0 + 32c .. + 31
-    const int row = i >> 2, c = i & 3;
-    const int64_t n = n0 + row, k = k0 + 32 * c;
-    const bool ok = n < a.N && k < a.K;
-    cp_async16(pk_u + row * kFragPkRow + c * 16, ok ? a.packed + ((n * a.K + k) >> 1) : a.packed, ok ? 16u : 0u);
-  }
-  asm volatile("cp.async.commit_group;" ::: "memory");
 
-  // ---- this thread's four block constants (rows g, g + 8 of each 16-row half)
-  const int wn = warp & 1, wk = warp >> 1;
-  const int g = lane >> 2, c = lane & 3;
-  const int64_t kb = k0 + wk * 64;                   // the warp's NF4 block column
+  // this thread's row: packed codes of both blocks and their constants,
+  // loaded while the operands arrive and the MMAs run
+  const int64_t n = n0 + warp * 32 + lane;
   const int64_t kblocks = a.K >> 6;
-  uint32_t q[4];
-  float s2[4];
+  uint4 pk[4];
+  uint32_t q[2];
+  float s2[2];
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int64_t n = n0 + wn * 32 + (u >> 1) * 16 + (u & 1) * 8 + g;
-    q[u] = 0u;
-    s2[u] = 0.0f;
-    if (n < a.N && kb < a.K) load_scale_parts(a.double_quant, a.c1, a.c2, n * kblocks + (kb >> 6), q[u], s2[u]);
+  for (int b = 0; b < 2; ++b) {
+    const int64_t k = k0 + 64 * b;
+    pk[2 * b] = pk[2 * b + 1] = make_uint4(0u, 0u, 0u, 0u);
+    q[b] = 0u;
+    s2[b] = 0.0f;
+    if (n < a.N && k < a.K) {
+      const uint4* src = reinterpret_cast<const uint4*>(a.packed + ((n * a.K + k) >> 1));
+      pk[2 * b] = __ldcs(src);
+      pk[2 * b + 1] = __ldcs(src + 1);
+      load_scale_parts(a.double_quant, a.c1, a.c2, n * kblocks + (k >> 6), q[b], s2[b]);
+    }
   }
-  asm volatile("cp.async.wait_all;" ::: "memory");
+  tc_fence_before();
   __syncthreads();
-  if (kb >= a.K || n0 + wn * 32 >= a.N) return;      // the warp's tile lies past the weight
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
 
-  const uint32_t st_u = smem_u32(stage + warp * 4096);
-  const uint32_t sel = uint32_t(c) | (uint32_t(c + 4) << 4);   // byte c of two words
-#pragma unroll 1
-  for (int mt = 0; mt < 2; ++mt) {
-    float acc[8][4];
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[nt][e] = 0.0f;
-    const int mrow = wn * 32 + mt * 16;              // first row of W (in the tile) of this half
-    for (int kk = 0; kk < rp / 16; ++kk) {
-      // A operand (rows of W x rank) from B stored rank-major: matrix i of
-      // the four is rank 8 (i >> 1) .. + 7 by rows 8 (i & 1) .. + 7
-      uint32_t af[4];
-      {
-        const int i = lane >> 3;
-        const int j = kk * 16 + (i >> 1) * 8 + (lane & 7);
-        ldsm_x4_trans(bs_u + j * kFragBRow + (mrow + (i & 1) * 8) * 2, af[0], af[1], af[2], af[3]);
+  if (warp == 0) {
+    if (elect_one()) {
+      const uint32_t bytes = uint32_t(P.nch) * kTcChunk;
+      mbar_arrive_expect_tx(full, bytes);
+      for (int ch = 0; ch < P.nch; ++ch) {
+        uint8_t* o = ops + ch * kTcChunk;
+        tma_load_2d(o, &P.tm_b, full, int32_t(n0), int32_t(64 * ch));
+        tma_load_2d(o + 8192, &P.tm_b, full, int32_t(n0 + 64), int32_t(64 * ch));
+        tma_load_2d(o + 16384, &P.tm_a, full, int32_t(64 * ch), int32_t(k0));
       }
-#pragma unroll
-      for (int np = 0; np < 4; ++np) {               // pairs of 8-column tiles
-        const int row = wk * 64 + np * 16 + (lane & 7) + ((lane >> 4) << 3);
-        const int col = kk * 16 + ((lane >> 3) & 1) * 8;
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(as_u + row * a_row + col * 2, b0, b1, b2, b3);
-        mma16816<F16>(acc[2 * np], af, b0, b1);
-        mma16816<F16>(acc[2 * np + 1], af, b2, b3);
+      const bool ok = mbar_wait(full, 0u, nullptr, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        const uint32_t idesc = make_idesc(128, 128, 1, 0, F16);
+        for (int ch = 0; ch < P.nch; ++ch) {
+          const uint32_t o = smem_u32(ops + ch * kTcChunk);
+          mma_ss_k64(tmem_base, make_sdesc_sw128(o, 8192, 1024), 128u, make_sdesc_sw128(o + 16384, 16, 1024), 2u,
+                     idesc, ch > 0 ? 1u : 0u);
+        }
+      }
+      mma_commit(done);   // arrives once the MMAs above are complete (at once if none)
+      if (!ok) {          // let the loads land before the CTA exits
+        const long long t0 = clock64();
+        while (!mbar_try_wait(full, 0u) && clock64() - t0 < 200000000ll) {
+        }
       }
     }
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int row = mrow + h * 8 + g;
-      const uint32_t qu = mt ? q[2 + h] : q[h];   // selects: the arrays stay in registers
-      const float s2u = mt ? s2[2 + h] : s2[h];
-      const BlockTable t = make_table(P.code, scale_from_parts(a.double_quant, qu, s2u), F16);
-      const uint32_t src = pk_u + row * kFragPkRow + wk * 32;
-      const uint4 lo = lds128(src), hi = lds128(src + 16);
-      // byte c of each of the block's eight words: columns 8 nt + 2c, + 1
-      const uint32_t w0 = prmt(prmt(lo.x, lo.y, sel), prmt(lo.z, lo.w, sel), 0x5410u);
-      const uint32_t w1 = prmt(prmt(hi.x, hi.y, sel), prmt(hi.z, hi.w, sel), 0x5410u);
-      uint32_t o[8];
-      lookup8(t, w0, P.km, o[0], o[1], o[2], o[3]);
-      lookup8(t, w1, P.km, o[4], o[5], o[6], o[7]);
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
-        o[nt] = pack2(F16, fmaf(a.s, acc[nt][2 * h], half_lo_to_f32(F16, o[nt])),
-                      fmaf(a.s, acc[nt][2 * h + 1], half_hi_to_f32(F16, o[nt])));
-      // rows mt 16 + h 8 + 0..7 of the warp's tile; 16-byte chunk nt of a row
-      // sits at chunk nt ^ (row & 7) (128-byte swizzle)
-      const uint32_t lrow = uint32_t(mt * 16 + h * 8 + (lane & 7));
-      const uint32_t rbase = st_u + lrow * 128u;
-      const uint32_t ch = uint32_t(lane >> 3);
-      stsm_x4(rbase + ((ch ^ (lrow & 7u)) << 4), o[0], o[1], o[2], o[3]);
-      stsm_x4(rbase + (((ch + 4u) ^ (lrow & 7u)) << 4), o[4], o[5], o[6], o[7]);
-    }
+    __syncwarp();
   }
-  fence_proxy_async_smem();   // generic-proxy writes, read next by the TMA engine
-  __syncwarp();
-  if (lane == 0) {
-    tma_store_2d(&P.tm_out, stage + warp * 4096, int32_t(kb), int32_t(n0 + wn * 32));
-    bulk_commit();
-    bulk_wait_all();
+
+  // warp-uniform: the tensor-memory loads below are collective
+  const bool ok = __all_sync(0xffffffffu, mbar_wait(done, 0u, nullptr, abort_flag) && !*abort_flag);
+  tc_fence_after();
+  if (ok && n0 + warp * 32 < a.N) {
+    const uint32_t taddr = tmem_base + (uint32_t(warp * 32) << 16);
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      if (k0 + 64 * b >= a.K) break;
+      const BlockTable t = make_table(P.code, scale_from_parts(a.double_quant, q[b], s2[b]), F16);
+      uint8_t* tile = stage + (warp * 2 + b) * 4096;
+      const uint32_t row = smem_u32(tile) + uint32_t(lane) * 128u;
+      const uint32_t w[8] = {pk[2 * b].x, pk[2 * b].y, pk[2 * b].z, pk[2 * b].w,
+                             pk[2 * b + 1].x, pk[2 * b + 1].y, pk[2 * b + 1].z, pk[2 * b + 1].w};
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(taddr + uint32_t(64 * b + 32 * h), v);   // columns 64b + 32h .. + 31 of p
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {   // word 4h + i: columns 8 (4h + i) .. + 7
+          uint32_t o[4];
+          lookup8(t, w[4 * h + i], P.km, o[0], o[1], o[2], o[3]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            o[e] = pack2(F16, fmaf(a.s, __uint_as_float(v[8 * i + 2 * e]), half_lo_to_f32(F16, o[e])),
+                         fmaf(a.s, __uint_as_float(v[8 * i + 2 * e + 1]), half_hi_to_f32(F16, o[e])));
+          const uint32_t chunk = uint32_t(4 * h + i) ^ uint32_t(lane & 7);
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(row + (chunk << 4)), "r"(o[0]), "r"(o[1]),
+                       "r"(o[2]), "r"(o[3])
+                       : "memory");
+        }
+      }
+      fence_proxy_async_smem();   // generic-proxy writes, read next by the TMA engine
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(&P.tm_out, tile, int32_t(k0 + 64 * b), int32_t(n0 + warp * 32));
+        bulk_commit();
+      }
+    }
+    if (lane == 0) bulk_wait_all();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 128);
   }
 }
 
-size_t merge_frag_smem_bytes(int rp) {
-  return 1024 + size_t(kFragStage) + size_t(rp) * kFragBRow + size_t(kFragCols) * (rp * 2 + 16) +
-         size_t(kFragRows) * kFragPkRow;
-}
+size_t merge_tc_smem_bytes(int nch) { return 1024 + size_t(kTcStage) + size_t(nch) * kTcChunk + 32; }
 
 }  // namespace
 
@@ -461,26 +445,28 @@ size_t merge_smem_bytes(int r) {
 }
 
 cudaError_t launch_merge(const MergeArgs& a, const float code[16], cudaStream_t stream) {
-  const int64_t ktiles = (a.K + kFragCols - 1) / kFragCols;
-  const int64_t tiles = ktiles * ((a.N + kFragRows - 1) / kFragRows);
+  const int64_t tc_ktiles = (a.K + kTcTile - 1) / kTcTile;
+  const int64_t tc_tiles = tc_ktiles * ((a.N + kTcTile - 1) / kTcTile);
   if (a.K % 64 == 0 && a.N % 8 == 0 && a.r % 8 == 0 && a.K < (int64_t(1) << 31) && a.N < (int64_t(1) << 31) &&
-      tiles < (int64_t(1) << 31)) {
-    MergeFragParams P;
+      tc_tiles < (int64_t(1) << 31)) {
+    MergeTcParams P;
+    memset(&P, 0, sizeof(P));
     P.a = a;
     for (int i = 0; i < 16; ++i) P.code.v[i] = code[i];
     P.km = make_shift_muls();
-    P.rp = (a.r + 15) / 16 * 16;
-    P.a_chunks = uint32_t(P.rp / 8);
-    P.a_magic = uint32_t(((uint64_t(1) << 32) + P.a_chunks - 1) / P.a_chunks);
-    P.ktiles = ktiles;
-    if (!encode_tmap_2d(&P.tm_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.out, uint64_t(a.K), uint64_t(a.N),
-                        uint64_t(a.K) * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B))
-      return cudaErrorInvalidValue;
-    const size_t smem = merge_frag_smem_bytes(P.rp);
-    void (*kern)(const MergeFragParams) = a.f16 ? nf4_merge_frag_kernel<true> : nf4_merge_frag_kernel<false>;
+    P.nch = (a.r + 63) / 64;
+    P.ktiles = tc_ktiles;
+    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;   // 2-byte elements (bf16 or fp16)
+    const auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
+    bool ok = encode_tmap_2d(&P.tm_b, BF, a.B, uint64_t(a.N), uint64_t(a.r), uint64_t(a.N) * 2, 64, 64, SW);
+    ok &= encode_tmap_2d(&P.tm_a, BF, a.A, uint64_t(a.r), uint64_t(a.K), uint64_t(a.r) * 2, 64, 128, SW);
+    ok &= encode_tmap_2d(&P.tm_out, BF, a.out, uint64_t(a.K), uint64_t(a.N), uint64_t(a.K) * 2, 64, 32, SW);
+    if (!ok) return cudaErrorInvalidValue;
+    const size_t smem = merge_tc_smem_bytes(P.nch);
+    void (*kern)(const MergeTcParams) = a.f16 ? nf4_merge_tc_kernel<true> : nf4_merge_tc_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
-    kern<<<unsigned(tiles), kFragThreads, smem, stream>>>(P);
+    kern<<<unsigned(tc_tiles), kTcThreads, smem, stream>>>(P);
     return cudaGetLastError();
   }
   MergeParams P;

@@ -131,7 +131,8 @@ def test_merge_bf16(cfg):
 
 
 @pytest.mark.parametrize("qt,dq", [(0, 0), (1, 1), (0, 2)])
-@pytest.mark.parametrize("N,K,r,s", [(1024, 1024, 16, 1.0), (520, 640, 72, 0.5), (13, 100, 3, 2.0)])
+@pytest.mark.parametrize("N,K,r,s", [(1024, 1024, 16, 1.0), (520, 640, 72, 0.5), (136, 576, 8, 1.5),
+                                     (13, 100, 3, 2.0)])
 def test_merge_f16_and_formats(qt, dq, N, K, r, s):
     W = workloads.weight(N, K, 0.02, seed=N + r, device=DEV)
     io = workloads.layer_inputs(1, N, K, r, seed=N + r, device=DEV)
