@@ -951,11 +951,17 @@ SkinnyPlan plan_skinny(int kind, int64_t M, int64_t N, int64_t K, int /*r*/, int
   }
   p.tiles = cdiv(p.rows, 128);
   p.splits = choose_splits(p.tiles, p.steps, 2 * num_sms, 2, (2 * num_sms * 7) / 8);
-  // dA and dB run while the dX GEMM's last wave still holds most SMs: a few
-  // longer CTAs in pairs place sooner on the SMs it leaves idle than
-  // clusters of 8 short ones (the 4096 x 4096 backward at 2048 tokens: 98
-  // instead of 106 us)
-  if ((kind == kSkinnyDA || kind == kSkinnyDB) && p.splits > 2) p.splits = 2;
+  // Beside a fused GEMM (more than 16 tokens) the rank-r kernels share the
+  // SMs with it, and few long CTAs serve it better than clusters of short
+  // ones: T and G run beside its first wave, which their CTAs would keep off
+  // the SMs, so they split at most 2 ways; dA and dB run beside its last
+  // wave on the few SMs it leaves idle, unsplit.  At 2048 tokens this took
+  // the 4096 x 4096 forward from 82 to 73 us and the backward from 106 to
+  // 86-89 us.  (1-16 tokens: T runs beside the decode kernel, unchanged.)
+  if (M > 16) {
+    const int cap = (kind == kSkinnyDA || kind == kSkinnyDB) ? 1 : 2;
+    if (p.splits > cap) p.splits = cap;
+  }
   return p;
 }
 
