@@ -952,14 +952,23 @@ SkinnyPlan plan_skinny(int kind, int64_t M, int64_t N, int64_t K, int /*r*/, int
   p.tiles = cdiv(p.rows, 128);
   p.splits = choose_splits(p.tiles, p.steps, 2 * num_sms, 2, (2 * num_sms * 7) / 8);
   // Beside a fused GEMM (more than 16 tokens) the rank-r kernels share the
-  // SMs with it, and few long CTAs serve it better than clusters of short
-  // ones: T and G run beside its first wave, which their CTAs would keep off
-  // the SMs, so they split at most 2 ways; dA and dB run beside its last
-  // wave on the few SMs it leaves idle, unsplit.  At 2048 tokens this took
-  // the 4096 x 4096 forward from 82 to 73 us and the backward from 106 to
-  // 86-89 us.  (1-16 tokens: T runs beside the decode kernel, unchanged.)
+  // SMs with it, and fewer, longer CTAs serve it better than clusters of
+  // short ones.  T runs beside the forward GEMM's first wave, which its CTAs
+  // would keep off the SMs: at most 2 ways, or as many as keep each partial
+  // sum within 64 steps (4096 terms, so that the fp32 sums that T's bf16
+  // rounding sees stay as accurate as before).  dA and dB run beside the dX
+  // GEMM's last wave on the few SMs it leaves idle: unsplit.  G keeps its
+  // split: dA starts only once G is complete.  At 2048 tokens this took the
+  // 4096 x 4096 forward from 82 to 70 us and the backward from 106 to 84 us.
+  // (1-16 tokens: T runs beside the decode kernel, unchanged.)
   if (M > 16) {
-    const int cap = (kind == kSkinnyDA || kind == kSkinnyDB) ? 1 : 2;
+    int cap = 8;
+    if (kind == kSkinnyT) {
+      const int64_t need = cdiv(p.steps, 64);
+      cap = need <= 2 ? 2 : (need <= 4 ? 4 : 8);
+    } else if (kind == kSkinnyDA || kind == kSkinnyDB) {
+      cap = 1;
+    }
     if (p.splits > cap) p.splits = cap;
   }
   return p;
