@@ -954,18 +954,19 @@ SkinnyPlan plan_skinny(int kind, int64_t M, int64_t N, int64_t K, int /*r*/, int
   // Beside a fused GEMM (more than 16 tokens) the rank-r kernels share the
   // SMs with it, and fewer, longer CTAs serve it better than clusters of
   // short ones.  T runs beside the forward GEMM's first wave, which its CTAs
-  // would keep off the SMs: at most 2 ways, or as many as keep each partial
-  // sum within 64 steps (4096 terms, so that the fp32 sums that T's bf16
-  // rounding sees stay as accurate as before).  dA and dB run beside the dX
-  // GEMM's last wave on the few SMs it leaves idle: unsplit.  G keeps its
+  // would keep off the SMs: at most 2 ways while each partial sum stays
+  // within 128 steps (8192 terms); a longer reduction keeps its split, so
+  // that the fp32 sums that T's bf16 rounding sees stay accurate (4 ways
+  // measured slower than 2 or 8 on the 4096 x 11008 forward).  dA and dB
+  // run beside the dX GEMM's last wave on the few SMs it leaves idle:
+  // unsplit.  G keeps its
   // split: dA starts only once G is complete.  At 2048 tokens this took the
   // 4096 x 4096 forward from 82 to 70 us and the backward from 106 to 84 us.
   // (1-16 tokens: T runs beside the decode kernel, unchanged.)
   if (M > 16) {
     int cap = 8;
     if (kind == kSkinnyT) {
-      const int64_t need = cdiv(p.steps, 64);
-      cap = need <= 2 ? 2 : (need <= 4 ? 4 : 8);
+      cap = cdiv(p.steps, 2) <= 128 ? 2 : 8;
     } else if (kind == kSkinnyDA || kind == kSkinnyDB) {
       cap = 1;
     }

@@ -81,9 +81,8 @@ def check_plan(M, N, K, r, backward, sms):
         assert s in (1, 2, 4, 8)
         if M > 16 and kind >= 2:   # beside the dX GEMM's last wave: dA and dB unsplit
             assert s == 1, (kind, s)
-        if M > 16 and kind == 0:   # T: at most 2 ways unless a partial would pass 64 steps
-            steps = LOWRANK_STEPS[0](M, N, K)
-            assert s <= max(2, 1 << (cdiv(steps, 64) - 1).bit_length()), (s, steps)
+        if M > 16 and kind == 0 and cdiv(LOWRANK_STEPS[0](M, N, K), 2) <= 128:
+            assert s <= 2, s   # T: at most 2 ways while a partial stays within 128 steps
         if s > 1:
             assert nonempty(LOWRANK_STEPS[kind](M, N, K), s), (kind, s)
     return p
