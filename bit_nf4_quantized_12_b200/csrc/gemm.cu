@@ -951,26 +951,26 @@ SkinnyPlan plan_skinny(int kind, int64_t M, int64_t N, int64_t K, int /*r*/, int
   }
   p.tiles = cdiv(p.rows, 128);
   p.splits = choose_splits(p.tiles, p.steps, 2 * num_sms, 2, (2 * num_sms * 7) / 8);
-  // Beside a fused GEMM (more than 16 tokens) the rank-r kernels share the
-  // SMs with it, and fewer, longer CTAs serve it better than clusters of
-  // short ones.  T runs beside the forward GEMM's first wave, which its CTAs
-  // would keep off the SMs: at most 2 ways while each partial sum stays
-  // within 128 steps (8192 terms); a longer reduction keeps its split, so
-  // that the fp32 sums that T's bf16 rounding sees stay accurate (4 ways
-  // measured slower than 2 or 8 on the 4096 x 11008 forward).  dA and dB
-  // run beside the dX GEMM's last wave on the few SMs it leaves idle:
-  // unsplit.  G keeps its
-  // split: dA starts only once G is complete.  At 2048 tokens this took the
-  // 4096 x 4096 forward from 82 to 70 us and the backward from 106 to 84 us.
-  // (1-16 tokens: T runs beside the decode kernel, unchanged.)
-  if (M > 16) {
-    int cap = 8;
-    if (kind == kSkinnyT) {
-      cap = cdiv(p.steps, 2) <= 128 ? 2 : 8;
-    } else if (kind == kSkinnyDA || kind == kSkinnyDB) {
-      cap = 1;
+  // Beside a fused GEMM whose tiles fill the SMs without a split (more than
+  // 16 tokens), the rank-r kernels compete with it for SMs, and fewer,
+  // longer CTAs serve it better than clusters of short ones.  T runs beside
+  // the forward GEMM's first wave, which its CTAs would keep off the SMs: at
+  // most 2 ways while each partial sum stays within 128 steps (8192 terms);
+  // a longer reduction keeps its split, so that the fp32 sums that T's bf16
+  // rounding sees stay accurate (4 ways measured slower than 2 or 8 on the
+  // 4096 x 11008 forward).  dA and dB run beside the dX GEMM's last wave on
+  // the few SMs it leaves idle: unsplit.  G keeps its split: dA starts only
+  // once G is complete.  At 2048 tokens this took the 4096 x 4096 forward
+  // from 82 to 70 us and the backward from 106 to 84 us.  A GEMM with fewer
+  // tiles than SMs is short and splits its own reduction; T must then finish
+  // early, and every kernel keeps its split.  (1-16 tokens: T runs beside
+  // the decode kernel, unchanged.)
+  if (M > 16 && kind != kSkinnyG) {
+    const bool bwd = kind != kSkinnyT;
+    if (plan_nf4_gemm(bwd ? 1 : 0, M, N, K, 64, num_sms).splits == 1) {
+      const int cap = bwd ? 1 : (cdiv(p.steps, 2) <= 128 ? 2 : 8);
+      if (p.splits > cap) p.splits = cap;
     }
-    if (p.splits > cap) p.splits = cap;
   }
   return p;
 }

@@ -79,10 +79,13 @@ def check_plan(M, N, K, r, backward, sms):
             assert s == 0
             continue
         assert s in (1, 2, 4, 8)
-        if M > 16 and kind >= 2:   # beside the dX GEMM's last wave: dA and dB unsplit
+        # beside a fused GEMM that fills the SMs unsplit: dA and dB unsplit, T at
+        # most 2 ways while a partial stays within 128 steps
+        fills = M > 16 and binding.plan(M, N, K, 64, backward=kind != 0, num_sms=sms)["splits"] == 1
+        if fills and kind >= 2:
             assert s == 1, (kind, s)
-        if M > 16 and kind == 0 and cdiv(LOWRANK_STEPS[0](M, N, K), 2) <= 128:
-            assert s <= 2, s   # T: at most 2 ways while a partial stays within 128 steps
+        if fills and kind == 0 and cdiv(LOWRANK_STEPS[0](M, N, K), 2) <= 128:
+            assert s <= 2, s
         if s > 1:
             assert nonempty(LOWRANK_STEPS[kind](M, N, K), s), (kind, s)
     return p
