@@ -148,7 +148,10 @@ nf4_status nf4_dequant(nf4_weight w, int32_t dtype, uint16_t* out, void* stream)
  *   out = round(Wd + s (A B)^T),  Wd = nf4_dequant(w, dtype),
  * A [K, r], B [r, N], out [N, K] (device, compute type dtype).  Arithmetic:
  * Wd as in nf4_dequant; p = sum_j A[k,j] B[j,n] accumulated in fp32 (exact
- * products, order unspecified); out = round(fma(s, p, Wd)).  1 <= r <= 256. */
+ * products, order unspecified); out = round(fma(s, p, Wd)).  1 <= r <= 256.
+ * For K % 64 == 0 with N and r multiples of 8 the product runs on the tensor
+ * cores behind bounded waits; there is no status word, so a wait that gave
+ * up (a lost arrival, not seen in practice) would leave out unspecified. */
 nf4_status nf4_lora_merge(nf4_weight w, const uint16_t* A, const uint16_t* B, int32_t r, float s, int32_t dtype,
                           uint16_t* out, void* stream);
 
