@@ -959,16 +959,21 @@ SkinnyPlan plan_skinny(int kind, int64_t M, int64_t N, int64_t K, int /*r*/, int
   // a longer reduction keeps its split, so that the fp32 sums that T's bf16
   // rounding sees stay accurate (4 ways measured slower than 2 or 8 on the
   // 4096 x 11008 forward).  dA and dB run beside the dX GEMM's last wave on
-  // the few SMs it leaves idle: unsplit.  G keeps its split: dA starts only
-  // once G is complete.  At 2048 tokens this took the 4096 x 4096 forward
-  // from 82 to 70 us and the backward from 106 to 84 us.  A GEMM with fewer
-  // tiles than SMs is short and splits its own reduction; T must then finish
-  // early, and every kernel keeps its split.  (1-16 tokens: T runs beside
-  // the decode kernel, unchanged.)
-  if (M > 16 && kind != kSkinnyG) {
+  // the few SMs it leaves idle: unsplit.  G keeps its split (dA starts only
+  // once G is complete) unless the dX GEMM runs in less than one wave: then
+  // G's CTAs must fit in the SMs the GEMM leaves idle, 2 ways at most (the
+  // 70B gate backward at 512 tokens: 228 instead of 274 us).  At 2048
+  // tokens this took the 4096 x 4096 forward from 82 to 70 us and the
+  // backward from 106 to 84 us.  A GEMM that splits its own reduction is
+  // short, T must then finish early, and every kernel keeps its split.
+  // (1-16 tokens: T runs beside the decode kernel, unchanged.)
+  if (M > 16) {
     const bool bwd = kind != kSkinnyT;
-    if (plan_nf4_gemm(bwd ? 1 : 0, M, N, K, 64, num_sms).splits == 1) {
-      const int cap = bwd ? 1 : (cdiv(p.steps, 2) <= 128 ? 2 : 8);
+    const Nf4GemmPlan g = plan_nf4_gemm(bwd ? 1 : 0, M, N, K, 64, num_sms);
+    if (g.splits == 1) {
+      int cap = 1;
+      if (kind == kSkinnyT) cap = cdiv(p.steps, 2) <= 128 ? 2 : 8;
+      if (kind == kSkinnyG) cap = g.tiles_w * g.tiles_t < num_sms ? 2 : 8;
       if (p.splits > cap) p.splits = cap;
     }
   }

@@ -81,9 +81,12 @@ def check_plan(M, N, K, r, backward, sms):
         assert s in (1, 2, 4, 8)
         # beside a fused GEMM that fills the SMs unsplit: dA and dB unsplit, T at
         # most 2 ways while a partial stays within 128 steps
-        fills = M > 16 and binding.plan(M, N, K, 64, backward=kind != 0, num_sms=sms)["splits"] == 1
+        gp = binding.plan(M, N, K, 64, backward=kind != 0, num_sms=sms)
+        fills = M > 16 and gp["splits"] == 1
         if fills and kind >= 2:
             assert s == 1, (kind, s)
+        if fills and kind == 1 and gp["tiles_w"] * gp["tiles_t"] < sms:
+            assert s <= 2, s   # G beside a dX GEMM of less than one wave
         if fills and kind == 0 and cdiv(LOWRANK_STEPS[0](M, N, K), 2) <= 128:
             assert s <= 2, s
         if s > 1:
