@@ -1,5 +1,5 @@
 """GPU parity of the QLoRA linear layer (forward, backward, decode shapes)
-against the float64 oracle, with the tolerance the build states:
+against the float64 oracle, with the layer's stated tolerance:
 relative Frobenius <= 2e-3, elementwise relative <= 1e-2 (denominator
 floored at 1e-2 x rms of the reference)."""
 import numpy as np

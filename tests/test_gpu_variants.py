@@ -10,7 +10,7 @@ LoRA merge against the oracle.
     value cancels to far below its inputs; every such element must lie within
     that arithmetic's error bound of the exact value, and they must be rare;
   - the QLoRA linear layer in FP16, and in bf16 on the variant formats,
-    within the build's GEMM tolerance (relative Frobenius 2e-3, elementwise
+    within the linear layer's stated tolerance (relative Frobenius 2e-3, elementwise
     1e-2 with the denominator floored at 1e-2 x rms)."""
 import numpy as np
 import pytest
